@@ -1,0 +1,16 @@
+"""CPU oracle for the sparse decode path (test infrastructure only).
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py``'s CPU-baseline and
+reference legs import this package; the library never does.
+"""
+from .sd_oracle import (  # noqa: F401
+    attend_rows,
+    bf16_bits_to_f64,
+    decode_step,
+    dense_attention,
+    gather_token_rows,
+    indexer_scores,
+    sparse_attention,
+    topk_indices,
+    topk_row,
+)

@@ -1,0 +1,337 @@
+"""Benchmark of one sparse decode step (indexer -> top-k -> sparse attention).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl ours|reference]
+
+Prints ONE JSON line (rank 0). A step is ``sd_decode_step`` over one synthetic
+batch of the named workload (default: 32 requests x 65536 cached tokens, MLA
+latent rows shared by 128 heads, top-k 2048). Inputs are resident in HBM; L2 is
+flushed (a 256 MiB write) before every step, outside the timed events. With
+N > 1 (torchrun) each rank runs its own batch (different seed): the path shards
+by request with no collective, so the scaling is weak and the value is the
+total queries/s of all ranks over the slowest rank's time.
+
+``--impl reference`` times the CPU oracle (the only reference this path has)
+on a bounded sample of the same workload, on rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from top_sparse_decode_paged_b200 import workloads as W  # noqa: E402
+
+METRIC = "decode queries/s and achieved HBM GB/s (indexer+top-k+sparse attn), 1 B200"
+DEFAULT_CONFIG = "b32_l65536_mla"
+L2_FLUSH_BYTES = 256 << 20
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+def _dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def rank_spec(name: str, rank: int) -> W.Spec:
+    """Each rank draws its own batch of the same shape (weak scaling)."""
+    base = W.spec(name)
+    return W.spec(name, seed=base.seed + 1000 * rank) if rank else base
+
+
+def max_over_ranks(value: float, world: int) -> float:
+    """Slowest rank's time (all ranks take this collective in the same order)."""
+    if world == 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([value], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+class ClockSampler:
+    """Samples nvidia-smi clocks and throttle reasons while the timed region runs."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.rows = []
+        self._stop = threading.Event()
+        self._t = None
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                out = subprocess.run(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                                      "--format=csv,noheader,nounits"], capture_output=True, text=True,
+                                     timeout=5).stdout.strip()
+                if out:
+                    self.rows.append([x.strip() for x in out.split(",")])
+            except Exception:
+                pass
+            self._stop.wait(0.1)
+
+    def __enter__(self):
+        self._t = threading.Thread(target=self._run, daemon=True)
+        self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        self._t.join(timeout=10)
+
+    def summary(self):
+        if not self.rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        sm = [float(r[0]) for r in self.rows if r[0].replace(".", "").isdigit()]
+        mx = [float(r[1]) for r in self.rows if r[1].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in self.rows for i in range(4) if r[3 + i] == "Active"})
+        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(self.rows)}
+
+
+def run_oracle_sample(wl, n_req: int):
+    """Times the CPU oracle on the first n_req requests of the batch."""
+    import oracle
+    t0 = time.perf_counter()
+    oracle.decode_step(wl, requests=list(range(n_req)))
+    return time.perf_counter() - t0
+
+
+def _blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info()]
+        return max(n) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def cpu_baseline(name: str, budget_s: float = 15.0):
+    """The oracle as it stands on a bounded sample: requests are added until the
+    sample has taken about budget_s seconds of host time."""
+    wl = W.make(W.spec(name))
+    done, spent = 0, 0.0
+    while done < wl.seqlens.shape[0] and spent < budget_s:
+        t0 = time.perf_counter()
+        import oracle
+        oracle.decode_step(wl, requests=[done])
+        spent += time.perf_counter() - t0
+        done += 1
+    return {"value": done / spent, "unit": "queries/s", "cores": _blas_threads(), "kind": "oracle",
+            "sample": f"{done} of {wl.seqlens.shape[0]} requests of {name}, {spent:.1f} s host time"}
+
+
+def bench_reference(args, rank, world):
+    if rank != 0:
+        return
+    n_steps = args.steps
+    wl = W.make(W.spec(args.config))
+    times = []
+    per_step = max(1, min(wl.seqlens.shape[0], 2))
+    for i in range(args.warmup + n_steps):
+        t = run_oracle_sample(wl, per_step)
+        if i >= args.warmup:
+            times.append(t)
+    ms = 1e3 * float(np.mean(times)) / per_step * wl.seqlens.shape[0]
+    value = per_step / float(np.mean(times))
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "queries/s", "n_gpus": world,
+        "steps": n_steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "int64/f64", "data": "synthetic",
+        "config": _config(wl.spec, "host memory (CPU oracle)"),
+        "cpu_baseline": {"value": value, "unit": "queries/s", "cores": _blas_threads(), "kind": "oracle",
+                         "sample": f"{per_step} requests per step of {args.config}"},
+        "e2e": {"value": value, "unit": "queries/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def _config(s: W.Spec, l2: str):
+    cfg = {"workload": s.name, "B": s.B, "page": s.page_size, "kv_heads": s.G, "Hi": s.Hi, "Di": s.Di,
+           "k": s.k, "H": s.H, "Dk": s.Dk, "Dv": s.Dv, "l2": l2}
+    if s.seqlen is not None:
+        cfg["seqlen"] = s.seqlen
+    if s.ragged is not None:
+        cfg["seqlen_loguniform"] = list(s.ragged)
+    return cfg
+
+
+def bench_ours(args, rank, world, local):
+    import torch
+    import top_sparse_decode_paged_b200 as sd
+    from top_sparse_decode_paged_b200.api import StageTimer
+
+    torch.cuda.set_device(local)
+    spec = rank_spec(args.config, rank)
+    wl = W.make(spec)
+    s = wl.spec
+    dev = "cuda"
+    t = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(dev)  # noqa: E731
+    qi, w, ki = t(wl.qi), t(wl.w), t(wl.ki_pages)
+    bt, sl = t(wl.block_table), t(wl.seqlens)
+    q = t(wl.q.view(np.int16)).view(torch.bfloat16)
+    kp = t(wl.k_pages.view(np.int16)).view(torch.bfloat16)
+    vp = None if wl.v_pages is None else t(wl.v_pages.view(np.int16)).view(torch.bfloat16)
+    B, G = wl.seqlens.shape[0], s.G
+    Lmax = wl.max_seqlen
+    idx = torch.empty((B, G, s.k), dtype=torch.int32, device=dev)
+    out = torch.empty((B, s.H, s.Dv), dtype=torch.bfloat16, device=dev)
+    ws = sd.alloc_workspace(B, G, Lmax, s.k, s.H, s.Dv)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        sd.sd_decode_step(qi, w, ki, q, kp, vp, bt, sl, s.k, Lmax, s.scale, s.Dv,
+                          indices=idx, out=out, workspace=ws)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    launches_per_step = sd.last_launch_count()
+    torch.cuda.synchronize()
+
+    timer = StageTimer()
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local if "CUDA_VISIBLE_DEVICES" not in os.environ else int(
+            os.environ["CUDA_VISIBLE_DEVICES"].split(",")[local])) as clocks:
+        for i in range(args.steps):
+            flush.zero_()
+            timer.arm()
+            starts[i].record(stream)
+            step()
+            ends[i].record(stream)
+        torch.cuda.synchronize()
+        StageTimer.disarm()
+        if world > 1:
+            dist.barrier()
+    step_ms = sum(a.elapsed_time(b) for a, b in zip(starts, ends)) / args.steps
+    stage_tot, n_rec = timer.totals_ms()
+    stage_ms = {k_: v / n_rec for k_, v in stage_tot.items()}
+    step_ms = max_over_ranks(step_ms, world)
+
+    # end to end through the public call: per-step queries H2D from pinned
+    # host memory, the step, and the result (indices + output) D2H
+    h_qi = torch.from_numpy(wl.qi).pin_memory()
+    h_w = torch.from_numpy(wl.w).pin_memory()
+    h_q = torch.from_numpy(wl.q.view(np.int16)).pin_memory()
+    h_bt = torch.from_numpy(wl.block_table).pin_memory()
+    h_sl = torch.from_numpy(wl.seqlens).pin_memory()
+    h_idx = torch.empty((B, G, s.k), dtype=torch.int32).pin_memory()
+    h_out = torch.empty((B, s.H, s.Dv), dtype=torch.int16).pin_memory()
+    q16 = q.view(torch.int16)
+    h2d = sum(x.numel() * x.element_size() for x in (h_qi, h_w, h_q, h_bt, h_sl))
+    d2h = h_idx.numel() * 4 + h_out.numel() * 2
+    e_steps = max(3, min(args.steps, 50))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e_ms = 0.0
+    for i in range(e_steps):
+        flush.zero_()
+        e0.record(stream)
+        qi.copy_(h_qi, non_blocking=True)
+        w.copy_(h_w, non_blocking=True)
+        q16.copy_(h_q, non_blocking=True)
+        bt.copy_(h_bt, non_blocking=True)
+        sl.copy_(h_sl, non_blocking=True)
+        step()
+        h_idx.copy_(idx, non_blocking=True)
+        h_out.copy_(out.view(torch.int16), non_blocking=True)
+        e1.record(stream)
+        e1.synchronize()
+        e_ms += e0.elapsed_time(e1)
+    e_ms = max_over_ranks(e_ms / e_steps, world)
+
+    alg = W.algorithmic_bytes(s, wl.seqlens)
+    idx_bytes = int(np.sum(wl.seqlens.astype(np.int64))) * s.G * s.Di
+    peak, peak_kind = _peaks()
+    idx_gbs = idx_bytes / (stage_ms["indexer"] * 1e-3) / 1e9 if stage_ms["indexer"] > 0 else None
+    line = {
+        "metric": METRIC,
+        "value": world * B / (step_ms * 1e-3),
+        "unit": "queries/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": step_ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "int8/bf16", "data": "synthetic",
+        "config": _config(s, "flushed before every step (256 MiB write, outside the timed events)"),
+        "hbm_gbs_step": alg / (step_ms * 1e-3) / 1e9,
+        "hbm_frac_step": alg / (step_ms * 1e-3) / 1e9 / peak,
+        "algorithmic_bytes_per_step": alg,
+        "stage_ms": stage_ms,
+        "roofline": {"kernel": "indexer", "bound": "hbm", "achieved": idx_gbs, "peak": peak,
+                     "peak_kind": peak_kind, "unit": "GB/s",
+                     "frac": (idx_gbs / peak) if idx_gbs else None,
+                     "traffic": None, "algorithmic_bytes_per_launch": idx_bytes},
+        "e2e": {"value": world * B / (e_ms * 1e-3), "unit": "queries/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clocks.summary(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(args.config)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--config", default=DEFAULT_CONFIG, choices=list(W.SPECS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    rank, world, local = _dist_env()
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        if args.impl == "ours":
+            torch.cuda.set_device(local)
+        dist.init_process_group("nccl" if args.impl == "ours" else "gloo",
+                                timeout=datetime.timedelta(seconds=300))
+    try:
+        if args.impl == "reference":
+            bench_reference(args, rank, world)
+        else:
+            bench_ours(args, rank, world, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

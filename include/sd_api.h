@@ -1,0 +1,165 @@
+/*
+ * sd_api.h -- C ABI of the top-k sparse decode library for NVIDIA B200 (sm_100a).
+ *
+ * One decode step over a paged KV cache, for a batch of B requests with one
+ * query token each:
+ *
+ *   1. indexer score  s[b,g,t] = sum_h w[b,g,h] * max(0, sum_d qi[b,g,h,d] * ki[t,g,d])
+ *                     for every cached token t < seqlens[b], keys read in place
+ *                     from the paged indexer pool through the block table;
+ *   2. top-k          per (request, KV head) the min(k, seqlen) tokens of highest
+ *                     score, ties to the lower token index, written in ascending
+ *                     token order and padded with -1;
+ *   3. sparse attn    o[b,h] = sum_j softmax_j(scale * q[b,h] . K_j) V_j over the
+ *                     selected rows of KV head g = h / (H/G), gathered from the
+ *                     paged K/V pools, followed by a split combine.
+ *
+ * Where this comes from. The pages describe the DSA decode data flow: an
+ * indexer scores the cached tokens, a top-k kernel fills a persistent top-k
+ * buffer, and core sparse attention consumes it ("Overlap DSA heuristic
+ * prev_topk write-back on the aux stream", Description). Predicted indices are
+ * request-local token ids translated to pool rows through the block table, and
+ * negative entries are invalid ("Unify sparse attention framework with clean
+ * backend interfaces", review notes on DSA global index conversion). The golden
+ * reference attends over selected tokens of a logical cache rebuilt from
+ * pages ("Add DSA Vanilla sparse attention", Walkthrough). A typed, fixed
+ * signature beats a generic keyword carrier ("Compact pseudo-KV/topological
+ * sparse attention benchmark evidence", the 0.756x kwargs result). The pages
+ * never write the formulas out; the readings taken (ReLU per indexer head,
+ * integer head weights, lowest-index ties, ascending order) are stated in the
+ * design notes.
+ *
+ * Conventions for every call
+ *   - All array pointers are DEVICE pointers owned by the caller; the library
+ *     never allocates, frees or keeps them. Arrays are dense, row-major, with
+ *     the shapes given per argument. bf16 arrays are passed as raw uint16 bits.
+ *   - Pools are NHD: [num_pages, page_size, kv_heads, dim]. Token t of request
+ *     b lives at page block_table[b * max_pages_per_req + t / page_size],
+ *     slot t % page_size.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream). Every call only
+ *     enqueues work on it: no host synchronisation, no allocation, so a call can
+ *     be captured in a CUDA graph. Buffers keep the addresses the caller gives.
+ *   - `workspace` is caller-owned device scratch of at least the size that
+ *     sd_workspace_size() returns for the same shape (256-byte aligned).
+ *   - Argument errors are found on the host before any launch and returned as
+ *     a status; nothing is enqueued then. Errors in device-resident data (a
+ *     seqlen beyond the block table, a block-table entry outside the pool, an
+ *     index at or past seqlen) cannot be seen on the host: the kernels mask the
+ *     offending token (a bad indexer page scores INT32_MIN, a bad attention
+ *     row is skipped), clamp the length, and OR a bit into a sticky per-device
+ *     error word that sd_get_device_errors() reads.
+ *
+ * Supported shapes (others return SD_ERR_UNSUPPORTED):
+ *   indexer  Di in {32, 64, 128}, 1 <= Hi <= 64, G * Di <= 1024
+ *   top-k    1 <= k <= 2048, max_seqlen <= 1 << 20
+ *   attn     (Dk, Dv) in {(64, 64), (128, 128), (576, 512)}, H % G == 0,
+ *            H / G <= 128; with v_pages == NULL, V is the first Dv columns of
+ *            the K row (MLA latent rows, or MQA with V = K)
+ */
+#ifndef SD_API_H
+#define SD_API_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum sd_status {
+  SD_OK = 0,
+  SD_ERR_INVALID_ARG = 1,   /* null pointer, negative size, inconsistent shape */
+  SD_ERR_UNSUPPORTED = 2,   /* a valid shape this build has no kernel for      */
+  SD_ERR_WORKSPACE = 3,     /* workspace missing, too small or misaligned      */
+  SD_ERR_CUDA = 4           /* a CUDA runtime call failed (see sd_last_cuda_error) */
+} sd_status;
+
+/* Bits of the sticky per-device error word (sd_get_device_errors). */
+#define SD_DEVERR_SEQLEN 0x1u   /* seqlens[b] < 0, > max_seqlen or > the block table  */
+#define SD_DEVERR_PAGE 0x2u     /* a needed block-table entry outside [0, num_pages)  */
+#define SD_DEVERR_INDEX 0x4u    /* an attention index >= seqlens[b] (row skipped)     */
+
+/* Geometry shared by the indexer pool and the K/V pools of one cache. */
+typedef struct sd_paged_desc {
+  int32_t num_pages;          /* pages in each pool                           */
+  int32_t page_size;          /* tokens per page, >= 1                        */
+  int32_t max_pages_per_req;  /* row stride of block_table                    */
+  int32_t kv_heads;           /* G: KV heads (1 for MLA latent rows)          */
+} sd_paged_desc;
+
+/* Device scratch (bytes) that any of the three calls below needs for this
+ * shape: scores (unless the caller passes its own), top-k state and split
+ * attention partials. Pure function of its arguments; 0 on invalid input. */
+size_t sd_workspace_size(int32_t B, int32_t G, int32_t max_seqlen, int32_t k,
+                         int32_t H, int32_t Dv);
+
+/* Steps 1 + 2: indexer scores and per-(request, KV head) top-k.
+ *   qi          int8  [B, G, Hi, Di]  indexer queries
+ *   w           int32 [B, G, Hi]      indexer head weights
+ *   ki_pages    int8  [num_pages, page_size, G, Di]  indexer key pool
+ *   block_table int32 [B, max_pages_per_req]  physical page per logical page
+ *   seqlens     int32 [B]             cached tokens per request (incl. current)
+ *   max_seqlen  host upper bound of seqlens (sizes grids and scores)
+ *   indices     int32 [B, G, k]  OUT  ascending request-local tokens, -1 padded
+ *   scores      int32 [B, G, max_seqlen]  OUT, nullable; entries t >= seqlens[b]
+ *               are left unwritten. When NULL the scores live in the workspace. */
+sd_status sd_indexer_topk(const int8_t* qi, const int32_t* w, const int8_t* ki_pages,
+                          const int32_t* block_table, const int32_t* seqlens,
+                          sd_paged_desc pd, int32_t B, int32_t Hi, int32_t Di,
+                          int32_t max_seqlen, int32_t k, int32_t* indices, int32_t* scores,
+                          void* workspace, size_t workspace_bytes, void* stream);
+
+/* Step 3: attention over selected rows, then the split combine.
+ *   q        bf16 [B, H, Dk]
+ *   k_pages  bf16 [num_pages, page_size, G, Dk]
+ *   v_pages  bf16 [num_pages, page_size, G, Dv], or NULL: V = K row[:Dv]
+ *   indices  int32 [B, G, k] request-local tokens; entries < 0 are skipped
+ *   scale    softmax scale applied to q . K
+ *   out      bf16 [B, H, Dv] OUT (round to nearest even); zero when nothing is selected
+ *   lse      fp32 [B, H] OUT, nullable: natural-log sum of exp(scale * q . K_j),
+ *            -inf when nothing is selected */
+sd_status sd_sparse_attn(const uint16_t* q, const uint16_t* k_pages, const uint16_t* v_pages,
+                         const int32_t* block_table, const int32_t* seqlens,
+                         const int32_t* indices, sd_paged_desc pd, int32_t B, int32_t H,
+                         int32_t Dk, int32_t Dv, int32_t k, float scale, uint16_t* out,
+                         float* lse, void* workspace, size_t workspace_bytes, void* stream);
+
+/* Steps 1 + 2 + 3 in one call on one stream (arguments as above). */
+sd_status sd_decode_step(const int8_t* qi, const int32_t* w, const int8_t* ki_pages,
+                         const uint16_t* q, const uint16_t* k_pages, const uint16_t* v_pages,
+                         const int32_t* block_table, const int32_t* seqlens, sd_paged_desc pd,
+                         int32_t B, int32_t Hi, int32_t Di, int32_t H, int32_t Dk, int32_t Dv,
+                         int32_t max_seqlen, int32_t k, float scale, int32_t* indices,
+                         int32_t* scores, uint16_t* out, float* lse, void* workspace,
+                         size_t workspace_bytes, void* stream);
+
+/* Stage timing for monitoring and benchmarks (no counterpart on the pages).
+ * `events` points to 2 * n cudaEvent_t handles created by the caller; while
+ * set, every call of this thread records events[2*i] just before and
+ * events[2*i+1] just after stage i on the call's stream, for the stages
+ * 0 = indexer scores, 1 = top-k, 2 = split attention, 3 = combine (a stage
+ * a call does not run records nothing). n = 0 or events = NULL switches it
+ * off. The handles must outlive their use; the library does not own them. */
+sd_status sd_set_stage_events(void* const* events, int32_t n);
+
+/* Reads (and with clear != 0 resets) the sticky device error word of the
+ * current device. Synchronises the device: for tests and debugging only. */
+sd_status sd_get_device_errors(uint32_t* bits, int32_t clear);
+
+/* Human-readable name of a status. Never NULL. */
+const char* sd_status_str(sd_status status);
+
+/* The cudaError_t of the last failing CUDA call in this thread (0 if none). */
+int32_t sd_last_cuda_error(void);
+
+/* Number of kernel launches the last successful call enqueued (per thread). */
+int32_t sd_last_launch_count(void);
+
+/* Library ABI version, (major << 16) | minor. */
+int32_t sd_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SD_API_H */

@@ -1,0 +1,82 @@
+"""The C ABI library without a GPU: it loads, exports every symbol the header
+declares, sizes workspaces deterministically and rejects bad arguments before
+any CUDA call."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import top_sparse_decode_paged_b200 as sd
+from top_sparse_decode_paged_b200 import api
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_functions():
+    text = open(os.path.join(ROOT, "include", "sd_api.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(sd_[a-z_]+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from top_sparse_decode_paged_b200 import build
+    build.build()
+    return sd.load_library()
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = _declared_functions()
+    assert len(names) >= 9
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(api.EXPORTED)
+
+
+def test_version_and_status_strings(lib):
+    assert lib.sd_version() >= 1
+    assert lib.sd_status_str(0) == b"SD_OK"
+    assert lib.sd_status_str(3) == b"SD_ERR_WORKSPACE"
+    assert lib.sd_status_str(99) == b"SD_ERR_UNKNOWN"
+
+
+def test_workspace_size_is_deterministic_and_rejects_bad_shapes(lib):
+    a = sd.workspace_size(32, 1, 65536, 2048, 128, 512)
+    assert a == sd.workspace_size(32, 1, 65536, 2048, 128, 512)
+    assert a >= 32 * 65536 * 4 and a % 256 == 0
+    assert sd.workspace_size(-1, 1, 10, 4, 4, 64) == 0
+    assert sd.workspace_size(1, 3, 10, 4, 4, 64) == 0     # H % G != 0
+
+
+def _call_indexer(lib, **over):
+    args = dict(qi=256, w=256, ki=256, bt=256, sl=256, B=1, Hi=4, Di=32, L=64, k=8, idx=256)
+    args.update(over)
+    desc = api.PagedDesc(4, 16, 4, 1)
+    return lib.sd_indexer_topk(args["qi"], args["w"], args["ki"], args["bt"], args["sl"], desc,
+                               args["B"], args["Hi"], args["Di"], args["L"], args["k"], args["idx"],
+                               None, None, 0, None)
+
+
+def test_argument_errors_return_before_any_launch(lib):
+    assert _call_indexer(lib, qi=None) == 1                  # SD_ERR_INVALID_ARG
+    assert _call_indexer(lib, k=0) == 1
+    assert _call_indexer(lib, Di=48) == 2                    # SD_ERR_UNSUPPORTED
+    assert _call_indexer(lib, k=4096) == 2
+    assert _call_indexer(lib, Hi=65) == 2
+    assert _call_indexer(lib) == 3                           # no scores, no workspace
+    assert lib.sd_last_launch_count() == 0
+
+
+def test_attention_argument_errors(lib):
+    desc = api.PagedDesc(4, 16, 4, 1)
+    f = lib.sd_sparse_attn
+    # Dv > Dk with V taken from the K row
+    assert f(256, 256, None, 256, 256, 256, desc, 1, 4, 64, 128, 8, ctypes.c_float(0.1), 256, None,
+             None, 0, None) == 1
+    # unsupported head width
+    assert f(256, 256, None, 256, 256, 256, desc, 1, 4, 96, 96, 8, ctypes.c_float(0.1), 256, None,
+             None, 0, None) == 2
+    # non-finite scale
+    assert f(256, 256, None, 256, 256, 256, desc, 1, 4, 64, 64, 8, ctypes.c_float(float("nan")), 256,
+             None, None, 0, None) == 1

@@ -1,0 +1,142 @@
+"""Edge cases and degenerate inputs on the GPU path (through the C ABI)."""
+import numpy as np
+import pytest
+
+import oracle
+from top_sparse_decode_paged_b200 import workloads as W
+
+from helpers import assert_out_close, run_step, to_device
+
+pytestmark = pytest.mark.gpu
+
+
+def _sd():
+    import top_sparse_decode_paged_b200 as sd
+    sd.device_errors(clear=True)
+    return sd
+
+
+def test_heavy_ties_take_lowest_tokens():
+    sd = _sd()
+    wl = W.make(W.spec("b4_l4096_mla", B=2, seqlens=(4096, 3000)))
+    wl.ki_pages[:] = 0          # every score is 0: the first k tokens win
+    got = run_step(wl, to_device(wl))
+    for b in range(2):
+        assert got["indices"][b, 0].tolist() == list(range(2048))
+    assert sd.device_errors() == 0
+
+
+def test_k_at_least_seqlen_equals_dense_attention():
+    wl = W.make(W.spec("b4_l4096_mla", seqlens=(2048, 100, 1, 1999), seed=21))
+    got = run_step(wl, to_device(wl))
+    for b, L in enumerate(wl.seqlens):
+        assert got["indices"][b, 0, :L].tolist() == list(range(L))
+        assert (got["indices"][b, 0, L:] == -1).all()
+    dense, _ = oracle.dense_attention(wl.q, wl.k_pages, None, 512, wl.block_table, wl.seqlens, 1, wl.spec.scale)
+    assert_out_close(got["out"], dense, "dense")
+
+
+def test_empty_request_gives_zero_output_and_minus_one_indices():
+    sd = _sd()
+    wl = W.make(W.spec("tiny", seqlens=(0,), spare_pages=1))
+    # the generator makes a 1-column block table of -1 for an empty request
+    got = run_step(wl, to_device(wl))
+    assert (got["indices"] == -1).all()
+    assert (got["out"] == 0).all()
+    assert np.isneginf(got["lse"]).all()
+    assert sd.device_errors() == 0
+
+
+def test_single_selected_row_is_returned_exactly():
+    wl = W.make(W.spec("perhead_b16_gqa", seqlens=(300, 77), k=1, seed=22))
+    got = run_step(wl, to_device(wl))
+    ref = oracle.decode_step(wl)
+    for b in range(2):
+        assert np.array_equal(got["indices"][b], ref["indices"][b])
+        # one row: softmax weight exactly 1, out = V row exactly (bf16 -> bf16)
+        assert np.array_equal(got["out"][b], ref["out"][b])
+
+
+def test_bad_block_table_entry_sets_error_bit_and_masks():
+    sd = _sd()
+    wl = W.make(W.spec("tiny", seqlens=(200,)))
+    wl.block_table[0, 3] = wl.num_pages + 5     # tokens 48..63 point outside the pool
+    got = run_step(wl, to_device(wl))
+    bits = sd.device_errors()
+    assert bits & sd.SD_DEVERR_PAGE
+    assert not (set(range(48, 64)) & set(got["indices"][0, 0].tolist()))
+
+
+def test_seqlen_past_block_table_sets_error_bit():
+    import torch
+    sd = _sd()
+    wl = W.make(W.spec("tiny", seqlens=(64,)))
+    d = to_device(wl)
+    d["seqlens"] = torch.tensor([10_000], dtype=torch.int32, device="cuda")
+    idx = sd.sd_indexer_topk(d["qi"], d["w"], d["ki_pages"], d["block_table"], d["seqlens"], 32, 64)
+    torch.cuda.synchronize()
+    assert sd.device_errors() & sd.SD_DEVERR_SEQLEN
+    assert (idx.cpu().numpy() >= 0).all()
+
+
+def test_index_past_seqlen_is_skipped_and_flagged():
+    import torch
+    sd = _sd()
+    wl = W.make(W.spec("tiny", seqlens=(100,)))
+    d = to_device(wl)
+    sel = np.array([[[5, 9, 300, 40] + [-1] * 28]], dtype=np.int32)
+    out = sd.sd_sparse_attn(d["q"], d["k_pages"], None, d["block_table"], d["seqlens"],
+                            torch.from_numpy(sel).cuda(), wl.spec.scale, 64)
+    torch.cuda.synchronize()
+    assert sd.device_errors() & sd.SD_DEVERR_INDEX
+    ref, _ = oracle.sparse_attention(wl.q, wl.k_pages, None, 64, wl.block_table, wl.seqlens,
+                                     [np.array([[5, 9, 40]])], wl.spec.scale)
+    assert_out_close(out.float().cpu().numpy(), ref, "skip")
+
+
+def test_invalid_arguments_raise_before_launch():
+    import torch
+    sd = _sd()
+    wl = W.make(W.spec("tiny"))
+    d = to_device(wl)
+    with pytest.raises(sd.SdError):
+        sd.sd_indexer_topk(d["qi"], d["w"], d["ki_pages"], d["block_table"], d["seqlens"], 4096, 256)
+    with pytest.raises(sd.SdError):
+        sd.sd_sparse_attn(d["q"], d["k_pages"], None, d["block_table"], d["seqlens"],
+                          torch.zeros((1, 1, 4), dtype=torch.int32, device="cuda"), 0.1, 96)
+
+
+def test_cuda_graph_capture_and_replay_with_new_inputs():
+    import torch
+    import top_sparse_decode_paged_b200 as sd
+    wl = W.make(W.spec("b4_l4096_mla", B=2, seqlens=(4096, 2500), seed=23))
+    d = to_device(wl)
+    s = wl.spec
+    ws = sd.alloc_workspace(2, 1, wl.max_seqlen, s.k, s.H, s.Dv)
+    idx = torch.empty((2, 1, s.k), dtype=torch.int32, device="cuda")
+    out = torch.empty((2, s.H, s.Dv), dtype=torch.bfloat16, device="cuda")
+    run = lambda: sd.sd_decode_step(d["qi"], d["w"], d["ki_pages"], d["q"], d["k_pages"], None,  # noqa: E731
+                                    d["block_table"], d["seqlens"], s.k, wl.max_seqlen, s.scale, s.Dv,
+                                    indices=idx, out=out, workspace=ws)
+    stream = torch.cuda.Stream()
+    with torch.cuda.stream(stream):
+        run()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        run()
+    wl2 = W.make(W.spec("b4_l4096_mla", B=2, seqlens=(4096, 2500), seed=24))
+    d2 = to_device(wl2)
+    for key in ("qi", "w", "q"):
+        d[key].copy_(d2[key])
+    g.replay()
+    torch.cuda.synchronize()
+    ref = oracle.decode_step(dict_to_wl(wl, wl2))
+    assert np.array_equal(idx.cpu().numpy()[0], ref["indices"][0])
+    assert np.array_equal(idx.cpu().numpy()[1], ref["indices"][1])
+    assert_out_close(out.float().cpu().numpy(), ref["out"], "graph")
+
+
+def dict_to_wl(base, queries_from):
+    import dataclasses
+    return dataclasses.replace(base, qi=queries_from.qi, w=queries_from.w, q=queries_from.q)

@@ -1,0 +1,26 @@
+"""Top-k sparse decode attention over a paged KV cache, for NVIDIA B200 (sm_100a).
+
+The computation lives in ``libsd.so`` (hand-written CUDA kernels behind the C
+ABI of ``include/sd_api.h``); this package is a thin ctypes binding over it
+plus the seeded synthetic-input generator used by tests and benchmarks.
+"""
+from .api import (  # noqa: F401
+    EXPORTED,
+    SD_DEVERR_INDEX,
+    SD_DEVERR_PAGE,
+    SD_DEVERR_SEQLEN,
+    SdError,
+    alloc_workspace,
+    device_errors,
+    last_launch_count,
+    load_library,
+    sd_decode_step,
+    sd_indexer_topk,
+    sd_sparse_attn,
+    workspace_size,
+)
+
+__all__ = [
+    "sd_indexer_topk", "sd_sparse_attn", "sd_decode_step", "workspace_size", "alloc_workspace",
+    "device_errors", "load_library", "SdError",
+]

@@ -1,0 +1,305 @@
+// Host side of the C ABI declared in include/sd_api.h: argument checks,
+// workspace carve-up, kernel selection and launches on the caller's stream.
+// Nothing here allocates or synchronises (except sd_get_device_errors).
+
+#include <cuda_runtime.h>
+#include <math.h>
+
+#include <algorithm>
+#include <stdint.h>
+
+#include "../../include/sd_api.h"
+#include "attn_mma.cuh"
+#include "indexer_dp4a.cuh"
+#include "sd_common.cuh"
+#include "topk_radix.cuh"
+
+namespace {
+
+thread_local int32_t t_last_cuda_error = 0;
+thread_local int32_t t_launches = 0;
+thread_local cudaEvent_t t_stage_events[8];
+thread_local int32_t t_stage_count = 0;
+
+enum Stage { kStageIndexer = 0, kStageTopk = 1, kStageAttn = 2, kStageCombine = 3 };
+
+void stage_mark(int stage, int edge, cudaStream_t st) {
+  if (stage < t_stage_count) cudaEventRecord(t_stage_events[2 * stage + edge], st);
+}
+
+constexpr size_t kAlign = 256;
+constexpr int kMaxK = 2048;
+constexpr int kMaxSeqlen = 1 << 20;
+constexpr int kAttnTargetCtas = 296;  // two waves' worth of CTAs on 148 SMs
+constexpr int kAttnMaxSplits = 16;
+
+size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+sd_status cuda_check(cudaError_t e) {
+  if (e == cudaSuccess) return SD_OK;
+  t_last_cuda_error = static_cast<int32_t>(e);
+  return SD_ERR_CUDA;
+}
+
+sd_status after_launch() {
+  ++t_launches;
+  return cuda_check(cudaGetLastError());
+}
+
+struct AttnPlan {
+  int mt, hb, n_hb, n_splits, slots_per_split;
+};
+
+// Split plan for the attention: a deterministic function of the shape only,
+// so that sd_workspace_size() can size the partials without a device query.
+AttnPlan attn_plan(int B, int G, int H, int k) {
+  AttnPlan p;
+  const int qpk = H / G;
+  p.mt = qpk >= 32 ? 2 : 1;
+  p.hb = 16 * p.mt;
+  p.n_hb = sd::ceil_div(qpk, p.hb);
+  const long long base = (long long)B * G * p.n_hb;
+  const int max_splits = std::min(kAttnMaxSplits, sd::ceil_div(k, sd::kAttnTile));
+  long long want = (kAttnTargetCtas + base - 1) / base;
+  int splits = static_cast<int>(std::max(1LL, std::min<long long>(want, max_splits)));
+  p.slots_per_split = sd::ceil_div(sd::ceil_div(k, splits), sd::kAttnTile) * sd::kAttnTile;
+  p.n_splits = sd::ceil_div(k, p.slots_per_split);
+  return p;
+}
+
+size_t scores_bytes(int B, int G, int max_seqlen) {
+  return align_up(sizeof(int32_t) * (size_t)B * G * (size_t)max_seqlen);
+}
+
+size_t attn_bytes(int B, int G, int H, int k, int Dv) {
+  const AttnPlan p = attn_plan(B, G, H, k);
+  const size_t n = (size_t)B * H * p.n_splits;
+  return align_up(sizeof(float) * n * Dv) + align_up(sizeof(float2) * n);
+}
+
+bool ws_ok(const void* ws, size_t have, size_t need) {
+  if (need == 0) return true;
+  return ws != nullptr && have >= need && (reinterpret_cast<uintptr_t>(ws) % kAlign) == 0;
+}
+
+bool geom_ok(const sd_paged_desc& pd) {
+  return pd.num_pages > 0 && pd.page_size > 0 && pd.max_pages_per_req > 0 && pd.kv_heads > 0;
+}
+
+sd_status check_indexer_args(const int8_t* qi, const int32_t* w, const int8_t* ki_pages,
+                             const int32_t* bt, const int32_t* seqlens, const sd_paged_desc& pd,
+                             int B, int Hi, int Di, int max_seqlen, int k, const int32_t* indices) {
+  if (!qi || !w || !ki_pages || !bt || !seqlens || !indices) return SD_ERR_INVALID_ARG;
+  if (!geom_ok(pd) || B < 0 || Hi <= 0 || Di <= 0 || max_seqlen < 0 || k <= 0)
+    return SD_ERR_INVALID_ARG;
+  if (Di != 32 && Di != 64 && Di != 128) return SD_ERR_UNSUPPORTED;
+  if (Hi > 64 || pd.kv_heads * Di > 1024) return SD_ERR_UNSUPPORTED;
+  if (k > kMaxK || max_seqlen > kMaxSeqlen) return SD_ERR_UNSUPPORTED;
+  return SD_OK;
+}
+
+sd_status check_attn_args(const uint16_t* q, const uint16_t* k_pages, const int32_t* bt,
+                          const int32_t* seqlens, const int32_t* indices, const sd_paged_desc& pd,
+                          int B, int H, int Dk, int Dv, int k, float scale, const uint16_t* out,
+                          bool v_separate) {
+  if (!q || !k_pages || !bt || !seqlens || !indices || !out) return SD_ERR_INVALID_ARG;
+  if (!geom_ok(pd) || B < 0 || H <= 0 || Dk <= 0 || Dv <= 0 || k <= 0 || !isfinite(scale))
+    return SD_ERR_INVALID_ARG;
+  if (H % pd.kv_heads != 0) return SD_ERR_INVALID_ARG;
+  if (!v_separate && Dv > Dk) return SD_ERR_INVALID_ARG;
+  const bool shape_ok = (Dk == 64 && Dv == 64) || (Dk == 128 && Dv == 128) || (Dk == 576 && Dv == 512);
+  if (!shape_ok || H / pd.kv_heads > 128 || k > kMaxK) return SD_ERR_UNSUPPORTED;
+  return SD_OK;
+}
+
+template <int DI>
+sd_status launch_indexer_t(const int8_t* qi, const int32_t* w, const int8_t* ki, const int32_t* bt,
+                           const int32_t* seqlens, int32_t* scores, const sd_paged_desc& pd, int B,
+                           int Hi, int max_seqlen, cudaStream_t st) {
+  const size_t smem = sd::indexer_dp4a_smem(pd.kv_heads, Hi, DI);
+  dim3 grid(sd::ceil_div(max_seqlen, sd::kIdxTokensPerCta), B);
+  stage_mark(kStageIndexer, 0, st);
+  sd::indexer_dp4a_kernel<DI><<<grid, sd::kIdxThreads, smem, st>>>(
+      qi, w, ki, bt, seqlens, scores, pd.num_pages, pd.page_size, pd.max_pages_per_req,
+      pd.kv_heads, Hi, max_seqlen);
+  stage_mark(kStageIndexer, 1, st);
+  return after_launch();
+}
+
+sd_status launch_indexer_topk(const int8_t* qi, const int32_t* w, const int8_t* ki, const int32_t* bt,
+                              const int32_t* seqlens, const sd_paged_desc& pd, int B, int Hi, int Di,
+                              int max_seqlen, int k, int32_t* indices, int32_t* scores,
+                              cudaStream_t st) {
+  const int G = pd.kv_heads;
+  if (B == 0) return SD_OK;
+  if (max_seqlen > 0) {
+    sd_status s = SD_OK;
+    if (Di == 32) s = launch_indexer_t<32>(qi, w, ki, bt, seqlens, scores, pd, B, Hi, max_seqlen, st);
+    else if (Di == 64) s = launch_indexer_t<64>(qi, w, ki, bt, seqlens, scores, pd, B, Hi, max_seqlen, st);
+    else s = launch_indexer_t<128>(qi, w, ki, bt, seqlens, scores, pd, B, Hi, max_seqlen, st);
+    if (s != SD_OK) return s;
+  }
+  const int cap = std::min(max_seqlen, pd.max_pages_per_req * pd.page_size);
+  stage_mark(kStageTopk, 0, st);
+  sd::topk_radix_kernel<<<B * G, sd::kTopkThreads, 0, st>>>(scores, seqlens, indices, G,
+                                                             std::max(max_seqlen, 1), cap, k);
+  stage_mark(kStageTopk, 1, st);
+  return after_launch();
+}
+
+template <int DK, int DV, int MT>
+sd_status launch_attn_t(const uint16_t* q, const uint16_t* kp, const uint16_t* vp, const int32_t* bt,
+                        const int32_t* seqlens, const int32_t* indices, const sd_paged_desc& pd,
+                        int B, int H, int k, float scale, uint16_t* out, float* lse,
+                        const AttnPlan& p, float* part_o, float2* part_ml, int seqlen_cap,
+                        cudaStream_t st) {
+  using C = sd::AttnMmaCfg<DK, DV, MT>;
+  const size_t smem = C::smem_bytes(vp != nullptr);
+  auto kern = sd::attn_split_mma_kernel<DK, DV, MT>;
+  sd_status s = cuda_check(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                static_cast<int>(smem)));
+  if (s != SD_OK) return s;
+  const float scale_log2 = scale * 1.4426950408889634f;
+  dim3 grid(p.n_splits, p.n_hb, B * pd.kv_heads);
+  stage_mark(kStageAttn, 0, st);
+  kern<<<grid, C::THREADS, smem, st>>>(
+      reinterpret_cast<const __nv_bfloat16*>(q), reinterpret_cast<const __nv_bfloat16*>(kp),
+      reinterpret_cast<const __nv_bfloat16*>(vp), bt, seqlens, indices, pd.num_pages, pd.page_size,
+      pd.max_pages_per_req, pd.kv_heads, H, k, seqlen_cap, scale_log2, p.n_hb, p.n_splits,
+      p.slots_per_split, part_o, part_ml);
+  stage_mark(kStageAttn, 1, st);
+  if ((s = after_launch()) != SD_OK) return s;
+  stage_mark(kStageCombine, 0, st);
+  sd::attn_combine_kernel<DV><<<B * H, 128, 0, st>>>(part_o, part_ml, p.n_splits,
+                                                      reinterpret_cast<__nv_bfloat16*>(out), lse);
+  stage_mark(kStageCombine, 1, st);
+  return after_launch();
+}
+
+sd_status launch_attn(const uint16_t* q, const uint16_t* kp, const uint16_t* vp, const int32_t* bt,
+                      const int32_t* seqlens, const int32_t* indices, const sd_paged_desc& pd, int B,
+                      int H, int Dk, int Dv, int k, float scale, uint16_t* out, float* lse,
+                      void* ws, int seqlen_cap, cudaStream_t st) {
+  if (B == 0) return SD_OK;
+  const AttnPlan p = attn_plan(B, pd.kv_heads, H, k);
+  const size_t n = (size_t)B * H * p.n_splits;
+  float* part_o = static_cast<float*>(ws);
+  float2* part_ml = reinterpret_cast<float2*>(static_cast<char*>(ws) + align_up(sizeof(float) * n * Dv));
+#define SD_ATTN(DK_, DV_)                                                                              \
+  return p.mt == 2 ? launch_attn_t<DK_, DV_, 2>(q, kp, vp, bt, seqlens, indices, pd, B, H, k, scale, \
+                                                out, lse, p, part_o, part_ml, seqlen_cap, st)         \
+                   : launch_attn_t<DK_, DV_, 1>(q, kp, vp, bt, seqlens, indices, pd, B, H, k, scale, \
+                                                out, lse, p, part_o, part_ml, seqlen_cap, st)
+  if (Dk == 576) { SD_ATTN(576, 512); }
+  if (Dk == 128) { SD_ATTN(128, 128); }
+  SD_ATTN(64, 64);
+#undef SD_ATTN
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t sd_workspace_size(int32_t B, int32_t G, int32_t max_seqlen, int32_t k, int32_t H, int32_t Dv) {
+  if (B < 0 || G <= 0 || max_seqlen < 0 || k <= 0 || H <= 0 || Dv <= 0 || H % G != 0) return 0;
+  return scores_bytes(B, G, max_seqlen) + attn_bytes(B, G, H, k, Dv);
+}
+
+sd_status sd_indexer_topk(const int8_t* qi, const int32_t* w, const int8_t* ki_pages,
+                          const int32_t* block_table, const int32_t* seqlens, sd_paged_desc pd,
+                          int32_t B, int32_t Hi, int32_t Di, int32_t max_seqlen, int32_t k,
+                          int32_t* indices, int32_t* scores, void* workspace, size_t workspace_bytes,
+                          void* stream) {
+  t_launches = 0;
+  sd_status s = check_indexer_args(qi, w, ki_pages, block_table, seqlens, pd, B, Hi, Di, max_seqlen,
+                                   k, indices);
+  if (s != SD_OK) return s;
+  if (scores == nullptr) {
+    if (!ws_ok(workspace, workspace_bytes, scores_bytes(B, pd.kv_heads, max_seqlen)))
+      return SD_ERR_WORKSPACE;
+    scores = static_cast<int32_t*>(workspace);
+  }
+  return launch_indexer_topk(qi, w, ki_pages, block_table, seqlens, pd, B, Hi, Di, max_seqlen, k,
+                             indices, scores, static_cast<cudaStream_t>(stream));
+}
+
+sd_status sd_sparse_attn(const uint16_t* q, const uint16_t* k_pages, const uint16_t* v_pages,
+                         const int32_t* block_table, const int32_t* seqlens, const int32_t* indices,
+                         sd_paged_desc pd, int32_t B, int32_t H, int32_t Dk, int32_t Dv, int32_t k,
+                         float scale, uint16_t* out, float* lse, void* workspace,
+                         size_t workspace_bytes, void* stream) {
+  t_launches = 0;
+  sd_status s = check_attn_args(q, k_pages, block_table, seqlens, indices, pd, B, H, Dk, Dv, k, scale,
+                                out, v_pages != nullptr);
+  if (s != SD_OK) return s;
+  if (!ws_ok(workspace, workspace_bytes, attn_bytes(B, pd.kv_heads, H, k, Dv))) return SD_ERR_WORKSPACE;
+  const int cap = pd.max_pages_per_req * pd.page_size;
+  return launch_attn(q, k_pages, v_pages, block_table, seqlens, indices, pd, B, H, Dk, Dv, k, scale,
+                     out, lse, workspace, cap, static_cast<cudaStream_t>(stream));
+}
+
+sd_status sd_decode_step(const int8_t* qi, const int32_t* w, const int8_t* ki_pages, const uint16_t* q,
+                         const uint16_t* k_pages, const uint16_t* v_pages, const int32_t* block_table,
+                         const int32_t* seqlens, sd_paged_desc pd, int32_t B, int32_t Hi, int32_t Di,
+                         int32_t H, int32_t Dk, int32_t Dv, int32_t max_seqlen, int32_t k, float scale,
+                         int32_t* indices, int32_t* scores, uint16_t* out, float* lse, void* workspace,
+                         size_t workspace_bytes, void* stream) {
+  t_launches = 0;
+  sd_status s = check_indexer_args(qi, w, ki_pages, block_table, seqlens, pd, B, Hi, Di, max_seqlen,
+                                   k, indices);
+  if (s != SD_OK) return s;
+  s = check_attn_args(q, k_pages, block_table, seqlens, indices, pd, B, H, Dk, Dv, k, scale, out,
+                      v_pages != nullptr);
+  if (s != SD_OK) return s;
+  const size_t sb = scores_bytes(B, pd.kv_heads, max_seqlen);
+  if (!ws_ok(workspace, workspace_bytes, sd_workspace_size(B, pd.kv_heads, max_seqlen, k, H, Dv)))
+    return SD_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int32_t* sc = scores ? scores : static_cast<int32_t*>(workspace);
+  s = launch_indexer_topk(qi, w, ki_pages, block_table, seqlens, pd, B, Hi, Di, max_seqlen, k, indices,
+                          sc, st);
+  if (s != SD_OK) return s;
+  const int launches = t_launches;
+  const int cap = std::min(max_seqlen, pd.max_pages_per_req * pd.page_size);
+  s = launch_attn(q, k_pages, v_pages, block_table, seqlens, indices, pd, B, H, Dk, Dv, k, scale, out,
+                  lse, static_cast<char*>(workspace) + sb, cap, st);
+  t_launches += launches;
+  return s;
+}
+
+sd_status sd_set_stage_events(void* const* events, int32_t n) {
+  if (n < 0 || n > 4 || (n > 0 && events == nullptr)) return SD_ERR_INVALID_ARG;
+  for (int i = 0; i < 2 * n; ++i) {
+    if (events[i] == nullptr) return SD_ERR_INVALID_ARG;
+    t_stage_events[i] = static_cast<cudaEvent_t>(events[i]);
+  }
+  t_stage_count = n;
+  return SD_OK;
+}
+
+sd_status sd_get_device_errors(uint32_t* bits, int32_t clear) {
+  if (!bits) return SD_ERR_INVALID_ARG;
+  sd_status s = cuda_check(cudaDeviceSynchronize());
+  if (s != SD_OK) return s;
+  s = cuda_check(cudaMemcpyFromSymbol(bits, sd::g_error_bits, sizeof(uint32_t)));
+  if (s != SD_OK || !clear) return s;
+  const uint32_t zero = 0;
+  return cuda_check(cudaMemcpyToSymbol(sd::g_error_bits, &zero, sizeof(uint32_t)));
+}
+
+const char* sd_status_str(sd_status status) {
+  switch (status) {
+    case SD_OK: return "SD_OK";
+    case SD_ERR_INVALID_ARG: return "SD_ERR_INVALID_ARG";
+    case SD_ERR_UNSUPPORTED: return "SD_ERR_UNSUPPORTED";
+    case SD_ERR_WORKSPACE: return "SD_ERR_WORKSPACE";
+    case SD_ERR_CUDA: return "SD_ERR_CUDA";
+  }
+  return "SD_ERR_UNKNOWN";
+}
+
+int32_t sd_last_cuda_error(void) { return t_last_cuda_error; }
+int32_t sd_last_launch_count(void) { return t_launches; }
+int32_t sd_version(void) { return (0 << 16) | 1; }
+
+}  // extern "C"

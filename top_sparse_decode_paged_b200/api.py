@@ -197,6 +197,8 @@ class StageTimer:
 
     def arm(self):
         ev = [torch.cuda.Event(enable_timing=True) for _ in range(8)]
+        for e in ev:
+            e.record()  # torch creates the CUDA event lazily, on its first record
         arr = (ctypes.c_void_p * 8)(*[e.cuda_event for e in ev])
         _check(load_library().sd_set_stage_events(arr, 4))
         self._pairs.append(ev)

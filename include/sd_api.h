@@ -133,6 +133,31 @@ sd_status sd_decode_step(const int8_t* qi, const int32_t* w, const int8_t* ki_pa
                          int32_t* scores, uint16_t* out, float* lse, void* workspace,
                          size_t workspace_bytes, void* stream);
 
+/* Steps 1 + 2 without any workspace (the pages have no counterpart; this is a
+ * deployment convenience). It is sd_indexer_topk for callers that cannot
+ * allocate device memory: a plugin that runs inside a host application which
+ * owns every device allocation, or a serving loop that must not allocate once
+ * it has started. Such callers cannot provide a scores workspace. Here the
+ * scores live in a scratch array that the library itself holds on each device
+ * it is used on, from first use until process exit:
+ * SD_NOALLOC_MAX_SCORES int32 values (16 MiB).
+ *   Arguments, outputs and errors are as for sd_indexer_topk. There is no
+ *   scores output. The call returns SD_ERR_WORKSPACE, with nothing enqueued,
+ *   when B * G * max_seqlen > SD_NOALLOC_MAX_SCORES.
+ *   The first call on a device looks up that device's scratch address (a
+ *   runtime query, not an allocation). Make that first call before any stream
+ *   capture on that device.
+ *   Every call on a device shares the one scratch array. Calls whose work
+ *   overlaps on the GPU (other streams, other threads) race on it and give
+ *   undefined results: serialise them. The array keeps the last call's scores,
+ *   and that is harmless, because every score a call reads it has written
+ *   first. The call never allocates or frees device memory. */
+#define SD_NOALLOC_MAX_SCORES (4u << 20)
+sd_status sd_indexer_topk_noalloc(const int8_t* qi, const int32_t* w, const int8_t* ki_pages,
+                                  const int32_t* block_table, const int32_t* seqlens,
+                                  sd_paged_desc pd, int32_t B, int32_t Hi, int32_t Di,
+                                  int32_t max_seqlen, int32_t k, int32_t* indices, void* stream);
+
 /* Stage timing for monitoring and benchmarks (no counterpart on the pages).
  * `events` points to 2 * n cudaEvent_t handles created by the caller; while
  * set, every call of this thread records events[2*i] just before and

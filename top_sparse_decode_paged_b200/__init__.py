@@ -6,21 +6,24 @@ plus the seeded synthetic-input generator used by tests and benchmarks.
 """
 from .api import (  # noqa: F401
     EXPORTED,
+    NOALLOC_MAX_SCORES,
     SD_DEVERR_INDEX,
     SD_DEVERR_PAGE,
     SD_DEVERR_SEQLEN,
     SdError,
+    StageTimer,
     alloc_workspace,
     device_errors,
     last_launch_count,
     load_library,
     sd_decode_step,
     sd_indexer_topk,
+    sd_indexer_topk_noalloc,
     sd_sparse_attn,
     workspace_size,
 )
 
 __all__ = [
-    "sd_indexer_topk", "sd_sparse_attn", "sd_decode_step", "workspace_size", "alloc_workspace",
-    "device_errors", "load_library", "SdError",
+    "sd_indexer_topk", "sd_indexer_topk_noalloc", "sd_sparse_attn", "sd_decode_step",
+    "workspace_size", "alloc_workspace", "device_errors", "load_library", "SdError", "StageTimer",
 ]

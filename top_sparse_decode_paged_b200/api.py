@@ -21,7 +21,8 @@ SD_DEVERR_SEQLEN = 0x1
 SD_DEVERR_PAGE = 0x2
 SD_DEVERR_INDEX = 0x4
 
-EXPORTED = ("sd_workspace_size", "sd_indexer_topk", "sd_sparse_attn", "sd_decode_step",
+EXPORTED = ("sd_workspace_size", "sd_indexer_topk", "sd_indexer_topk_noalloc", "sd_sparse_attn",
+            "sd_decode_step",
             "sd_set_stage_events", "sd_get_device_errors", "sd_status_str", "sd_last_cuda_error",
             "sd_last_launch_count", "sd_version")
 
@@ -56,6 +57,8 @@ def load_library(path: str = LIB_PATH):
     lib.sd_workspace_size.argtypes = [i32] * 6
     lib.sd_indexer_topk.restype = i32
     lib.sd_indexer_topk.argtypes = [p, p, p, p, p, PagedDesc, i32, i32, i32, i32, i32, p, p, p, sz, p]
+    lib.sd_indexer_topk_noalloc.restype = i32
+    lib.sd_indexer_topk_noalloc.argtypes = [p, p, p, p, p, PagedDesc, i32, i32, i32, i32, i32, p, p]
     lib.sd_sparse_attn.restype = i32
     lib.sd_sparse_attn.argtypes = [p, p, p, p, p, p, PagedDesc, i32, i32, i32, i32, i32,
                                    ctypes.c_float, p, p, p, sz, p]
@@ -134,6 +137,28 @@ def sd_indexer_topk(qi, w, ki_pages, block_table, seqlens, k: int, max_seqlen: i
     _check(lib.sd_indexer_topk(_ptr(qi), _ptr(w), _ptr(ki_pages), _ptr(block_table), _ptr(seqlens),
                                _desc(ki_pages, block_table), B, Hi, Di, max_seqlen, k, _ptr(indices),
                                _ptr(scores), _ptr(workspace), ws_bytes, _stream(stream)))
+    return indices
+
+
+NOALLOC_MAX_SCORES = 4 << 20
+
+
+def sd_indexer_topk_noalloc(qi, w, ki_pages, block_table, seqlens, k: int, max_seqlen: int, indices,
+                            stream=None):
+    """Indexer + top-k for callers that cannot allocate device memory.
+
+    The library keeps the scores in its own fixed scratch array (16 MiB per
+    device; B * G * max_seqlen <= NOALLOC_MAX_SCORES), so this call takes no
+    workspace. ``indices`` [B, G, k] int32 must be provided by the caller.
+    Calls on one device share the scratch array: do not let them overlap on
+    the GPU. Make the first call on a device before any CUDA-graph capture."""
+    lib = load_library()
+    B, G, Hi, Di = qi.shape
+    assert qi.dtype == torch.int8 and ki_pages.dtype == torch.int8 and w.dtype == torch.int32
+    assert tuple(indices.shape) == (B, G, k) and indices.dtype == torch.int32
+    _check(lib.sd_indexer_topk_noalloc(_ptr(qi), _ptr(w), _ptr(ki_pages), _ptr(block_table),
+                                       _ptr(seqlens), _desc(ki_pages, block_table), B, Hi, Di,
+                                       max_seqlen, k, _ptr(indices), _stream(stream)))
     return indices
 
 

@@ -6,6 +6,7 @@
 #include <math.h>
 
 #include <algorithm>
+#include <mutex>
 #include <stdint.h>
 
 #include "../../include/sd_api.h"
@@ -303,3 +304,54 @@ int32_t sd_last_launch_count(void) { return t_launches; }
 int32_t sd_version(void) { return (0 << 16) | 1; }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Allocation-free indexer + top-k. The scores go to a fixed scratch array in
+// this library's device image instead of a caller workspace. The host-side name
+// g_noalloc_scores is a stand-in, not a device address. Host code must never
+// hand it to a kernel. Each device's real address is looked up once, with
+// that device current, and cached here.
+// ---------------------------------------------------------------------------
+static __device__ __align__(256) int32_t g_noalloc_scores[SD_NOALLOC_MAX_SCORES];
+
+namespace {
+constexpr int kNoallocMaxDevices = 64;
+std::mutex g_noalloc_mutex;
+int32_t* g_noalloc_addr[kNoallocMaxDevices] = {};
+
+// The current device's address of g_noalloc_scores (looked up on first use).
+sd_status noalloc_scores_for_current_device(int32_t** out) {
+  int dev = 0;
+  sd_status s = cuda_check(cudaGetDevice(&dev));
+  if (s != SD_OK) return s;
+  if (dev < 0 || dev >= kNoallocMaxDevices) return SD_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+  if (g_noalloc_addr[dev] == nullptr) {
+    void* p = nullptr;
+    s = cuda_check(cudaGetSymbolAddress(&p, g_noalloc_scores));
+    if (s != SD_OK) return s;
+    g_noalloc_addr[dev] = static_cast<int32_t*>(p);
+  }
+  *out = g_noalloc_addr[dev];
+  return SD_OK;
+}
+}  // namespace
+
+extern "C" sd_status sd_indexer_topk_noalloc(const int8_t* qi, const int32_t* w, const int8_t* ki_pages,
+                                             const int32_t* block_table, const int32_t* seqlens,
+                                             sd_paged_desc pd, int32_t B, int32_t Hi, int32_t Di,
+                                             int32_t max_seqlen, int32_t k, int32_t* indices,
+                                             void* stream) {
+  t_launches = 0;
+  sd_status s = check_indexer_args(qi, w, ki_pages, block_table, seqlens, pd, B, Hi, Di, max_seqlen,
+                                   k, indices);
+  if (s != SD_OK) return s;
+  if ((size_t)B * pd.kv_heads * (size_t)max_seqlen > (size_t)SD_NOALLOC_MAX_SCORES) return SD_ERR_WORKSPACE;
+  int32_t* scores = nullptr;
+  s = noalloc_scores_for_current_device(&scores);
+  if (s != SD_OK) return s;
+  // Scores are written for every t < seqlens[b] before top-k reads them, so
+  // nothing left over from an earlier call is ever read.
+  return launch_indexer_topk(qi, w, ki_pages, block_table, seqlens, pd, B, Hi, Di, max_seqlen, k,
+                             indices, scores, static_cast<cudaStream_t>(stream));
+}

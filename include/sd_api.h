@@ -78,6 +78,7 @@ typedef enum sd_status {
 #define SD_DEVERR_SEQLEN 0x1u   /* seqlens[b] < 0, > max_seqlen or > the block table  */
 #define SD_DEVERR_PAGE 0x2u     /* a needed block-table entry outside [0, num_pages)  */
 #define SD_DEVERR_INDEX 0x4u    /* an attention index >= seqlens[b] (row skipped)     */
+#define SD_DEVERR_TIMEOUT 0x8u  /* a bounded on-chip wait ran out (the kernel unwound) */
 
 /* Geometry shared by the indexer pool and the K/V pools of one cache. */
 typedef struct sd_paged_desc {

@@ -24,6 +24,9 @@ SMALL = {
     "h128_small": W.spec("b32_l65536_mla", seqlens=(9000, 5003, 1500), seed=12),
     "ragged_small": W.spec("ragged_b64_mla", B=6, ragged=(1024, 8192), seed=13),
     "perhead_small": W.spec("perhead_b16_gqa", seqlens=(4096, 3001, 700), seed=14),
+    "mla_page16": W.spec("b4_l4096_mla", seqlens=(3000, 1234, 129), page_size=16, seed=15),
+    "mla_page32": W.spec("b4_l4096_mla", seqlens=(2500, 4097), page_size=32, seed=16),
+    "mla_page48_fallback": W.spec("b4_l4096_mla", seqlens=(2100, 777), page_size=48, seed=17),
 }
 
 

@@ -2,6 +2,7 @@
 // workspace carve-up, kernel selection and launches on the caller's stream.
 // Nothing here allocates or synchronises (except sd_get_device_errors).
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <math.h>
 
@@ -12,6 +13,7 @@
 #include "../../include/sd_api.h"
 #include "attn_mma.cuh"
 #include "indexer_dp4a.cuh"
+#include "indexer_umma.cuh"
 #include "sd_common.cuh"
 #include "topk_radix.cuh"
 
@@ -127,13 +129,87 @@ sd_status launch_indexer_t(const int8_t* qi, const int32_t* w, const int8_t* ki,
   return after_launch();
 }
 
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no link
+// dependency on libcuda); looked up once per process.
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_tiled_fn() {
+  static EncodeTiledFn fn = []() -> EncodeTiledFn {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return nullptr;
+    return reinterpret_cast<EncodeTiledFn>(p);
+  }();
+  return fn;
+}
+
+// A 2-D int8 map over `rows` rows of 128 bytes, boxes of box_rows x 128 B,
+// 128-byte swizzle (the K-major UMMA operand layout).
+bool encode_rows128(CUtensorMap* map, const void* base, uint64_t rows, uint32_t box_rows) {
+  EncodeTiledFn fn = encode_tiled_fn();
+  if (fn == nullptr || (reinterpret_cast<uintptr_t>(base) & 15u) != 0) return false;
+  const cuuint64_t dims[2] = {128, rows};
+  const cuuint64_t strides[1] = {128};
+  const cuuint32_t box[2] = {128, box_rows};
+  const cuuint32_t estride[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estride,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return 148;
+  return n;
+}
+
+// The tensor-core indexer covers one KV head of 128-byte keys with 64 heads and
+// pages that tile a 128-token block; everything else takes the dp4a kernel.
+bool umma_indexer_fits(const sd_paged_desc& pd, int Hi, int Di, const void* qi, const void* ki) {
+  const int P = pd.page_size;
+  return pd.kv_heads == 1 && Di == 128 && Hi == 64 && P >= 8 && P <= 128 && (128 % P) == 0 &&
+         (reinterpret_cast<uintptr_t>(qi) & 15u) == 0 && (reinterpret_cast<uintptr_t>(ki) & 15u) == 0;
+}
+
+sd_status launch_indexer_umma(const int8_t* qi, const int32_t* w, const int8_t* ki, const int32_t* bt,
+                              const int32_t* seqlens, int32_t* scores, const sd_paged_desc& pd, int B,
+                              int max_seqlen, cudaStream_t st, bool* launched) {
+  constexpr int HI = 64;
+  using Lay = sd::IndexerUmmaLayout<HI>;
+  *launched = false;
+  CUtensorMap tm_keys, tm_q;
+  if (!encode_rows128(&tm_keys, ki, (uint64_t)pd.num_pages * pd.page_size, pd.page_size)) return SD_OK;
+  if (!encode_rows128(&tm_q, qi, (uint64_t)B * HI, HI)) return SD_OK;
+  auto kern = sd::indexer_umma_kernel<HI>;
+  sd_status s = cuda_check(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                static_cast<int>(Lay::kSmemAlloc)));
+  if (s != SD_OK) return s;
+  stage_mark(kStageIndexer, 0, st);
+  kern<<<sm_count(), sd::kUmmaThreads, Lay::kSmemAlloc, st>>>(tm_keys, tm_q, w, bt, seqlens, scores, B,
+                                                              pd.num_pages, pd.page_size,
+                                                              pd.max_pages_per_req, max_seqlen);
+  stage_mark(kStageIndexer, 1, st);
+  *launched = true;
+  return after_launch();
+}
+
 sd_status launch_indexer_topk(const int8_t* qi, const int32_t* w, const int8_t* ki, const int32_t* bt,
                               const int32_t* seqlens, const sd_paged_desc& pd, int B, int Hi, int Di,
                               int max_seqlen, int k, int32_t* indices, int32_t* scores,
                               cudaStream_t st) {
   const int G = pd.kv_heads;
   if (B == 0) return SD_OK;
-  if (max_seqlen > 0) {
+  bool done = false;
+  if (max_seqlen > 0 && umma_indexer_fits(pd, Hi, Di, qi, ki)) {
+    sd_status s = launch_indexer_umma(qi, w, ki, bt, seqlens, scores, pd, B, max_seqlen, st, &done);
+    if (s != SD_OK) return s;
+  }
+  if (max_seqlen > 0 && !done) {
     sd_status s = SD_OK;
     if (Di == 32) s = launch_indexer_t<32>(qi, w, ki, bt, seqlens, scores, pd, B, Hi, max_seqlen, st);
     else if (Di == 64) s = launch_indexer_t<64>(qi, w, ki, bt, seqlens, scores, pd, B, Hi, max_seqlen, st);

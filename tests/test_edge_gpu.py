@@ -140,3 +140,39 @@ def test_cuda_graph_capture_and_replay_with_new_inputs():
 def dict_to_wl(base, queries_from):
     import dataclasses
     return dataclasses.replace(base, qi=queries_from.qi, w=queries_from.w, q=queries_from.q)
+
+
+def _indices_vs_oracle(wl):
+    got = run_step(wl, to_device(wl))
+    sc = oracle.indexer_scores(wl.qi, wl.w, wl.ki_pages, wl.block_table, wl.seqlens)
+    ref = oracle.topk_indices(sc, wl.spec.k)
+    for b in range(wl.seqlens.shape[0]):
+        L = int(wl.seqlens[b])
+        assert np.array_equal(got["scores"][b][:, :L], sc[b]), f"scores b={b}"
+        assert np.array_equal(got["indices"][b], ref[b]), f"indices b={b}"
+    return got
+
+
+def test_topk_two_level_ties_at_the_threshold():
+    """Scores take two values; more tokens hold the high value than k, so the
+    threshold is the high value and the lowest-index ones must win."""
+    wl = W.make(W.spec("b4_l4096_mla", B=2, seqlens=(20000, 9000), seed=41))
+    rng = np.random.default_rng(5)
+    wl.ki_pages[:] = 0
+    row = rng.integers(-64, 65, size=128).astype(np.int8)
+    for b, L in enumerate(wl.seqlens):
+        hot = rng.choice(int(L), size=3000, replace=False)   # > k = 2048
+        for t in hot:
+            wl.ki_pages[wl.block_table[b, t // 64], t % 64, 0] = row
+    _indices_vs_oracle(wl)
+
+
+def test_topk_cluster_slices_with_ragged_rows():
+    """Rows of 4097, 20000 and 131072 tokens in one batch: the top-k runs with
+    the largest cluster and slices whose ends fall mid-row and past short rows."""
+    _indices_vs_oracle(W.make(W.spec("b4_l4096_mla", seqlens=(4097, 20000, 131072, 2049), seed=42)))
+
+
+def test_topk_single_cta_fallback_beyond_cluster_capacity():
+    """max_seqlen above 8 x 16384 takes the one-CTA-per-row kernel."""
+    _indices_vs_oracle(W.make(W.spec("b4_l4096_mla", seqlens=(131073, 5000), seed=43)))

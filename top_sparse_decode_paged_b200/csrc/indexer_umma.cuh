@@ -143,39 +143,61 @@ __global__ void __launch_bounds__(kUmmaThreads, 1) indexer_umma_kernel(
   const long long count = total * (blockIdx.x + 1) / gridDim.x - first;
 
   if (warp == 0) {
-    // ---------------- TMA producer ----------------
-    if (sm100::elect_one()) {
-      TileCursor c;
-      c.init(seqlens, B, cap, first, count);
-      int stage = 0;
-      uint32_t phase = 0;
-      int nq = 0, cur_b = -1;
-      while (c.valid() && !*abort_flag) {
-        if (c.b != cur_b) {
-          const int slot = nq & 1;
-          if (!sm100::mbar_wait(&qempty[slot], ((nq >> 1) & 1) ^ 1)) { *abort_flag = 1; break; }
-          sm100::mbar_arrive_expect_tx(&qfull[slot], Lay::kQBytes);
-          sm100::tma_load_2d(qbuf + slot * Lay::kQBytes, &tm_q, &qfull[slot], 0, c.b * HI);
-          cur_b = c.b;
-          ++nq;
+    // ---------------- TMA producer (whole warp) ----------------
+    // The 32 lanes keep a window of 32 consecutive block-table entries of the
+    // current request, fetched in one coalesced load, so the page lookups of
+    // 16+ tiles cost one memory round trip. Lane j issues the copy of the
+    // tile's j-th page; lane 0 does the barrier bookkeeping.
+    TileCursor c;
+    c.init(seqlens, B, cap, first, count);
+    int stage = 0;
+    uint32_t phase = 0;
+    int nq = 0, cur_b = -1;
+    int win_b = -1, win_p0 = 0, win_val = -1;
+    while (c.valid() && !*abort_flag) {
+      if (c.b != cur_b) {
+        const int slot = nq & 1;
+        bool ok = true;
+        if (lane == 0) {
+          ok = sm100::mbar_wait(&qempty[slot], ((nq >> 1) & 1) ^ 1);
+          if (ok) {
+            sm100::mbar_arrive_expect_tx(&qfull[slot], Lay::kQBytes);
+            sm100::tma_load_2d(qbuf + slot * Lay::kQBytes, &tm_q, &qfull[slot], 0, c.b * HI);
+          }
         }
-        if (!sm100::mbar_wait(&empty[stage], phase ^ 1)) { *abort_flag = 1; break; }
-        const int t0 = c.tile * kUmmaTile;
-        uint32_t bytes = 0;
-        for (int t = t0; t < t0 + kUmmaTile && t < c.L; t += page_size) {
-          const int phys = block_table[(size_t)c.b * max_pages + t / page_size];
-          if (phys >= 0 && phys < num_pages) bytes += page_size * kUmmaRowBytes;
+        if (!__shfl_sync(0xffffffffu, ok, 0)) {
+          if (lane == 0) *abort_flag = 1;
+          break;
         }
-        sm100::mbar_arrive_expect_tx(&full[stage], bytes);
-        for (int t = t0; t < t0 + kUmmaTile && t < c.L; t += page_size) {
-          const int phys = block_table[(size_t)c.b * max_pages + t / page_size];
-          if (phys >= 0 && phys < num_pages)
-            sm100::tma_load_2d(kstage + stage * Lay::kTileBytes + (t - t0) * kUmmaRowBytes, &tm_keys,
-                               &full[stage], 0, phys * page_size);
-        }
-        if (++stage == kUmmaStages) { stage = 0; phase ^= 1; }
-        c.next(seqlens, B, cap);
+        cur_b = c.b;
+        ++nq;
       }
+      const int t0 = c.tile * kUmmaTile;
+      const int p_first = t0 / page_size;
+      const int npages = ceil_div(min(kUmmaTile, c.L - t0), page_size);
+      if (c.b != win_b || p_first < win_p0 || p_first + npages > win_p0 + 32) {
+        win_b = c.b;
+        win_p0 = p_first;
+        const int p = win_p0 + lane;
+        win_val = p < max_pages ? block_table[(size_t)c.b * max_pages + p] : -1;
+      }
+      const int phys = __shfl_sync(0xffffffffu, win_val, min(p_first - win_p0 + lane, 31));
+      const bool mine = lane < npages && phys >= 0 && phys < num_pages;
+      const uint32_t vmask = __ballot_sync(0xffffffffu, mine);
+      bool ok = true;
+      if (lane == 0) {
+        ok = sm100::mbar_wait(&empty[stage], phase ^ 1);
+        if (ok) sm100::mbar_arrive_expect_tx(&full[stage], __popc(vmask) * page_size * kUmmaRowBytes);
+      }
+      if (!__shfl_sync(0xffffffffu, ok, 0)) {
+        if (lane == 0) *abort_flag = 1;
+        break;
+      }
+      if (mine)
+        sm100::tma_load_2d(kstage + stage * Lay::kTileBytes + lane * page_size * kUmmaRowBytes, &tm_keys,
+                           &full[stage], 0, phys * page_size);
+      if (++stage == kUmmaStages) { stage = 0; phase ^= 1; }
+      c.next(seqlens, B, cap);
     }
   } else if (warp == 1) {
     // ---------------- MMA issuer ----------------
@@ -228,6 +250,9 @@ __global__ void __launch_bounds__(kUmmaThreads, 1) indexer_umma_kernel(
         for (int h = 0; h < HI; ++h) wreg[h] = __ldg(w + (size_t)c.b * HI + h);
         cur_b = c.b;
       }
+      const int t = c.tile * kUmmaTile + row;
+      int phys = 0;
+      if (t < c.L) phys = block_table[(size_t)c.b * max_pages + t / page_size];  // overlaps the wait
       const bool ok = sm100::mbar_wait(&accfull[acc], accphase);
       __syncwarp();  // tcgen05.ld is warp-collective: reconverge after the polling loop
       if (!ok) { *abort_flag = 1; break; }
@@ -243,9 +268,7 @@ __global__ void __launch_bounds__(kUmmaThreads, 1) indexer_umma_kernel(
       }
       sm100::tc_fence_before();
       sm100::mbar_arrive(&accempty[acc]);
-      const int t = c.tile * kUmmaTile + row;
       if (t < c.L) {
-        const int phys = block_table[(size_t)c.b * max_pages + t / page_size];
         if (phys < 0 || phys >= num_pages) {
           raise_error(SD_DEVERR_PAGE);
           s = INT32_MIN;

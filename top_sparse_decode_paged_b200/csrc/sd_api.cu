@@ -15,6 +15,7 @@
 #include "indexer_dp4a.cuh"
 #include "indexer_umma.cuh"
 #include "sd_common.cuh"
+#include "topk_cluster.cuh"
 #include "topk_radix.cuh"
 
 namespace {
@@ -198,6 +199,43 @@ sd_status launch_indexer_umma(const int8_t* qi, const int32_t* w, const int8_t* 
   return after_launch();
 }
 
+// Top-k: one thread-block cluster per row when the row fits in the cluster's
+// shared memory (max_seqlen <= 8 x 16384), else one CTA per row over L2.
+sd_status launch_topk(const int32_t* scores, const int32_t* seqlens, int32_t* indices, int B, int G,
+                      int max_seqlen, int cap, int k, cudaStream_t st) {
+  const int cs = sd::topk_cluster_size(max_seqlen);
+  const int rows = B * G;
+  stage_mark(kStageTopk, 0, st);
+  if (cs > 0 && rows <= 65535) {
+    const size_t smem = sizeof(sd::TopkClusterSmem);
+    sd_status s = cuda_check(cudaFuncSetAttribute(sd::topk_cluster_kernel,
+                                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                  static_cast<int>(smem)));
+    if (s != SD_OK) return s;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(cs, rows, 1);
+    cfg.blockDim = dim3(sd::kTkThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = cs;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    s = cuda_check(cudaLaunchKernelEx(&cfg, sd::topk_cluster_kernel, scores, seqlens, indices, G,
+                                      std::max(max_seqlen, 1), cap, k));
+    stage_mark(kStageTopk, 1, st);
+    ++t_launches;
+    return s;
+  }
+  sd::topk_radix_kernel<<<rows, sd::kTopkThreads, 0, st>>>(scores, seqlens, indices, G,
+                                                           std::max(max_seqlen, 1), cap, k);
+  stage_mark(kStageTopk, 1, st);
+  return after_launch();
+}
+
 sd_status launch_indexer_topk(const int8_t* qi, const int32_t* w, const int8_t* ki, const int32_t* bt,
                               const int32_t* seqlens, const sd_paged_desc& pd, int B, int Hi, int Di,
                               int max_seqlen, int k, int32_t* indices, int32_t* scores,
@@ -217,11 +255,7 @@ sd_status launch_indexer_topk(const int8_t* qi, const int32_t* w, const int8_t* 
     if (s != SD_OK) return s;
   }
   const int cap = std::min(max_seqlen, pd.max_pages_per_req * pd.page_size);
-  stage_mark(kStageTopk, 0, st);
-  sd::topk_radix_kernel<<<B * G, sd::kTopkThreads, 0, st>>>(scores, seqlens, indices, G,
-                                                             std::max(max_seqlen, 1), cap, k);
-  stage_mark(kStageTopk, 1, st);
-  return after_launch();
+  return launch_topk(scores, seqlens, indices, B, G, max_seqlen, cap, k, st);
 }
 
 template <int DK, int DV, int MT>

@@ -114,7 +114,9 @@ sd_status sd_indexer_topk(const int8_t* qi, const int32_t* w, const int8_t* ki_p
  *   q        bf16 [B, H, Dk]
  *   k_pages  bf16 [num_pages, page_size, G, Dk]
  *   v_pages  bf16 [num_pages, page_size, G, Dv], or NULL: V = K row[:Dv]
- *   indices  int32 [B, G, k] request-local tokens; entries < 0 are skipped
+ *   indices  int32 [B, G, k] request-local tokens. Only the first min(k, seqlens[b])
+ *            slots of a row are read (a selection has at most seqlen distinct
+ *            tokens, so it fits there); entries < 0 in them are skipped
  *   scale    softmax scale applied to q . K
  *   out      bf16 [B, H, Dv] OUT (round to nearest even); zero when nothing is selected
  *   lse      fp32 [B, H] OUT, nullable: natural-log sum of exp(scale * q . K_j),

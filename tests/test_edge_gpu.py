@@ -176,3 +176,64 @@ def test_topk_cluster_slices_with_ragged_rows():
 def test_topk_single_cta_fallback_beyond_cluster_capacity():
     """max_seqlen above 8 x 16384 takes the one-CTA-per-row kernel."""
     _indices_vs_oracle(W.make(W.spec("b4_l4096_mla", seqlens=(131073, 5000), seed=43)))
+
+
+def test_h128_k_at_least_seqlen_equals_dense_and_empty_request():
+    """128-head MLA rows (tensor-core attention path) with k >= seqlen, an
+    empty request in the middle, and requests shorter than one 256-token tile."""
+    sd = _sd()
+    wl = W.make(W.spec("b32_l65536_mla", seqlens=(2048, 300, 0, 1, 1999), seed=44))
+    got = run_step(wl, to_device(wl))
+    live = [b for b in range(5) if wl.seqlens[b] > 0]
+    dense, lse = oracle.dense_attention(wl.q, wl.k_pages, None, 512, wl.block_table, wl.seqlens, 1,
+                                        wl.spec.scale, requests=live)
+    assert_out_close(got["out"][live], dense, "dense h128")
+    np.testing.assert_allclose(got["lse"][live], lse, rtol=0, atol=2e-3)
+    assert (got["out"][2] == 0).all() and np.isneginf(got["lse"][2]).all()
+    assert (got["indices"][2] == -1).all()
+    assert sd.device_errors() == 0
+
+
+def test_h128_single_selected_row_is_exact():
+    wl = W.make(W.spec("b32_l65536_mla", seqlens=(3000, 700), k=1, seed=45))
+    got = run_step(wl, to_device(wl))
+    ref = oracle.decode_step(wl)
+    assert np.array_equal(got["indices"][:, :, :1], np.stack(ref["indices"]))
+    assert np.array_equal(got["out"], ref["out"])
+
+
+def test_h128_graph_replay_many_ranges():
+    """A captured 128-head step replayed with new queries; every CTA pair of
+    the attention covers parts of several requests (B=40 > 74 ranges / 2)."""
+    import torch
+    import top_sparse_decode_paged_b200 as sd
+    wl = W.make(W.spec("b32_l65536_mla", B=40, seqlen=3000, seed=46))
+    d = to_device(wl)
+    s = wl.spec
+    ws = sd.alloc_workspace(40, 1, wl.max_seqlen, s.k, s.H, s.Dv)
+    idx = torch.empty((40, 1, s.k), dtype=torch.int32, device="cuda")
+    out = torch.empty((40, s.H, s.Dv), dtype=torch.bfloat16, device="cuda")
+    run = lambda: sd.sd_decode_step(d["qi"], d["w"], d["ki_pages"], d["q"], d["k_pages"], None,  # noqa: E731
+                                    d["block_table"], d["seqlens"], s.k, wl.max_seqlen, s.scale, s.Dv,
+                                    indices=idx, out=out, workspace=ws)
+    stream = torch.cuda.Stream()
+    with torch.cuda.stream(stream):
+        run()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        run()
+    wl2 = W.make(W.spec("b32_l65536_mla", B=40, seqlen=3000, seed=47))
+    d2 = to_device(wl2)
+    for key in ("qi", "w", "q"):
+        d[key].copy_(d2[key])
+    g.replay()
+    torch.cuda.synchronize()
+    import dataclasses
+    mixed = dataclasses.replace(wl, qi=wl2.qi, w=wl2.w, q=wl2.q)
+    req = [0, 13, 39]
+    ref = oracle.decode_step(mixed, requests=req)
+    got_idx = idx.cpu().numpy()
+    for i, b in enumerate(req):
+        assert np.array_equal(got_idx[b], ref["indices"][i])
+    assert_out_close(out.float().cpu().numpy()[req], ref["out"], "graph h128")

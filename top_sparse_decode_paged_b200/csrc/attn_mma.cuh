@@ -78,7 +78,7 @@ __global__ void __launch_bounds__(AttnMmaCfg<DK, DV, MT>::THREADS) attn_split_mm
   const int nh = min(HB, qpk - hb * HB);          // valid heads in this block
   const int L = checked_seqlen(seqlens, b, seqlen_cap);
   const int slot0 = split * slots_per_split;
-  const int slot1 = min(k, slot0 + slots_per_split);
+  const int slot1 = min(min(k, L), slot0 + slots_per_split);  // only the first min(k, L) slots are read
   const int ntiles = slot1 > slot0 ? ceil_div(slot1 - slot0, kAttnTile) : 0;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int mt = warp >> 2;   // m16 tile of this warp

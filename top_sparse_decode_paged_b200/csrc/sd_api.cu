@@ -12,6 +12,7 @@
 
 #include "../../include/sd_api.h"
 #include "attn_mma.cuh"
+#include "attn_umma.cuh"
 #include "indexer_dp4a.cuh"
 #include "indexer_umma.cuh"
 #include "sd_common.cuh"
@@ -75,10 +76,17 @@ size_t scores_bytes(int B, int G, int max_seqlen) {
   return align_up(sizeof(int32_t) * (size_t)B * G * (size_t)max_seqlen);
 }
 
+// The tensor-core MLA attention serves the 128-head, 576/512 latent-row shape.
+bool umma_attn_fits(int G, int H, int Dk, int Dv, bool v_separate) {
+  return !v_separate && G == 1 && H == sd::kAuHeads && Dk == sd::kAuDk && Dv == sd::kAuDv;
+}
+
 size_t attn_bytes(int B, int G, int H, int k, int Dv) {
   const AttnPlan p = attn_plan(B, G, H, k);
   const size_t n = (size_t)B * H * p.n_splits;
-  return align_up(sizeof(float) * n * Dv) + align_up(sizeof(float2) * n);
+  size_t bytes = align_up(sizeof(float) * n * Dv) + align_up(sizeof(float2) * n);
+  if (G == 1 && H == sd::kAuHeads && Dv == sd::kAuDv) bytes = std::max(bytes, align_up(sd::attn_umma_workspace(B)));
+  return bytes;
 }
 
 bool ws_ok(const void* ws, size_t have, size_t need) {
@@ -158,6 +166,21 @@ bool encode_rows128(CUtensorMap* map, const void* base, uint64_t rows, uint32_t 
   const cuuint32_t box[2] = {128, box_rows};
   const cuuint32_t estride[2] = {1, 1};
   return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estride,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// A 2-D bf16 map (row-major, `row_bytes` apart) with boxes of box_cols x box_rows
+// and 128-byte swizzle; box_cols * 2 must be 128.
+bool encode_bf16_rows(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows, uint64_t row_bytes,
+                      uint32_t box_cols, uint32_t box_rows) {
+  EncodeTiledFn fn = encode_tiled_fn();
+  if (fn == nullptr || (reinterpret_cast<uintptr_t>(base) & 15u) != 0 || (row_bytes & 15u) != 0) return false;
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {row_bytes};
+  const cuuint32_t box[2] = {box_cols, box_rows};
+  const cuuint32_t estride[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estride,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -287,11 +310,45 @@ sd_status launch_attn_t(const uint16_t* q, const uint16_t* kp, const uint16_t* v
   return after_launch();
 }
 
+sd_status launch_attn_umma(const uint16_t* q, const uint16_t* kp, const int32_t* bt, const int32_t* seqlens,
+                           const int32_t* indices, const sd_paged_desc& pd, int B, int k, float scale,
+                           uint16_t* out, float* lse, void* ws, int seqlen_cap, cudaStream_t st) {
+  using Lay = sd::AttnUmmaLayout;
+  const size_t slots = static_cast<size_t>(sd::kAuRanges) + B;
+  float* part_o = static_cast<float*>(ws);
+  float2* part_ml = reinterpret_cast<float2*>(
+      static_cast<char*>(ws) + align_up(slots * 2 * sd::kAuHeads * (sd::kAuDv / 2) * sizeof(float)));
+  CUtensorMap tm_q, tm_kv;
+  const uint64_t rows = (uint64_t)pd.num_pages * pd.page_size;
+  if (!encode_bf16_rows(&tm_q, q, sd::kAuDk, (uint64_t)B * sd::kAuHeads, sd::kAuDk * 2, 64, sd::kAuHeads) ||
+      !encode_bf16_rows(&tm_kv, kp, sd::kAuDk, rows, sd::kAuDk * 2, 64, 1) || rows >= (1ull << 31))
+    return SD_ERR_UNSUPPORTED;
+  sd_status s = cuda_check(cudaFuncSetAttribute(sd::attn_mla_umma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                static_cast<int>(Lay::kSmemAlloc)));
+  if (s != SD_OK) return s;
+  const float scale_log2 = scale * 1.4426950408889634f;
+  stage_mark(kStageAttn, 0, st);
+  sd::attn_mla_umma_kernel<<<2 * sd::kAuRanges, sd::kAuThreads, Lay::kSmemAlloc, st>>>(
+      tm_q, tm_kv, reinterpret_cast<const __nv_bfloat16*>(kp), bt, seqlens, indices, B, k, pd.num_pages,
+      pd.page_size, pd.max_pages_per_req, seqlen_cap, scale_log2, part_o, part_ml);
+  stage_mark(kStageAttn, 1, st);
+  if ((s = after_launch()) != SD_OK) return s;
+  stage_mark(kStageCombine, 0, st);
+  sd::attn_mla_umma_combine_kernel<<<B * sd::kAuHeads, 128, 0, st>>>(
+      part_o, part_ml, seqlens, B, k, seqlen_cap, sd::kAuRanges, reinterpret_cast<__nv_bfloat16*>(out), lse);
+  stage_mark(kStageCombine, 1, st);
+  return after_launch();
+}
+
 sd_status launch_attn(const uint16_t* q, const uint16_t* kp, const uint16_t* vp, const int32_t* bt,
                       const int32_t* seqlens, const int32_t* indices, const sd_paged_desc& pd, int B,
                       int H, int Dk, int Dv, int k, float scale, uint16_t* out, float* lse,
                       void* ws, int seqlen_cap, cudaStream_t st) {
   if (B == 0) return SD_OK;
+  if (umma_attn_fits(pd.kv_heads, H, Dk, Dv, vp != nullptr)) {
+    const sd_status su = launch_attn_umma(q, kp, bt, seqlens, indices, pd, B, k, scale, out, lse, ws, seqlen_cap, st);
+    if (su != SD_ERR_UNSUPPORTED) return su;  // else: pointers the TMA cannot map; take the mma.sync kernel
+  }
   const AttnPlan p = attn_plan(B, pd.kv_heads, H, k);
   const size_t n = (size_t)B * H * p.n_splits;
   float* part_o = static_cast<float*>(ws);

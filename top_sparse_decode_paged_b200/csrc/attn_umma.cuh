@@ -14,12 +14,13 @@
 // K = 576); each then runs O += P V over its half (A = P from tensor memory,
 // B = V from shared memory).
 //
-// Data movement: Q (128 x 576 bf16, 147 KB) arrives by TMA and stays in shared
-// memory as nine 64-column tiles in the 128-byte-swizzled K-major layout.
-// Selected rows are gathered by four copy warps with coalesced cp.async (8 lanes
-// per 128-byte row piece, destination swizzle applied per 16-byte lane; skipped
-// selections copy zeros) into a two-slot ring of 32 KB chunks (256 tokens x 64
-// columns). A TMA tile::gather4 gather measured well below this on the part: it
+// Data movement: a four-slot ring of 48 KB slots. For each of the nine S steps
+// of a tile, a slot receives Q[:, 64 columns] (16 KB, one TMA tile; Q stays in
+// L2) and the tile's K[:, same columns] (32 KB, 256 rows x 128 bytes, gathered
+// by four copy warps with coalesced cp.async: 8 lanes per 128-byte row piece,
+// destination swizzle applied per 16-byte lane, skipped selections copy zeros).
+// The four V chunks of this CTA's half use the gather part of a slot. Keeping
+// Q out of shared memory is what buys the ring depth. A TMA tile::gather4 gather measured well below this on the part: it
 // moves one 128-byte row piece per ~20 cycles per SM. Each tile streams the nine K
 // chunks for S, then the four V chunks of this CTA's half; the same chunk
 // layout serves as the K-major B of S and as the MN-major B of P V. Whole rows
@@ -48,18 +49,20 @@ constexpr int kAuHeads = 128;              // M
 constexpr int kAuDk = 576, kAuDv = 512;
 constexpr int kAuQChunks = kAuDk / 64;     // 9
 constexpr int kAuVChunks = kAuDv / 2 / 64; // 4 per value half
-constexpr int kAuChunkBytes = kAuTile * 128;   // 32 KB
-constexpr int kAuQChunkBytes = kAuHeads * 128; // 16 KB
+constexpr int kAuChunkBytes = kAuTile * 128;   // 32 KB: 256 rows x 64 columns
+constexpr int kAuQChunkBytes = kAuHeads * 128; // 16 KB: 128 heads x 64 columns
+constexpr int kAuSlotBytes = kAuQChunkBytes + kAuChunkBytes;  // one ring slot
+constexpr int kAuSlots = 4;
 constexpr int kAuThreads = 288;
 constexpr int kAuRanges = 74;              // CTA pairs: 148 CTAs, one per SM
 constexpr float kAuRescaleLog2 = 8.0f;     // lazy rescale threshold (log2 units)
 constexpr int kAuPrefetchTiles = 3;       // L2 prefetch distance (tiles)
+constexpr int kMaxTopK = 2048;            // largest k the library accepts
 
 struct AttnUmmaLayout {
-  static constexpr int kOffQ = 0;
-  static constexpr int kOffRing = kAuQChunks * kAuQChunkBytes;      // 147456
-  static constexpr int kOffBar = kOffRing + 2 * kAuChunkBytes;      // 212992
-  static constexpr int kNumBars = 9;
+  static constexpr int kOffRing = 0;
+  static constexpr int kOffBar = kAuSlots * kAuSlotBytes;           // 196608
+  static constexpr int kNumBars = 2 * kAuSlots + 3;
   static constexpr int kOffMask = kOffBar + 8 * kNumBars;
   static constexpr int kOffMisc = kOffMask + 2 * 8 * 4;
   static constexpr int kBytes = kOffMisc + 16;
@@ -133,16 +136,13 @@ __global__ void __launch_bounds__(kAuThreads, 1) attn_mla_umma_kernel(
   extern __shared__ uint8_t smem_dyn[];
   const uint32_t raw = smem_u32(smem_dyn);
   uint8_t* smem = smem_dyn + (((raw + 1023u) & ~1023u) - raw);
-  uint8_t* sq = smem + Lay::kOffQ;
   uint8_t* ring = smem + Lay::kOffRing;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::kOffBar);
-  uint64_t* chunk_full = bars;       // [2], 128 copy-thread arrivals
-  uint64_t* chunk_empty = bars + 2;  // [2], MMA commit
-  uint64_t* q_full = bars + 4;       // TMA bytes
-  uint64_t* q_empty = bars + 5;      // MMA commit after a request's last S
-  uint64_t* s_full = bars + 6;       // MMA commit
-  uint64_t* p_full = bars + 7;       // 128 softmax arrivals
-  uint64_t* pv_done = bars + 8;      // MMA commit
+  uint64_t* chunk_full = bars;                   // [kAuSlots]: 128 copy arrivals + 1 TMA issuer
+  uint64_t* chunk_empty = bars + kAuSlots;       // [kAuSlots]: MMA commit
+  uint64_t* s_full = bars + 2 * kAuSlots;        // MMA commit
+  uint64_t* p_full = bars + 2 * kAuSlots + 1;    // 128 softmax arrivals
+  uint64_t* pv_done = bars + 2 * kAuSlots + 2;   // MMA commit
   uint32_t* mask_words = reinterpret_cast<uint32_t*>(smem + Lay::kOffMask);  // [2][8]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Lay::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Lay::kOffMisc + 4);
@@ -153,12 +153,10 @@ __global__ void __launch_bounds__(kAuThreads, 1) attn_mla_umma_kernel(
   const int half = blockIdx.x / n_ranges;  // which 256 value columns this CTA owns
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < 2; ++i) {
-      sm100::mbar_init(&chunk_full[i], 128);
+    for (int i = 0; i < kAuSlots; ++i) {
+      sm100::mbar_init(&chunk_full[i], 129);
       sm100::mbar_init(&chunk_empty[i], 1);
     }
-    sm100::mbar_init(q_full, 1);
-    sm100::mbar_init(q_empty, 1);
     sm100::mbar_init(s_full, 1);
     sm100::mbar_init(p_full, 128);
     sm100::mbar_init(pv_done, 1);
@@ -186,31 +184,20 @@ __global__ void __launch_bounds__(kAuThreads, 1) attn_mla_umma_kernel(
 
   if (warp < 4) {
     // ------------------------------ copies ------------------------------
-    // Q arrives by TMA (nine 16 KB tiles). Selected rows are gathered with
-    // cp.async, coalesced: in each copy instruction 8 lanes fetch one 128-byte
-    // row piece, so a warp moves 4 whole pieces (512 B); the 16-byte swizzle
-    // of the destination is applied per lane. Thread pt fetches rows
+    // Each S chunk c of a tile fills one ring slot with Q[:, 64c..64c+63] (a
+    // 16 KB TMA tile; Q is small and stays in L2) and the tile's K[:, 64c..]
+    // (32 KB gathered with cp.async). A V chunk fills the gather part only.
+    // The gather is coalesced: in each copy instruction 8 lanes fetch one
+    // 128-byte row piece, so a warp moves 4 pieces (512 B); the 16-byte
+    // swizzle of the destination is applied per lane. Thread pt fetches rows
     // 64*warp + 4*i + lane/8 (i = 0..15), 16-byte column j = lane % 8.
     const int pt = threadIdx.x;  // 0..127
     const int jseg = lane & 7;
     AttnCursor c;
     c.init(seqlens, B, seqlen_cap, k, first, count);
     long long n = 0;  // ring uses
-    int nreq = 0, cur_b = -1;
     bool ok = true;
     while (c.valid() && ok) {
-      if (c.b != cur_b) {
-        if (pt == 0) {
-          ok = sm100::mbar_wait(q_empty, (nreq & 1) ^ 1);
-          if (ok) {
-            sm100::mbar_arrive_expect_tx(q_full, kAuQChunks * kAuQChunkBytes);
-            for (int cc = 0; cc < kAuQChunks; ++cc)
-              sm100::tma_load_2d(sq + cc * kAuQChunkBytes, &tm_q, q_full, cc * 64, c.b * kAuHeads);
-          }
-        }
-        cur_b = c.b;
-        ++nreq;
-      }
       const int kb = min(k, c.L);
       const int s0 = c.tile * kAuTile;
       int row[16];
@@ -238,11 +225,17 @@ __global__ void __launch_bounds__(kAuThreads, 1) attn_mla_umma_kernel(
         }
       }
       for (int ci = 0; ci < kAuQChunks + kAuVChunks && ok; ++ci, ++n) {
-        const int cc = ci < kAuQChunks ? ci : half * kAuVChunks + (ci - kAuQChunks);
-        const int slot = static_cast<int>(n & 1);
-        ok = sm100::mbar_wait(&chunk_empty[slot], static_cast<uint32_t>((n >> 1) & 1) ^ 1) && !*abort_flag;
+        const bool is_s = ci < kAuQChunks;
+        const int cc = is_s ? ci : half * kAuVChunks + (ci - kAuQChunks);
+        const int slot = static_cast<int>(n % kAuSlots);
+        ok = sm100::mbar_wait(&chunk_empty[slot], static_cast<uint32_t>((n / kAuSlots) & 1) ^ 1) && !*abort_flag;
         if (!ok) break;
-        uint8_t* dst_base = ring + slot * kAuChunkBytes;
+        uint8_t* slot_base = ring + slot * kAuSlotBytes;
+        if (pt == 0) {
+          sm100::mbar_arrive_expect_tx(&chunk_full[slot], is_s ? kAuQChunkBytes : 0);
+          if (is_s) sm100::tma_load_2d(slot_base, &tm_q, &chunk_full[slot], cc * 64, c.b * kAuHeads);
+        }
+        uint8_t* dst_base = slot_base + kAuQChunkBytes;
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
           const int r = 64 * warp + 4 * i + (lane >> 3);
@@ -382,24 +375,19 @@ __global__ void __launch_bounds__(kAuThreads, 1) attn_mla_umma_kernel(
       AttnCursor c;
       c.init(seqlens, B, seqlen_cap, k, first, count);
       long long n = 0;
-      int ntile = 0, nreq = 0, cur_b = -1;
+      int ntile = 0;
       bool seg_first = true;
       while (c.valid() && !*abort_flag) {
         bool ok = true;
-        if (c.b != cur_b) {
-          if (!sm100::mbar_wait(q_full, nreq & 1)) { *abort_flag = 1; break; }
-          ++nreq;
-          cur_b = c.b;
-        }
         // S = Q K^T over the nine 64-column chunks
         for (int cc = 0; cc < kAuQChunks && ok; ++cc, ++n) {
-          const int slot = static_cast<int>(n & 1);
-          ok = sm100::mbar_wait(&chunk_full[slot], static_cast<uint32_t>((n >> 1) & 1));
+          const int slot = static_cast<int>(n % kAuSlots);
+          ok = sm100::mbar_wait(&chunk_full[slot], static_cast<uint32_t>((n / kAuSlots) & 1));
           if (ok && cc == 0 && ntile > 0) ok = sm100::mbar_wait(pv_done, (ntile - 1) & 1);
           if (!ok) break;
           sm100::tc_fence_after();
-          const uint32_t a0 = smem_u32(sq + cc * kAuQChunkBytes);
-          const uint32_t b0 = smem_u32(ring + slot * kAuChunkBytes);
+          const uint32_t a0 = smem_u32(ring + slot * kAuSlotBytes);
+          const uint32_t b0 = a0 + kAuQChunkBytes;
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
             sm100::mma_bf16_ss(tm_s, sm100::smem_desc_k_sw128(a0 + 32 * kk), sm100::smem_desc_k_sw128(b0 + 32 * kk),
@@ -411,16 +399,15 @@ __global__ void __launch_bounds__(kAuThreads, 1) attn_mla_umma_kernel(
         const int this_b = c.b;
         c.next(seqlens, B, seqlen_cap, k);
         const bool last_of_req = !c.valid() || c.b != this_b;
-        if (last_of_req) sm100::mma_commit(q_empty);
         // O += P V over this CTA's four value chunks
         if (!sm100::mbar_wait(p_full, ntile & 1)) { *abort_flag = 1; break; }
         sm100::tc_fence_after();
         for (int v = 0; v < kAuVChunks && ok; ++v, ++n) {
-          const int slot = static_cast<int>(n & 1);
-          ok = sm100::mbar_wait(&chunk_full[slot], static_cast<uint32_t>((n >> 1) & 1));
+          const int slot = static_cast<int>(n % kAuSlots);
+          ok = sm100::mbar_wait(&chunk_full[slot], static_cast<uint32_t>((n / kAuSlots) & 1));
           if (!ok) break;
           sm100::tc_fence_after();
-          const uint32_t b0 = smem_u32(ring + slot * kAuChunkBytes);
+          const uint32_t b0 = smem_u32(ring + slot * kAuSlotBytes + kAuQChunkBytes);
 #pragma unroll
           for (int i = 0; i < kAuTile / 16; ++i)
             sm100::mma_bf16_ts(tm_o + 64 * v, tm_s + 8 * i,
@@ -446,56 +433,64 @@ __global__ void __launch_bounds__(kAuThreads, 1) attn_mla_umma_kernel(
 }
 
 // Merges the per-range partials of one (request, head) into the bf16 output.
+// A request has at most ceil(k / 256) tiles and so at most that many covering
+// ranges; the loops over them are unrolled so that all their (m, l) loads,
+// then all their partial loads, are in flight together.
+constexpr int kAuMaxSeg = kMaxTopK / kAuTile;
+
 __global__ void __launch_bounds__(128) attn_mla_umma_combine_kernel(
     const float* __restrict__ part_o, const float2* __restrict__ part_ml, const int32_t* __restrict__ seqlens,
     int B, int k, int seqlen_cap, int n_ranges, __nv_bfloat16* __restrict__ out, float* __restrict__ lse) {
   const int b = blockIdx.x / kAuHeads, h = blockIdx.x % kAuHeads;
-  long long start = 0, total = 0;
-  int tiles_b = 0;
+  uint32_t start = 0, total = 0, tiles_b = 0;
   for (int i = 0; i < B; ++i) {
     int L = seqlens[i];
     L = L < 0 ? 0 : (L > seqlen_cap ? seqlen_cap : L);
-    const int n = ceil_div(min(k, L), kAuTile);
+    const uint32_t n = static_cast<uint32_t>(ceil_div(min(k, L), kAuTile));
     if (i < b) start += n;
     if (i == b) tiles_b = n;
     total += n;
   }
-  const long long end = start + tiles_b;
-  // range r (tiles [total*r/n, total*(r+1)/n)) wrote a partial for request b
-  // iff it overlaps [start, end); those ranges form the interval [r_lo, r_hi]
-  auto covers = [&](int r) {
-    const long long f = total * r / n_ranges, e = total * (r + 1) / n_ranges;
-    return max(f, start) < min(e, end);
-  };
-  int r_lo = 0, r_hi = -1;
-  if (end > start) {
-    r_lo = static_cast<int>(max(0LL, ((start + 1) * n_ranges + total - 1) / total - 1));
-    r_hi = static_cast<int>(min((long long)n_ranges - 1, (end * n_ranges + total - 1) / total - 1));
-  }
+  const uint32_t nr = static_cast<uint32_t>(n_ranges);
+  // Tile i of the list lies in range ((i + 1) * nr - 1) / total (range r holds
+  // tiles [total*r/nr, total*(r+1)/nr)); the request's tiles are consecutive,
+  // so their ranges are found in order, each once.
+  int seg_r[kAuMaxSeg];
+  float m[kAuMaxSeg], l[kAuMaxSeg];
   float M = -INFINITY;
-  for (int r = r_lo; r <= r_hi; ++r)
-    if (covers(r)) M = fmaxf(M, part_ml[((size_t)r + b) * kAuHeads + h].x);
-  float denom = 0.f;
-  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  uint32_t prev = 0xffffffffu;
+#pragma unroll
+  for (int j = 0; j < kAuMaxSeg; ++j) {
+    const uint32_t i = start + j;
+    const uint32_t r = j < static_cast<int>(tiles_b) ? ((i + 1) * nr - 1) / total : 0xffffffffu;
+    const bool fresh = r != 0xffffffffu && r != prev;
+    prev = r;
+    seg_r[j] = fresh ? static_cast<int>(r) : -1;
+    const float2 ml = fresh ? part_ml[((size_t)r + b) * kAuHeads + h] : make_float2(-INFINITY, 0.f);
+    m[j] = ml.x;
+    l[j] = ml.y;
+    M = fmaxf(M, ml.x);
+  }
   const int d0 = 4 * threadIdx.x;            // value columns d0..d0+3
   const int hf = d0 / (kAuDv / 2), dl = d0 % (kAuDv / 2);
-  for (int r = r_lo; r <= r_hi; ++r) {
-    if (!covers(r)) continue;
-    const size_t slot = static_cast<size_t>(r) + b;
-    const float2 ml = part_ml[slot * kAuHeads + h];
-    if (ml.x == -INFINITY) continue;
-    const float wgt = exp2f(ml.x - M);
-    denom += wgt * ml.y;
+  float denom = 0.f;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+  for (int j = 0; j < kAuMaxSeg; ++j) {
+    if (seg_r[j] < 0 || m[j] == -INFINITY) continue;
+    const size_t slot = static_cast<size_t>(seg_r[j]) + b;
+    const float wgt = exp2f(m[j] - M);
+    denom += wgt * l[j];
     const float4 o = *reinterpret_cast<const float4*>(part_o + ((slot * 2 + hf) * kAuHeads + h) * (kAuDv / 2) + dl);
-    acc[0] += wgt * o.x;
-    acc[1] += wgt * o.y;
-    acc[2] += wgt * o.z;
-    acc[3] += wgt * o.w;
+    acc.x += wgt * o.x;
+    acc.y += wgt * o.y;
+    acc.z += wgt * o.z;
+    acc.w += wgt * o.w;
   }
   const float inv = denom > 0.f ? 1.f / denom : 0.f;
-  __nv_bfloat16* o = out + ((size_t)b * kAuHeads + h) * kAuDv + d0;
-#pragma unroll
-  for (int i = 0; i < 4; ++i) o[i] = __float2bfloat16_rn(acc[i] * inv);
+  __nv_bfloat162* o2 = reinterpret_cast<__nv_bfloat162*>(out + ((size_t)b * kAuHeads + h) * kAuDv + d0);
+  o2[0] = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
+  o2[1] = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
   if (lse != nullptr && threadIdx.x == 0)
     lse[(size_t)b * kAuHeads + h] = denom > 0.f ? (M + log2f(denom)) * 0.69314718055994530942f : -INFINITY;
 }

@@ -432,67 +432,82 @@ __global__ void __launch_bounds__(kAuThreads, 1) attn_mla_umma_kernel(
   }
 }
 
-// Merges the per-range partials of one (request, head) into the bf16 output.
-// A request has at most ceil(k / 256) tiles and so at most that many covering
-// ranges; the loops over them are unrolled so that all their (m, l) loads,
-// then all their partial loads, are in flight together.
+// Merges the per-range partials into the bf16 output. One block per (request,
+// group of 8 heads): warp 0 finds the request's segments once (a request has
+// at most ceil(k / 256) tiles, hence at most that many covering ranges: tile i
+// of the list lies in range ((i + 1) * n_ranges - 1) / total), the (m, l) of
+// 8 heads x those segments are staged in shared memory, and each thread merges
+// 4 value columns of all 8 heads, its partial loads all in flight together.
 constexpr int kAuMaxSeg = kMaxTopK / kAuTile;
+constexpr int kAuCombineHeads = 8;
 
 __global__ void __launch_bounds__(128) attn_mla_umma_combine_kernel(
     const float* __restrict__ part_o, const float2* __restrict__ part_ml, const int32_t* __restrict__ seqlens,
     int B, int k, int seqlen_cap, int n_ranges, __nv_bfloat16* __restrict__ out, float* __restrict__ lse) {
-  const int b = blockIdx.x / kAuHeads, h = blockIdx.x % kAuHeads;
-  uint32_t start = 0, total = 0, tiles_b = 0;
-  for (int i = 0; i < B; ++i) {
-    int L = seqlens[i];
-    L = L < 0 ? 0 : (L > seqlen_cap ? seqlen_cap : L);
-    const uint32_t n = static_cast<uint32_t>(ceil_div(min(k, L), kAuTile));
-    if (i < b) start += n;
-    if (i == b) tiles_b = n;
-    total += n;
-  }
-  const uint32_t nr = static_cast<uint32_t>(n_ranges);
-  // Tile i of the list lies in range ((i + 1) * nr - 1) / total (range r holds
-  // tiles [total*r/nr, total*(r+1)/nr)); the request's tiles are consecutive,
-  // so their ranges are found in order, each once.
-  int seg_r[kAuMaxSeg];
-  float m[kAuMaxSeg], l[kAuMaxSeg];
-  float M = -INFINITY;
-  uint32_t prev = 0xffffffffu;
+  constexpr int HG = kAuHeads / kAuCombineHeads;
+  const int b = blockIdx.x / HG;
+  const int h0 = (blockIdx.x % HG) * kAuCombineHeads;
+  __shared__ int seg_r[kAuMaxSeg];
+  __shared__ float2 ml_s[kAuCombineHeads][kAuMaxSeg];
+  const int tid = threadIdx.x, lane = tid & 31;
+  if (tid < 32) {
+    uint32_t before = 0, total = 0, mine = 0;
+    for (int i = lane; i < B; i += 32) {
+      int L = seqlens[i];
+      L = L < 0 ? 0 : (L > seqlen_cap ? seqlen_cap : L);
+      const uint32_t n = static_cast<uint32_t>(ceil_div(min(k, L), kAuTile));
+      before += i < b ? n : 0;
+      mine += i == b ? n : 0;
+      total += n;
+    }
 #pragma unroll
-  for (int j = 0; j < kAuMaxSeg; ++j) {
-    const uint32_t i = start + j;
-    const uint32_t r = j < static_cast<int>(tiles_b) ? ((i + 1) * nr - 1) / total : 0xffffffffu;
-    const bool fresh = r != 0xffffffffu && r != prev;
-    prev = r;
-    seg_r[j] = fresh ? static_cast<int>(r) : -1;
-    const float2 ml = fresh ? part_ml[((size_t)r + b) * kAuHeads + h] : make_float2(-INFINITY, 0.f);
-    m[j] = ml.x;
-    l[j] = ml.y;
-    M = fmaxf(M, ml.x);
+    for (int o = 16; o > 0; o >>= 1) {
+      before += __shfl_xor_sync(0xffffffffu, before, o);
+      total += __shfl_xor_sync(0xffffffffu, total, o);
+      mine += __shfl_xor_sync(0xffffffffu, mine, o);
+    }
+    const uint32_t nr = static_cast<uint32_t>(n_ranges);
+    const uint32_t r = lane < static_cast<int>(mine) ? ((before + lane + 1) * nr - 1) / total : 0xffffffffu;
+    const uint32_t prev = __shfl_up_sync(0xffffffffu, r, 1);
+    if (lane < kAuMaxSeg) seg_r[lane] = (r != 0xffffffffu && (lane == 0 || r != prev)) ? static_cast<int>(r) : -1;
   }
-  const int d0 = 4 * threadIdx.x;            // value columns d0..d0+3
+  __syncthreads();
+  if (tid < kAuCombineHeads * kAuMaxSeg) {
+    const int hh = tid / kAuMaxSeg, j = tid % kAuMaxSeg;
+    const int r = seg_r[j];
+    ml_s[hh][j] = r >= 0 ? part_ml[((size_t)r + b) * kAuHeads + h0 + hh] : make_float2(-INFINITY, 0.f);
+  }
+  __syncthreads();
+  const int d0 = 4 * tid;  // value columns d0..d0+3
   const int hf = d0 / (kAuDv / 2), dl = d0 % (kAuDv / 2);
-  float denom = 0.f;
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 2
+  for (int hh = 0; hh < kAuCombineHeads; ++hh) {
+    const int h = h0 + hh;
+    float M = -INFINITY;
 #pragma unroll
-  for (int j = 0; j < kAuMaxSeg; ++j) {
-    if (seg_r[j] < 0 || m[j] == -INFINITY) continue;
-    const size_t slot = static_cast<size_t>(seg_r[j]) + b;
-    const float wgt = exp2f(m[j] - M);
-    denom += wgt * l[j];
-    const float4 o = *reinterpret_cast<const float4*>(part_o + ((slot * 2 + hf) * kAuHeads + h) * (kAuDv / 2) + dl);
-    acc.x += wgt * o.x;
-    acc.y += wgt * o.y;
-    acc.z += wgt * o.z;
-    acc.w += wgt * o.w;
+    for (int j = 0; j < kAuMaxSeg; ++j) M = fmaxf(M, ml_s[hh][j].x);
+    float denom = 0.f;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int j = 0; j < kAuMaxSeg; ++j) {
+      const float2 ml = ml_s[hh][j];
+      if (ml.x == -INFINITY) continue;
+      const size_t slot = static_cast<size_t>(seg_r[j]) + b;
+      const float wgt = exp2f(ml.x - M);
+      denom += wgt * ml.y;
+      const float4 o = *reinterpret_cast<const float4*>(part_o + ((slot * 2 + hf) * kAuHeads + h) * (kAuDv / 2) + dl);
+      acc.x += wgt * o.x;
+      acc.y += wgt * o.y;
+      acc.z += wgt * o.z;
+      acc.w += wgt * o.w;
+    }
+    const float inv = denom > 0.f ? 1.f / denom : 0.f;
+    __nv_bfloat162* o2 = reinterpret_cast<__nv_bfloat162*>(out + ((size_t)b * kAuHeads + h) * kAuDv + d0);
+    o2[0] = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
+    o2[1] = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
+    if (lse != nullptr && tid == 0)
+      lse[(size_t)b * kAuHeads + h] = denom > 0.f ? (M + log2f(denom)) * 0.69314718055994530942f : -INFINITY;
   }
-  const float inv = denom > 0.f ? 1.f / denom : 0.f;
-  __nv_bfloat162* o2 = reinterpret_cast<__nv_bfloat162*>(out + ((size_t)b * kAuHeads + h) * kAuDv + d0);
-  o2[0] = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
-  o2[1] = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
-  if (lse != nullptr && threadIdx.x == 0)
-    lse[(size_t)b * kAuHeads + h] = denom > 0.f ? (M + log2f(denom)) * 0.69314718055994530942f : -INFINITY;
 }
 
 inline size_t attn_umma_workspace(int B) {

@@ -222,33 +222,41 @@ sd_status launch_indexer_umma(const int8_t* qi, const int32_t* w, const int8_t* 
   return after_launch();
 }
 
+template <int PER>
+sd_status launch_topk_cluster(const int32_t* scores, const int32_t* seqlens, int32_t* indices, int rows, int G,
+                              int max_seqlen, int cap, int k, int cs, cudaStream_t st) {
+  const size_t smem = sizeof(sd::TopkClusterSmem<PER>);
+  sd_status s = cuda_check(cudaFuncSetAttribute(sd::topk_cluster_kernel<PER>,
+                                                cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)));
+  if (s != SD_OK) return s;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(cs, rows, 1);
+  cfg.blockDim = dim3(sd::kTkThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = cs;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cuda_check(cudaLaunchKernelEx(&cfg, sd::topk_cluster_kernel<PER>, scores, seqlens, indices, G,
+                                       std::max(max_seqlen, 1), cap, k));
+}
+
 // Top-k: one thread-block cluster per row when the row fits in the cluster's
-// shared memory (max_seqlen <= 8 x 16384), else one CTA per row over L2.
+// shared memory (max_seqlen <= 8 x 512 x 32), else one CTA per row over L2.
 sd_status launch_topk(const int32_t* scores, const int32_t* seqlens, int32_t* indices, int B, int G,
                       int max_seqlen, int cap, int k, cudaStream_t st) {
-  const int cs = sd::topk_cluster_size(max_seqlen);
   const int rows = B * G;
+  const int cs16 = sd::topk_cluster_size(max_seqlen, 16);
+  const int cs32 = sd::topk_cluster_size(max_seqlen, 32);
   stage_mark(kStageTopk, 0, st);
-  if (cs > 0 && rows <= 65535) {
-    const size_t smem = sizeof(sd::TopkClusterSmem);
-    sd_status s = cuda_check(cudaFuncSetAttribute(sd::topk_cluster_kernel,
-                                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                  static_cast<int>(smem)));
-    if (s != SD_OK) return s;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(cs, rows, 1);
-    cfg.blockDim = dim3(sd::kTkThreads, 1, 1);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = cs;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    s = cuda_check(cudaLaunchKernelEx(&cfg, sd::topk_cluster_kernel, scores, seqlens, indices, G,
-                                      std::max(max_seqlen, 1), cap, k));
+  if ((cs16 > 0 || cs32 > 0) && rows <= 65535) {
+    // 32 scores per thread measured faster than 16 (fewer CTAs per cluster)
+    const sd_status s = cs32 > 0 ? launch_topk_cluster<32>(scores, seqlens, indices, rows, G, max_seqlen, cap, k, cs32, st)
+                                 : launch_topk_cluster<16>(scores, seqlens, indices, rows, G, max_seqlen, cap, k, cs16, st);
     stage_mark(kStageTopk, 1, st);
     ++t_launches;
     return s;
@@ -334,7 +342,7 @@ sd_status launch_attn_umma(const uint16_t* q, const uint16_t* kp, const int32_t*
   stage_mark(kStageAttn, 1, st);
   if ((s = after_launch()) != SD_OK) return s;
   stage_mark(kStageCombine, 0, st);
-  sd::attn_mla_umma_combine_kernel<<<B * sd::kAuHeads, 128, 0, st>>>(
+  sd::attn_mla_umma_combine_kernel<<<B * (sd::kAuHeads / sd::kAuCombineHeads), 128, 0, st>>>(
       part_o, part_ml, seqlens, B, k, seqlen_cap, sd::kAuRanges, reinterpret_cast<__nv_bfloat16*>(out), lse);
   stage_mark(kStageCombine, 1, st);
   return after_launch();

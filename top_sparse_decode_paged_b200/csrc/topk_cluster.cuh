@@ -3,8 +3,9 @@
 // Same result as topk_radix_kernel (score descending, ties to the lower token,
 // output in ascending token order, -1 padded), organised for B200:
 //   - a row of L scores is split over a cluster of CS CTAs (CS <= 8); each CTA
-//     copies its slice (<= 16384 scores) once from L2 into shared memory and
-//     never touches global memory again until it writes its part of the output;
+//     copies its slice (512 threads x 16 or 32 scores) once from L2 into shared
+//     memory and never touches global memory again until it writes its part of
+//     the output;
 //   - a cluster-wide min/max fixes the highest bit in which the keys differ,
 //     so radix passes start there (for scores of one row that is ~22 bits:
 //     two 11-bit passes, not four 8-bit ones);
@@ -26,15 +27,15 @@ namespace sd {
 namespace cg = cooperative_groups;
 
 constexpr int kTkThreads = 512;
-constexpr int kTkPerThread = 32;                              // scores per thread
-constexpr int kTkSlice = kTkThreads * kTkPerThread;           // 16384 per CTA
 constexpr int kTkBinsBits = 11;
 constexpr int kTkBins = 1 << kTkBinsBits;
 constexpr int kTkMaxCluster = 8;
-constexpr int kTkChunkStride = kTkPerThread + 1;              // padded per-thread chunk (words)
 
+// PER: scores per thread (16 or 32); a CTA holds a slice of 512 * PER scores.
+template <int PER>
 struct TopkClusterSmem {
-  uint32_t keys[kTkThreads * kTkChunkStride];  // thread t's chunk at t*33 (bank-conflict free)
+  static constexpr int kStride = PER + 1;       // padded per-thread chunk (words)
+  uint32_t keys[kTkThreads * kStride];          // thread t's chunk at t*(PER+1) (bank-conflict free)
   uint32_t hist[kTkBins];                       // this CTA's histogram (read by the cluster)
   uint32_t total[kTkBins];                      // cluster-wide histogram
   uint32_t red[kTkThreads / 32 * 2 + 8];        // block reduction / scan scratch
@@ -96,11 +97,14 @@ __device__ __forceinline__ uint32_t tk_block_reduce(uint32_t v, uint32_t* scratc
   return v;
 }
 
-__global__ void __launch_bounds__(kTkThreads, 1) topk_cluster_kernel(
+template <int PER>
+__global__ void __launch_bounds__(kTkThreads, 2) topk_cluster_kernel(
     const int32_t* __restrict__ scores, const int32_t* __restrict__ seqlens, int32_t* __restrict__ indices,
     int G, int max_seqlen, int seqlen_cap, int k) {
+  constexpr int kTkPerThread = PER;
+  constexpr int kTkChunkStride = PER + 1;
   extern __shared__ __align__(16) uint8_t tk_smem_raw[];
-  TopkClusterSmem& sm = *reinterpret_cast<TopkClusterSmem*>(tk_smem_raw);
+  TopkClusterSmem<PER>& sm = *reinterpret_cast<TopkClusterSmem<PER>*>(tk_smem_raw);
   cg::cluster_group cluster = cg::this_cluster();
   const int CS = static_cast<int>(cluster.num_blocks());
   const int crank = static_cast<int>(cluster.block_rank());
@@ -123,6 +127,7 @@ __global__ void __launch_bounds__(kTkThreads, 1) topk_cluster_kernel(
 
   // ---- load this CTA's slice (coalesced), keep keys in padded per-thread chunks ----
   uint32_t kmin = 0xffffffffu, kmax = 0u;
+#pragma unroll
   for (int j = 0; j < kTkPerThread; ++j) {
     const int e = j * kTkThreads + tid;           // element within the slice
     uint32_t u = 0u;                               // past the slice: never read again
@@ -275,10 +280,13 @@ __global__ void __launch_bounds__(kTkThreads, 1) topk_cluster_kernel(
   cluster.sync();  // no CTA leaves while others may still read its shared memory
 }
 
-inline int topk_cluster_size(int max_seqlen) {
+// Cluster size for rows of up to max_seqlen scores with PER scores per thread
+// (0: does not fit in kTkMaxCluster CTAs).
+inline int topk_cluster_size(int max_seqlen, int per) {
+  const long long slice = (long long)kTkThreads * per;
   int cs = 1;
-  while (cs < kTkMaxCluster && (long long)cs * kTkSlice < max_seqlen) cs <<= 1;
-  return (long long)cs * kTkSlice >= max_seqlen ? cs : 0;  // 0: does not fit
+  while (cs < kTkMaxCluster && cs * slice < max_seqlen) cs <<= 1;
+  return cs * slice >= max_seqlen ? cs : 0;
 }
 
 }  // namespace sd

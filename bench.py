@@ -34,6 +34,15 @@ METRIC = "decode queries/s and achieved HBM GB/s (indexer+top-k+sparse attn), 1 
 DEFAULT_CONFIG = "b32_l65536_mla"
 L2_FLUSH_BYTES = 256 << 20
 
+# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of one launch,
+# from the ncu captures summarised in profiles/, keyed by (workload, stage).
+# Valid only for the library version they were taken on; any other version
+# reports traffic as null.
+NCU_TRAFFIC = {
+    ("b32_l65536_mla", "indexer"): (0x00000002, 269.063936e6 + 9.028864e6),
+    ("b32_l65536_mla", "attn"): (0x00000002, 104.638464e6 + 4.646656e6),
+}
+
 
 def _peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
@@ -215,29 +224,62 @@ def bench_ours(args, rank, world, local):
     launches_per_step = sd.last_launch_count()
     torch.cuda.synchronize()
 
-    timer = StageTimer()
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    stage_tot = dict.fromkeys(StageTimer.STAGES, 0.0)
+    graph = None
+    if not args.no_graph:
+        # capture one step, with the stage events inside it; replays re-record them
+        timer = StageTimer()
+        side = torch.cuda.Stream()
+        side.wait_stream(stream)
+        with torch.cuda.stream(side):
+            step()
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        timer.arm()
+        with torch.cuda.graph(graph, stream=side):
+            step()
+        StageTimer.disarm()
+        stage_events = timer._pairs[0]
+        for _ in range(args.warmup):
+            flush.zero_()
+            graph.replay()
+        torch.cuda.synchronize()
     if world > 1:
         import torch.distributed as dist
         dist.barrier()
     torch.cuda.synchronize()
     with ClockSampler(local if "CUDA_VISIBLE_DEVICES" not in os.environ else int(
             os.environ["CUDA_VISIBLE_DEVICES"].split(",")[local])) as clocks:
-        for i in range(args.steps):
-            flush.zero_()
-            timer.arm()
-            starts[i].record(stream)
-            step()
-            ends[i].record(stream)
+        if graph is not None:
+            for i in range(args.steps):
+                flush.zero_()
+                starts[i].record(stream)
+                graph.replay()
+                ends[i].record(stream)
+                ends[i].synchronize()  # the stage events inside the graph are read before the next replay
+                for j, name in enumerate(StageTimer.STAGES):
+                    stage_tot[name] += stage_events[2 * j].elapsed_time(stage_events[2 * j + 1])
+        else:
+            timer = StageTimer()
+            for i in range(args.steps):
+                flush.zero_()
+                timer.arm()
+                starts[i].record(stream)
+                step()
+                ends[i].record(stream)
+            torch.cuda.synchronize()
+            StageTimer.disarm()
+            stage_tot, _ = timer.totals_ms()
         torch.cuda.synchronize()
-        StageTimer.disarm()
         if world > 1:
             dist.barrier()
     step_ms = sum(a.elapsed_time(b) for a, b in zip(starts, ends)) / args.steps
-    stage_tot, n_rec = timer.totals_ms()
-    stage_ms = {k_: v / n_rec for k_, v in stage_tot.items()}
+    stage_ms = {k_: v / args.steps for k_, v in stage_tot.items()}
     step_ms = max_over_ranks(step_ms, world)
+    if graph is not None:
+        del graph
 
     # end to end through the public call: per-step queries H2D from pinned
     # host memory, the step, and the result (indices + output) D2H
@@ -272,9 +314,24 @@ def bench_ours(args, rank, world, local):
     e_ms = max_over_ranks(e_ms / e_steps, world)
 
     alg = W.algorithmic_bytes(s, wl.seqlens)
-    idx_bytes = int(np.sum(wl.seqlens.astype(np.int64))) * s.G * s.Di
+    lens = wl.seqlens.astype(np.int64)
+    idx_bytes = int(lens.sum()) * s.G * s.Di
+    row_bytes = s.Dk * 2 if s.v_in_k else (s.Dk + s.Dv) * 2
+    attn_bytes = int(np.minimum(lens, s.k).sum()) * s.G * row_bytes
     peak, peak_kind = _peaks()
-    idx_gbs = idx_bytes / (stage_ms["indexer"] * 1e-3) / 1e9 if stage_ms["indexer"] > 0 else None
+    lib_version = int(sd.load_library().sd_version())
+
+    def roofline(stage, nbytes):
+        ms = stage_ms[stage]
+        achieved = nbytes / (ms * 1e-3) / 1e9 if ms > 0 else None
+        tv = NCU_TRAFFIC.get((s.name, stage))
+        traffic = tv[1] if tv and tv[0] == lib_version and rank_spec(args.config, 0).seed == s.seed else None
+        return {"kernel": stage, "bound": "hbm", "achieved": achieved, "peak": peak, "peak_kind": peak_kind,
+                "unit": "GB/s", "frac": (achieved / peak) if achieved else None, "traffic": traffic,
+                "algorithmic_bytes_per_launch": nbytes, "ms_per_launch": ms}
+
+    rooflines = {"indexer": roofline("indexer", idx_bytes), "attn": roofline("attn", attn_bytes)}
+    dominant = max(rooflines, key=lambda k_: stage_ms[k_])
     line = {
         "metric": METRIC,
         "value": world * B / (step_ms * 1e-3),
@@ -284,18 +341,18 @@ def bench_ours(args, rank, world, local):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "int8/bf16", "data": "synthetic",
         "config": _config(s, "flushed before every step (256 MiB write, outside the timed events)"),
+        "timing": "CUDA graph of one sd_decode_step, replayed" if not args.no_graph else "eager sd_decode_step calls",
         "hbm_gbs_step": alg / (step_ms * 1e-3) / 1e9,
         "hbm_frac_step": alg / (step_ms * 1e-3) / 1e9 / peak,
         "algorithmic_bytes_per_step": alg,
         "stage_ms": stage_ms,
-        "roofline": {"kernel": "indexer", "bound": "hbm", "achieved": idx_gbs, "peak": peak,
-                     "peak_kind": peak_kind, "unit": "GB/s",
-                     "frac": (idx_gbs / peak) if idx_gbs else None,
-                     "traffic": None, "algorithmic_bytes_per_launch": idx_bytes},
+        "roofline": rooflines[dominant],
+        "rooflines": rooflines,
         "e2e": {"value": world * B / (e_ms * 1e-3), "unit": "queries/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks.summary(),
+        "library_version": lib_version,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(args.config)
@@ -311,6 +368,7 @@ def main():
     ap.add_argument("--config", default=DEFAULT_CONFIG, choices=list(W.SPECS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-graph", action="store_true", help="time eager calls instead of a CUDA graph replay")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     rank, world, local = _dist_env()

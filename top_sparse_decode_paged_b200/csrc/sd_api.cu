@@ -29,7 +29,9 @@ thread_local int32_t t_stage_count = 0;
 enum Stage { kStageIndexer = 0, kStageTopk = 1, kStageAttn = 2, kStageCombine = 3 };
 
 void stage_mark(int stage, int edge, cudaStream_t st) {
-  if (stage < t_stage_count) cudaEventRecord(t_stage_events[2 * stage + edge], st);
+  // external: inside a stream capture the record becomes a real event node that
+  // a host can time after each graph replay
+  if (stage < t_stage_count) cudaEventRecordWithFlags(t_stage_events[2 * stage + edge], st, cudaEventRecordExternal);
 }
 
 constexpr size_t kAlign = 256;
@@ -476,7 +478,7 @@ const char* sd_status_str(sd_status status) {
 
 int32_t sd_last_cuda_error(void) { return t_last_cuda_error; }
 int32_t sd_last_launch_count(void) { return t_launches; }
-int32_t sd_version(void) { return (0 << 16) | 1; }
+int32_t sd_version(void) { return (0 << 16) | 2; }
 
 }  // extern "C"
 

@@ -237,3 +237,22 @@ def test_h128_graph_replay_many_ranges():
     for i, b in enumerate(req):
         assert np.array_equal(got_idx[b], ref["indices"][i])
     assert_out_close(out.float().cpu().numpy()[req], ref["out"], "graph h128")
+
+
+def test_h128_growing_logits_rescale_mid_request():
+    """The rope columns (512..575, which enter S but not V) of the key rows are
+    scaled up along the sequence, so every head's running max moves by far
+    more than 2^8 between tiles of one request and the lazy rescale of the
+    accumulated output runs many times."""
+    wl = W.make(W.spec("b32_l65536_mla", seqlens=(4096, 3000, 700), seed=48))
+    kf = (wl.k_pages.astype(np.uint32) << 16).view(np.float32)
+    for b, L in enumerate(wl.seqlens):
+        t = np.arange(int(L))
+        pg, sl = wl.block_table[b, t // 64], t % 64
+        kf[pg, sl, 0, 512:] *= (1.0 + 30.0 * t / L)[:, None].astype(np.float32)
+    wl.k_pages[:] = W.bf16_bits_from_f32(kf)
+    got = run_step(wl, to_device(wl))
+    ref = oracle.decode_step(wl)
+    assert np.array_equal(got["indices"], np.stack(ref["indices"]))
+    assert_out_close(got["out"], ref["out"], "rescale h128")
+    np.testing.assert_allclose(got["lse"], ref["lse"], rtol=1e-4, atol=2e-3)

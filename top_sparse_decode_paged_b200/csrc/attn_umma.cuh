@@ -4,70 +4,94 @@
 // attention" (Walkthrough), consuming the top-k buffer of the DSA decode
 // step ("Overlap DSA heuristic prev_topk write-back on the aux stream").
 //
-// Tensor memory holds 128 lanes x 512 fp32 columns, and the full output of one
-// request (128 heads x 512 values) alone would fill it. So each tile range is
-// served by two CTAs, each owning half of the value columns:
-//   TMEM cols [0,256)   O half  (128 heads x 256 values, fp32, accumulated)
-//   TMEM cols [256,512) S       (128 heads x 256 selected tokens, fp32)
-//   TMEM cols [256,384) P       (bf16 pairs, written over S by the softmax)
-// Both CTAs compute the same S = Q K^T (M = 128 heads, N = 256 tokens,
-// K = 576); each then runs O += P V over its half (A = P from tensor memory,
-// B = V from shared memory).
+// Budget. The queries of one request (128 heads x 576 bf16) take 144 KB and
+// its fp32 output (128 x 512) would fill all of tensor memory. So each tile
+// range is served by two CTAs that split the heads, 64 each. A CTA keeps its
+// 64 query heads resident (72 KB) and gathers every selected row of the range
+// itself; the two CTAs of a range read the same rows at about the same time,
+// so the second read is mostly an L2 hit.
 //
-// Data movement: a four-slot ring of 48 KB slots. For each of the nine S steps
-// of a tile, a slot receives Q[:, 64 columns] (16 KB, one TMA tile; Q stays in
-// L2) and the tile's K[:, same columns] (32 KB, 256 rows x 128 bytes, gathered
-// by four copy warps with coalesced cp.async: 8 lanes per 128-byte row piece,
-// destination swizzle applied per 16-byte lane, skipped selections copy zeros).
-// The four V chunks of this CTA's half use the gather part of a slot. Keeping
-// Q out of shared memory is what buys the ring depth. A TMA tile::gather4 gather measured well below this on the part: it
-// moves one 128-byte row piece per ~20 cycles per SM. Each tile streams the nine K
-// chunks for S, then the four V chunks of this CTA's half; the same chunk
-// layout serves as the K-major B of S and as the MN-major B of P V. Whole rows
-// of the next tile are prefetched into L2 while the current one is consumed.
+// Per 64-token tile:
+//   S   = Q K^T      M = 64 heads, N = 64 tokens, K = 576 (9 chunks of 64)
+//   O^T += V^T P^T   M = 128 value rows (x4 blocks), N = 64 heads, K = 64 tokens
+// Tensor memory: O^T in columns [0,256) (block j of 128 value rows at 64j),
+// S double-buffered at [256,320) and [320,384) in the M = 64 layout (head
+// 16 q + i in lane 32 q + i).
 //
-// Softmax: the thread of TMEM lane h owns head h's row, so the row max and
-// sum stay in registers. The running max is updated lazily: O is rescaled
-// only when a tile's max exceeds the reference by more than 2^8, so most tiles
-// skip the read-modify-write of O.
+// Shared memory: Q (9 chunks x 64 heads x 128 B), two 72 KB tile buffers
+// (9 chunks x 64 tokens x 128 B, the 128-byte swizzle), P^T (64 heads x 64
+// tokens bf16), and a small ring of row ids. A tile chunk is the K-major B of
+// S and, read MN-major, the A of O^T. Small-N MMAs are bound by reading their
+// operands from shared memory, which is why S uses M = 64 (only real heads)
+// and tiles are as wide as the buffers allow.
 //
-// Work: all requests' tiles (ceil(min(k, L) / 256) per request) form one list
+// Rows. Selections arrive resolved to pool rows (page * page_size + slot, -1
+// to skip): the decode step's top-k writes them, a standalone call runs
+// attn_rows_kernel. A warp streams each tile's 64 row ids into the ring a few
+// tiles ahead, so no dependent block-table load sits on the gather's path.
+// Gathers use coalesced cp.async: 8 lanes fetch one 128-byte row piece, the
+// destination swizzle is applied per 16-byte lane, and skipped rows copy
+// zeros. Measured on the part: scattered 1152-byte rows stream from HBM at
+// about 3.1 TB/s by cp.async and 2.8 TB/s by 1-D bulk copies; pushing half of
+// each tile to the partner CTA over distributed shared memory was slower than
+// reading it twice through L2.
+//
+// Softmax: a 16-lane tensor-memory load spreads each warp's 16 heads over all
+// 32 threads (2 heads x 16 tokens each); max and sum are combined over the 4
+// threads of a head with shuffles. The running max is updated lazily: O is
+// rescaled only when a tile's max exceeds the reference by more than 2^8.
+//
+// Work: all requests' tiles (ceil(min(k, L) / 64) per request) form one list
 // that is cut into equal contiguous ranges, one per CTA pair. A range that
 // covers parts of several requests writes one partial (O, m, l) per request.
 // The combine kernel merges them.
 //
-// Roles (288 threads): warps 0-3 copy, warps 4-7 run the softmax and write
-// partials (warp w owns TMEM lanes 32*(w%4)..+31), warp 8 issues the MMAs. Every wait is bounded (a timeout flags SD_DEVERR_TIMEOUT).
+// Roles (320 threads): warps 0-3 copy (thread 0 also loads Q by TMA), warps
+// 4-7 run the softmax, rescale and write partials (warp w owns TMEM lanes
+// 32*(w%4)..+31), warp 8 issues the MMAs as their inputs become ready, warp 9
+// streams row ids. Every wait is bounded (a timeout flags SD_DEVERR_TIMEOUT).
 #pragma once
 
 #include "sm100.cuh"
 
 namespace sd {
 
-constexpr int kAuTile = 256;               // selected tokens per tile (N of S)
-constexpr int kAuHeads = 128;              // M
+constexpr int kAuTile = 64;                // selected tokens per tile
+constexpr int kAuTileWords = kAuTile / 32; // 32-bit valid-token words per tile
+constexpr int kAuHeads = 128;              // query heads of a request
+constexpr int kAuHalfHeads = 64;           // query heads per CTA (M of S)
 constexpr int kAuDk = 576, kAuDv = 512;
-constexpr int kAuQChunks = kAuDk / 64;     // 9
-constexpr int kAuVChunks = kAuDv / 2 / 64; // 4 per value half
-constexpr int kAuChunkBytes = kAuTile * 128;   // 32 KB: 256 rows x 64 columns
-constexpr int kAuQChunkBytes = kAuHeads * 128; // 16 KB: 128 heads x 64 columns
-constexpr int kAuSlotBytes = kAuQChunkBytes + kAuChunkBytes;  // one ring slot
-constexpr int kAuSlots = 4;
-constexpr int kAuThreads = 288;
+constexpr int kAuChunks = kAuDk / 64;      // 9 column chunks of 64
+constexpr int kAuVBlocks = kAuDv / 128;    // 4 blocks of 128 value rows
+constexpr int kAuChunkBytes = kAuTile * 128;              // 8 KB
+constexpr int kAuTileBytes = kAuChunks * kAuChunkBytes;   // 72 KB
+constexpr int kAuQChunkBytes = kAuHalfHeads * 128;        // 8 KB
+constexpr int kAuQBytes = kAuChunks * kAuQChunkBytes;     // 72 KB
+constexpr int kAuPBytes = kAuHalfHeads * 128;             // 8 KB: 64 head rows of up to 64 tokens
+constexpr int kAuBufs = 2;
+constexpr int kAuThreads = 320;
+constexpr int kAuRidSlots = 4;             // row-id lookahead (tiles)
 constexpr int kAuRanges = 74;              // CTA pairs: 148 CTAs, one per SM
 constexpr float kAuRescaleLog2 = 8.0f;     // lazy rescale threshold (log2 units)
-constexpr int kAuPrefetchTiles = 3;       // L2 prefetch distance (tiles)
-constexpr int kMaxTopK = 2048;            // largest k the library accepts
+constexpr int kMaxTopK = 2048;             // largest k the library accepts
+static_assert(kAuTile % 32 == 0 && kAuTile <= 64, "tile of 32 or 64 tokens");
+
+// Row-id slots per request in the resolved-row array (whole tiles).
+__host__ __device__ constexpr int attn_kpad(int k) { return (k + kAuTile - 1) / kAuTile * kAuTile; }
 
 struct AttnUmmaLayout {
-  static constexpr int kOffRing = 0;
-  static constexpr int kOffBar = kAuSlots * kAuSlotBytes;           // 196608
-  static constexpr int kNumBars = 2 * kAuSlots + 3;
-  static constexpr int kOffMask = kOffBar + 8 * kNumBars;
-  static constexpr int kOffMisc = kOffMask + 2 * 8 * 4;
+  static constexpr int kOffQ = 0;
+  static constexpr int kOffRing = kOffQ + kAuQBytes;
+  static constexpr int kOffP = kOffRing + kAuBufs * kAuTileBytes;
+  static constexpr int kOffBar = kOffP + kAuPBytes;
+  static constexpr int kNumBars = 2 * kAuBufs + 9 + 2 * kAuRidSlots;
+  static constexpr int kOffRid = kOffBar + 8 * kNumBars;             // [slots][tile] pool row ids (-1: skip)
+  static constexpr int kOffAlpha = kOffRid + 4 * kAuTile * kAuRidSlots;  // [64] rescale factors
+  static constexpr int kOffMisc = kOffAlpha + 4 * kAuHalfHeads;
   static constexpr int kBytes = kOffMisc + 16;
   static constexpr size_t kSmemAlloc = kBytes + 1024;
 };
+static_assert(AttnUmmaLayout::kSmemAlloc <= 232448, "attention shared memory");
 
 // Walks a contiguous range of the attention tile list (request-major).
 struct AttnCursor {
@@ -126,47 +150,79 @@ __device__ __forceinline__ long long attn_row_of(const int32_t* indices, const i
   return (long long)page * page_size + (t % page_size);
 }
 
+// Resolves selections to pool rows for a standalone attention call (the
+// decode step has the top-k write them): rows[b][s] for s < attn_kpad(k),
+// -1 past min(k, L_b) and for skipped selections.
+__global__ void __launch_bounds__(256) attn_rows_kernel(const int32_t* __restrict__ indices,
+                                                        const int32_t* __restrict__ block_table,
+                                                        const int32_t* __restrict__ seqlens, int k, int seqlen_cap,
+                                                        int page_size, int max_pages, int num_pages,
+                                                        int32_t* __restrict__ rows) {
+  const int b = blockIdx.y;
+  const int s = blockIdx.x * 256 + threadIdx.x;
+  const int kpad = attn_kpad(k);
+  if (s >= kpad) return;
+  const int L = checked_seqlen(seqlens, b, seqlen_cap);
+  rows[(size_t)b * kpad + s] = static_cast<int>(
+      attn_row_of(indices, block_table, b, s, min(k, L), k, L, page_size, max_pages, num_pages));
+}
+
 __global__ void __launch_bounds__(kAuThreads, 1) attn_mla_umma_kernel(
-    const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kv,
-    const __nv_bfloat16* __restrict__ kv,
-    const int32_t* __restrict__ block_table, const int32_t* __restrict__ seqlens,
-    const int32_t* __restrict__ indices, int B, int k, int num_pages, int page_size, int max_pages,
-    int seqlen_cap, float scale_log2, float* __restrict__ part_o, float2* __restrict__ part_ml) {
+    const __grid_constant__ CUtensorMap tm_q, const __nv_bfloat16* __restrict__ kv,
+    const int32_t* __restrict__ seqlens, const int32_t* __restrict__ rows, int B, int k, int seqlen_cap,
+    float scale_log2, float* __restrict__ part_o, float2* __restrict__ part_ml) {
   using Lay = AttnUmmaLayout;
   extern __shared__ uint8_t smem_dyn[];
   const uint32_t raw = smem_u32(smem_dyn);
   uint8_t* smem = smem_dyn + (((raw + 1023u) & ~1023u) - raw);
+  uint8_t* qbuf = smem + Lay::kOffQ;
   uint8_t* ring = smem + Lay::kOffRing;
+  uint8_t* pbuf = smem + Lay::kOffP;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::kOffBar);
-  uint64_t* chunk_full = bars;                   // [kAuSlots]: 128 copy arrivals + 1 TMA issuer
-  uint64_t* chunk_empty = bars + kAuSlots;       // [kAuSlots]: MMA commit
-  uint64_t* s_full = bars + 2 * kAuSlots;        // MMA commit
-  uint64_t* p_full = bars + 2 * kAuSlots + 1;    // 128 softmax arrivals
-  uint64_t* pv_done = bars + 2 * kAuSlots + 2;   // MMA commit
-  uint32_t* mask_words = reinterpret_cast<uint32_t*>(smem + Lay::kOffMask);  // [2][8]
+  uint64_t* tile_full = bars;                    // [bufs] 128 copy-thread arrivals (cp.async)
+  uint64_t* tile_empty = bars + kAuBufs;         // [bufs] MMA commit after the tile's P V
+  uint64_t* q_full = bars + 2 * kAuBufs;         // 1 arrival + the Q bytes (TMA)
+  uint64_t* q_empty = q_full + 1;                // MMA commit after a request's last S
+  uint64_t* s_full = q_full + 2;                 // [2] MMA commit
+  uint64_t* s_free = q_full + 4;                 // [2] the four softmax warps have read S
+  uint64_t* p_full = q_full + 6;                 // the four epilogue warps: P written, O rescaled/read out
+  uint64_t* pv_done = q_full + 7;                // MMA commit after P V
+  uint64_t* mma_fin = q_full + 8;                // MMA commit at exit
+  uint64_t* rid_full = q_full + 9;               // [slots] 32 row-id lanes (cp.async)
+  uint64_t* rid_empty = rid_full + kAuRidSlots;  // [slots] 4 copy warps + the epilogue
+  int32_t* rid = reinterpret_cast<int32_t*>(smem + Lay::kOffRid);
+  float* alpha_s = reinterpret_cast<float*>(smem + Lay::kOffAlpha);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Lay::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Lay::kOffMisc + 4);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_ranges = gridDim.x / 2;
   const int range = blockIdx.x % n_ranges;
-  const int half = blockIdx.x / n_ranges;  // which 256 value columns this CTA owns
+  const int hh = blockIdx.x / n_ranges;  // which 64 query heads this CTA owns
+  const int kpad = attn_kpad(k);
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kAuSlots; ++i) {
-      sm100::mbar_init(&chunk_full[i], 129);
-      sm100::mbar_init(&chunk_empty[i], 1);
+    for (int i = 0; i < kAuBufs; ++i) {
+      sm100::mbar_init(&tile_full[i], 128);
+      sm100::mbar_init(&tile_empty[i], 1);
     }
-    sm100::mbar_init(s_full, 1);
-    sm100::mbar_init(p_full, 128);
+    sm100::mbar_init(q_full, 1);
+    sm100::mbar_init(q_empty, 1);
+    for (int i = 0; i < 2; ++i) {
+      sm100::mbar_init(&s_full[i], 1);
+      sm100::mbar_init(&s_free[i], 4);
+    }
+    sm100::mbar_init(p_full, 4);
     sm100::mbar_init(pv_done, 1);
+    sm100::mbar_init(mma_fin, 1);
+    for (int i = 0; i < kAuRidSlots; ++i) {
+      sm100::mbar_init(&rid_full[i], 32);
+      sm100::mbar_init(&rid_empty[i], 5);
+    }
     *abort_flag = 0;
     sm100::fence_barrier_init();
   }
-  if (warp == 0 && lane == 0) {
-    sm100::prefetch_tensormap(&tm_q);
-    sm100::prefetch_tensormap(&tm_kv);
-  }
+  if (warp == 0 && lane == 0) sm100::prefetch_tensormap(&tm_q);
   if (warp == 8) {
     sm100::tmem_alloc(tmem_slot, 512);
     sm100::tmem_relinquish();
@@ -175,8 +231,8 @@ __global__ void __launch_bounds__(kAuThreads, 1) attn_mla_umma_kernel(
   __syncthreads();
   sm100::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tm_o = tmem;          // cols [0,256)
-  const uint32_t tm_s = tmem + 256;    // cols [256,512); P over [256,384)
+  const uint32_t tm_o = tmem;          // cols [0,256): O^T, block j at 64j
+  const uint32_t tm_s = tmem + 256;    // S, two buffers of kAuTile columns
 
   const long long total = attn_total_tiles(seqlens, B, seqlen_cap, k);
   const long long first = total * range / n_ranges;
@@ -184,243 +240,318 @@ __global__ void __launch_bounds__(kAuThreads, 1) attn_mla_umma_kernel(
 
   if (warp < 4) {
     // ------------------------------ copies ------------------------------
-    // Each S chunk c of a tile fills one ring slot with Q[:, 64c..64c+63] (a
-    // 16 KB TMA tile; Q is small and stays in L2) and the tile's K[:, 64c..]
-    // (32 KB gathered with cp.async). A V chunk fills the gather part only.
-    // The gather is coalesced: in each copy instruction 8 lanes fetch one
-    // 128-byte row piece, so a warp moves 4 pieces (512 B); the 16-byte
-    // swizzle of the destination is applied per lane. Thread pt fetches rows
-    // 64*warp + 4*i + lane/8 (i = 0..15), 16-byte column j = lane % 8.
+    // Thread pt fetches 16-byte column `seg` of tokens pt/8 + 16 i in all
+    // nine chunks, so each copy instruction of a warp moves four 128-byte row
+    // pieces.
     const int pt = threadIdx.x;  // 0..127
-    const int jseg = lane & 7;
+    const int seg = lane & 7;
     AttnCursor c;
     c.init(seqlens, B, seqlen_cap, k, first, count);
-    long long n = 0;  // ring uses
+    long long n = 0;
+    int q_issued = 0, prev_b = -1;
     bool ok = true;
     while (c.valid() && ok) {
-      const int kb = min(k, c.L);
-      const int s0 = c.tile * kAuTile;
-      int row[16];
-#pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        const long long r = attn_row_of(indices, block_table, c.b, s0 + 64 * warp + 4 * i + (lane >> 3), kb, k, c.L,
-                                        page_size, max_pages, num_pages);
-        row[i] = static_cast<int>(r);  // -1: skipped, copied as zeros
-      }
-      // Whole selected rows into L2 ahead of their gathers: the tiles up to
-      // kAuPrefetchTiles ahead (on the first tile, those in between too).
-      {
-        AttnCursor nx = c;
-        for (int ahead = 0; ahead <= kAuPrefetchTiles && nx.valid(); ++ahead) {
-          if (ahead == kAuPrefetchTiles || (n == 0 && ahead < kAuPrefetchTiles)) {
-            const int nkb = min(k, nx.L);
-#pragma unroll
-            for (int rr = 0; rr < 2; ++rr) {
-              const long long r = attn_row_of(indices, block_table, nx.b, nx.tile * kAuTile + pt + 128 * rr, nkb, k,
-                                              nx.L, page_size, max_pages, num_pages);
-              if (r >= 0) sm100::prefetch_l2_bulk(kv + r * kAuDk, kAuDk * 2);
-            }
-          }
-          nx.next(seqlens, B, seqlen_cap, k);
-        }
-      }
-      for (int ci = 0; ci < kAuQChunks + kAuVChunks && ok; ++ci, ++n) {
-        const bool is_s = ci < kAuQChunks;
-        const int cc = is_s ? ci : half * kAuVChunks + (ci - kAuQChunks);
-        const int slot = static_cast<int>(n % kAuSlots);
-        ok = sm100::mbar_wait(&chunk_empty[slot], static_cast<uint32_t>((n / kAuSlots) & 1) ^ 1) && !*abort_flag;
-        if (!ok) break;
-        uint8_t* slot_base = ring + slot * kAuSlotBytes;
+      if (c.b != prev_b) {
+        // a new request: its 64 query heads into the Q buffer once the
+        // previous request's S products are done with it
+        prev_b = c.b;
         if (pt == 0) {
-          sm100::mbar_arrive_expect_tx(&chunk_full[slot], is_s ? kAuQChunkBytes : 0);
-          if (is_s) sm100::tma_load_2d(slot_base, &tm_q, &chunk_full[slot], cc * 64, c.b * kAuHeads);
+          if (q_issued > 0) ok = sm100::mbar_wait(q_empty, (q_issued - 1) & 1);
+          if (ok) {
+            sm100::mbar_arrive_expect_tx(q_full, kAuQBytes);
+            for (int cc = 0; cc < kAuChunks; ++cc)
+              sm100::tma_load_2d(qbuf + cc * kAuQChunkBytes, &tm_q, q_full, cc * 64,
+                                 c.b * kAuHeads + hh * kAuHalfHeads);
+            ++q_issued;
+          } else {
+            *abort_flag = 1;
+          }
         }
-        uint8_t* dst_base = slot_base + kAuQChunkBytes;
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const int r = 64 * warp + 4 * i + (lane >> 3);
-          const int rw = row[i];
-          const __nv_bfloat16* src = kv + (long long)(rw >= 0 ? rw : 0) * kAuDk + cc * 64 + jseg * 8;
-          cp_async_16(dst_base + r * 128 + ((jseg ^ (r & 7)) << 4), src, rw >= 0 ? 16 : 0);
-        }
-        sm100::cp_async_arrive_noinc(&chunk_full[slot]);
       }
+      const int rs = static_cast<int>(n % kAuRidSlots);
+      ok = ok && sm100::mbar_wait(&rid_full[rs], static_cast<uint32_t>((n / kAuRidSlots) & 1));
+      if (!ok) break;
+      int row[kAuTile / 16];
+#pragma unroll
+      for (int i = 0; i < kAuTile / 16; ++i) row[i] = rid[rs * kAuTile + (pt >> 3) + 16 * i];
+      __syncwarp();
+      if (lane == 0) sm100::mbar_arrive(&rid_empty[rs]);
+      const int slot = static_cast<int>(n % kAuBufs);
+      ok = ok && sm100::mbar_wait(&tile_empty[slot], static_cast<uint32_t>((n / kAuBufs) & 1) ^ 1) && !*abort_flag;
+      if (!ok) break;
+      uint8_t* tb = ring + slot * kAuTileBytes;
+#pragma unroll
+      for (int i = 0; i < kAuTile / 16; ++i) {
+        const int t = (pt >> 3) + 16 * i;
+        const int rw = row[i];
+        const __nv_bfloat16* src = kv + (long long)(rw >= 0 ? rw : 0) * kAuDk + seg * 8;
+        uint8_t* dst = tb + t * 128 + ((seg ^ (t & 7)) << 4);
+#pragma unroll
+        for (int cc = 0; cc < kAuChunks; ++cc) cp_async_16(dst + cc * kAuChunkBytes, src + cc * 64, rw >= 0 ? 16 : 0);
+      }
+      sm100::cp_async_arrive_noinc(&tile_full[slot]);
+      ++n;
       c.next(seqlens, B, seqlen_cap, k);
     }
     cp_async_wait<0>();
     if (!ok) *abort_flag = 1;
+    // the last Q load must have landed before the CTA exits
+    if (pt == 0 && q_issued > 0) sm100::mbar_wait(q_full, (q_issued - 1) & 1);
   } else if (warp < 8) {
-    // ------------------------ softmax and partials ------------------------
-    const int st = threadIdx.x - 128;         // 0..127
-    const int sw = warp - 4;                  // 0..3 (mask word owner)
+    // ------------------- softmax, rescale and partials -------------------
+    // S is an M = 64 accumulator: head 16 q + i sits in TMEM lane 32 q + i
+    // (i < 16). A 16-lane load spreads quadrant q's 16 heads over the warp:
+    // thread t holds heads 16 q + t/4 and 16 q + t/4 + 8, 16 of the 64 tokens
+    // each (tokens 8 r + 2 (t % 4) + {0, 1}); the 4 threads of a head combine
+    // their max and sum with shuffles.
+    constexpr int kReps = kAuTile / 8;  // 8-column repetitions of the 16x256b load
     const int quarter = warp & 3;
-    const int head = quarter * 32 + lane;     // TMEM lane == head
+    const int tq = lane & 3;
+    const int h0 = quarter * 16 + (lane >> 2);  // and h0 + 8
+    const int vrow = quarter * 32 + lane;       // value row of O^T within a block
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
     AttnCursor c;
     c.init(seqlens, B, seqlen_cap, k, first, count);
-    int ntile = 0;
-    bool seg_first = true;
-    float m_ref = -INFINITY, l_sum = 0.f;
+    long long j = 0;
+    int prev_b = -1;
+    float m_ref[2] = {-INFINITY, -INFINITY}, l_sum[2] = {0.f, 0.f};
     while (c.valid()) {
-      const int kb = min(k, c.L);
-      const int s0 = c.tile * kAuTile;
-      uint32_t* mw = mask_words + (ntile & 1) * 8;
-#pragma unroll
-      for (int rr = 0; rr < 2; ++rr) {
-        const bool v = attn_row_of(indices, block_table, c.b, s0 + st + rr * 128, kb, k, c.L, page_size,
-                                   max_pages, num_pages) >= 0;
-        const uint32_t bal = __ballot_sync(0xffffffffu, v);
-        if (lane == 0) mw[rr * 4 + sw] = bal;
+      const bool seg_first = c.b != prev_b;
+      prev_b = c.b;
+      if (seg_first) {
+        m_ref[0] = m_ref[1] = -INFINITY;
+        l_sum[0] = l_sum[1] = 0.f;
       }
-      // wait for S, then one barrier both publishes the mask words and makes
-      // the exit decision uniform over the 128 softmax threads
-      bool ok = sm100::mbar_wait(s_full, ntile & 1) && !*abort_flag;
+      const int rs = static_cast<int>(j % kAuRidSlots);
+      uint32_t mask[kAuTileWords];
+      bool ok = sm100::mbar_wait(&rid_full[rs], static_cast<uint32_t>((j / kAuRidSlots) & 1));
+#pragma unroll
+      for (int w = 0; w < kAuTileWords; ++w) mask[w] = __ballot_sync(0xffffffffu, rid[rs * kAuTile + 32 * w + lane] >= 0);
+      ok = ok && sm100::mbar_wait(&s_full[j & 1], static_cast<uint32_t>((j >> 1) & 1)) && !*abort_flag;
+      // one barrier makes the exit uniform and retires this tile's row-id slot
       ok = sm100::named_bar_and(1, 128, ok);
       if (!ok) { *abort_flag = 1; break; }
-      uint32_t mask[8];
-#pragma unroll
-      for (int j = 0; j < 8; ++j) mask[j] = mw[j];
+      if (threadIdx.x == 128) sm100::mbar_arrive(&rid_empty[rs]);
       sm100::tc_fence_after();
-
-      // pass 1: row max over the valid tokens
-      float mx = -INFINITY;
-#pragma unroll 1
-      for (int j = 0; j < 8; ++j) {
-        uint32_t r[32];
-        sm100::tmem_ld_32x32b_x32(tm_s + lane_base + 32 * j, r);
-        sm100::tmem_ld_wait();
+      uint32_t r[4 * kReps];
+      sm100::tmem_ld_16x256b(tm_s + kAuTile * static_cast<uint32_t>(j & 1) + lane_base, r);
+      sm100::tmem_ld_wait();
+      sm100::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) sm100::mbar_arrive(&s_free[j & 1]);
+      // valid bits of this thread's tokens 8 rr + 2 tq + {0, 1}
+      uint32_t vb = 0;
 #pragma unroll
-        for (int i = 0; i < 32; ++i)
-          if ((mask[j] >> i) & 1u) mx = fmaxf(mx, __uint_as_float(r[i]) * scale_log2);
+      for (int rr = 0; rr < kReps; ++rr) {
+        const int t0 = 8 * rr + 2 * tq;
+        vb |= ((mask[t0 >> 5] >> (t0 & 31)) & 3u) << (2 * rr);
       }
-      const float m_tile = mx;  // max of the scaled logits (any sign of scale)
-      const bool need = m_tile > m_ref + kAuRescaleLog2 || (m_ref == -INFINITY && m_tile > -INFINITY);
-      float alpha = 1.f;
-      if (need) {
-        alpha = exp2f(m_ref - m_tile);  // 0 when m_ref is -inf
-        l_sum *= alpha;
-        m_ref = m_tile;
+      uint32_t pk[2][kReps];  // [head][rr]: bf16 pair of tokens 8 rr + 2 tq + {0, 1}
+      bool need = false;
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        float mx = -INFINITY;
+#pragma unroll
+        for (int rr = 0; rr < kReps; ++rr) {
+          if ((vb >> (2 * rr)) & 1u) mx = fmaxf(mx, __uint_as_float(r[4 * rr + 2 * e]) * scale_log2);
+          if ((vb >> (2 * rr + 1)) & 1u) mx = fmaxf(mx, __uint_as_float(r[4 * rr + 2 * e + 1]) * scale_log2);
+        }
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+        const bool ne = mx > m_ref[e] + kAuRescaleLog2 || (m_ref[e] == -INFINITY && mx > -INFINITY);
+        float alpha = 1.f;
+        if (ne) {
+          alpha = exp2f(m_ref[e] - mx);  // 0 when m_ref is -inf
+          l_sum[e] *= alpha;
+          m_ref[e] = mx;
+        }
+        need = need || ne;
+        if (tq == 0) alpha_s[h0 + 8 * e] = alpha;
+        const float m_use = m_ref[e] == -INFINITY ? 0.f : m_ref[e];
+#pragma unroll
+        for (int rr = 0; rr < kReps; ++rr) {
+          const float p0 = ((vb >> (2 * rr)) & 1u)
+                               ? sm100::ex2_approx(__uint_as_float(r[4 * rr + 2 * e]) * scale_log2 - m_use) : 0.f;
+          const float p1 = ((vb >> (2 * rr + 1)) & 1u)
+                               ? sm100::ex2_approx(__uint_as_float(r[4 * rr + 2 * e + 1]) * scale_log2 - m_use) : 0.f;
+          const __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
+          l_sum[e] += __low2float(h2) + __high2float(h2);
+          pk[e][rr] = *reinterpret_cast<const uint32_t*>(&h2);
+        }
       }
-      // O holds earlier tiles of this segment: scale rows whose reference moved
-      // (warp-uniform branch: tcgen05.ld/st are warp-collective)
-      if (__any_sync(0xffffffffu, need) && !seg_first) {
+      // earlier tiles of this request are in O: rescale when any head's
+      // reference moved (alpha_s published by the barrier)
+      const bool rescale = sm100::named_bar_or(2, 128, need && !seg_first);
+      // O and the P buffer are free once the previous P V has completed
+      if (j > 0) {
+        bool okp = sm100::mbar_wait(pv_done, static_cast<uint32_t>((j - 1) & 1)) && !*abort_flag;
+        okp = sm100::named_bar_and(3, 128, okp);
+        if (!okp) { *abort_flag = 1; break; }
+        sm100::tc_fence_after();
+      }
+      if (rescale) {
 #pragma unroll 1
-        for (int j = 0; j < 8; ++j) {
-          uint32_t r[32];
-          sm100::tmem_ld_32x32b_x32(tm_o + lane_base + 32 * j, r);
+        for (int q8 = 0; q8 < 8; ++q8) {  // 4 value blocks x 2 halves of 32 head columns
+          uint32_t ro[32];
+          const uint32_t oa = tm_o + 32 * q8 + lane_base;
+          sm100::tmem_ld_32x32b_x32(oa, ro);
           sm100::tmem_ld_wait();
+          const float* al = alpha_s + 32 * (q8 & 1);
 #pragma unroll
-          for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
-          sm100::tmem_st_32x32b_x32(tm_o + lane_base + 32 * j, r);
+          for (int i = 0; i < 32; ++i) ro[i] = __float_as_uint(__uint_as_float(ro[i]) * al[i]);
+          sm100::tmem_st_32x32b_x32(oa, ro);
         }
         sm100::tmem_st_wait();
       }
-      const float m_use = m_ref == -INFINITY ? 0.f : m_ref;
-
-      // pass 2: P = 2^(s * scale_log2 - m_ref) as bf16, written over S
-#pragma unroll 1
-      for (int j = 0; j < 8; ++j) {
-        uint32_t r[32], pk[16];
-        sm100::tmem_ld_32x32b_x32(tm_s + lane_base + 32 * j, r);
-        sm100::tmem_ld_wait();
+      {
+        // P^T rows of heads h0, h0 + 8: this thread's 4-byte token pair in
+        // each 16-byte piece, 128-byte swizzle
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const float p0 = ((mask[j] >> (2 * i)) & 1u) ? sm100::ex2_approx(__uint_as_float(r[2 * i]) * scale_log2 - m_use) : 0.f;
-          const float p1 =
-              ((mask[j] >> (2 * i + 1)) & 1u) ? sm100::ex2_approx(__uint_as_float(r[2 * i + 1]) * scale_log2 - m_use) : 0.f;
-          const __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
-          l_sum += __low2float(h2) + __high2float(h2);
-          pk[i] = *reinterpret_cast<const uint32_t*>(&h2);
+        for (int e = 0; e < 2; ++e) {
+          const int h = h0 + 8 * e;
+          uint8_t* prow = pbuf + (h >> 3) * 1024 + (h & 7) * 128 + 4 * tq;
+#pragma unroll
+          for (int rr = 0; rr < kReps; ++rr) *reinterpret_cast<uint32_t*>(prow + ((rr ^ (h & 7)) << 4)) = pk[e][rr];
         }
-        sm100::tmem_st_32x32b_x16(tm_s + lane_base + 16 * j, pk);
+        sm100::fence_proxy_async_smem();
       }
-      sm100::tmem_st_wait();
       sm100::tc_fence_before();
-      sm100::mbar_arrive(p_full);
+      __syncwarp();
+      if (lane == 0) sm100::mbar_arrive(p_full);
 
       const int this_b = c.b;
       c.next(seqlens, B, seqlen_cap, k);
-      const bool seg_end = !c.valid() || c.b != this_b;
-      if (seg_end) {
-        bool okd = sm100::mbar_wait(pv_done, ntile & 1) && !*abort_flag;
-        okd = sm100::named_bar_and(2, 128, okd);
+      const bool seg_last = !c.valid() || c.b != this_b;
+      if (seg_last) {
+        bool okd = sm100::mbar_wait(pv_done, static_cast<uint32_t>(j & 1)) && !*abort_flag;
+        okd = sm100::named_bar_and(4, 128, okd);
         if (!okd) { *abort_flag = 1; break; }
         sm100::tc_fence_after();
         const size_t slot = static_cast<size_t>(range) + this_b;
-        float* dst = part_o + ((slot * 2 + half) * kAuHeads + head) * (kAuDv / 2);
+        float* dst = part_o + (slot * kAuHeads + hh * kAuHalfHeads) * kAuDv + vrow;
 #pragma unroll 1
-        for (int j = 0; j < 8; ++j) {
-          uint32_t r[32];
-          sm100::tmem_ld_32x32b_x32(tm_o + lane_base + 32 * j, r);
+        for (int q8 = 0; q8 < 8; ++q8) {  // block q8/2, head columns 32*(q8%2)..+31
+          uint32_t ro[32];
+          sm100::tmem_ld_32x32b_x32(tm_o + 32 * q8 + lane_base, ro);
           sm100::tmem_ld_wait();
+          float* d = dst + (q8 >> 1) * 128 + (size_t)(32 * (q8 & 1)) * kAuDv;
 #pragma unroll
-          for (int i = 0; i < 32; i += 4)
-            *reinterpret_cast<float4*>(dst + 32 * j + i) =
-                make_float4(__uint_as_float(r[i]), __uint_as_float(r[i + 1]), __uint_as_float(r[i + 2]),
-                            __uint_as_float(r[i + 3]));
+          for (int i = 0; i < 32; ++i) d[(size_t)i * kAuDv] = __uint_as_float(ro[i]);
         }
-        if (half == 0) part_ml[slot * kAuHeads + head] = make_float2(m_ref, l_sum);
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          float l = l_sum[e];
+          l += __shfl_xor_sync(0xffffffffu, l, 1);
+          l += __shfl_xor_sync(0xffffffffu, l, 2);
+          if (tq == 0) part_ml[slot * kAuHeads + hh * kAuHalfHeads + h0 + 8 * e] = make_float2(m_ref[e], l);
+        }
         sm100::tc_fence_before();
-        m_ref = -INFINITY;
-        l_sum = 0.f;
       }
-      seg_first = seg_end;
-      ++ntile;
+      ++j;
     }
-  } else {
+  } else if (warp == 8) {
     // ------------------------------ MMA issue ------------------------------
     if (sm100::elect_one()) {
-      constexpr uint32_t idesc_s = sm100::idesc_bf16(kAuHeads, kAuTile, false, false);
-      constexpr uint32_t idesc_pv = sm100::idesc_bf16(kAuHeads, 64, false, true);
-      AttnCursor c;
-      c.init(seqlens, B, seqlen_cap, k, first, count);
-      long long n = 0;
-      int ntile = 0;
-      bool seg_first = true;
-      while (c.valid() && !*abort_flag) {
-        bool ok = true;
-        // S = Q K^T over the nine 64-column chunks
-        for (int cc = 0; cc < kAuQChunks && ok; ++cc, ++n) {
-          const int slot = static_cast<int>(n % kAuSlots);
-          ok = sm100::mbar_wait(&chunk_full[slot], static_cast<uint32_t>((n / kAuSlots) & 1));
-          if (ok && cc == 0 && ntile > 0) ok = sm100::mbar_wait(pv_done, (ntile - 1) & 1);
-          if (!ok) break;
-          sm100::tc_fence_after();
-          const uint32_t a0 = smem_u32(ring + slot * kAuSlotBytes);
-          const uint32_t b0 = a0 + kAuQChunkBytes;
+      constexpr uint32_t idesc_s = sm100::idesc_bf16(kAuHalfHeads, kAuTile, false, false);
+      constexpr uint32_t idesc_pv = sm100::idesc_bf16(128, kAuHalfHeads, true, false);
+      const uint32_t qa = smem_u32(qbuf), pa = smem_u32(pbuf);
+      // Issue S and P V in the order their inputs become ready: S(i) needs
+      // tile i landed (and its request's Q) and S buffer i%2 read out;
+      // P V(j) needs P(j). Polling both keeps P V(j) from waiting for the
+      // next tile's rows, so a tile buffer is released as soon as its own
+      // P V is done.
+      AttnCursor cs, cp;
+      cs.init(seqlens, B, seqlen_cap, k, first, count);
+      cp.init(seqlens, B, seqlen_cap, k, first, count);
+      long long is = 0, ip = 0;
+      int q_seen = 0, prev_bs = -1, prev_bp = -1;
+      uint32_t idle = 0;
+      bool ok = true;
+      while (ip < count && ok) {
+        bool progressed = false;
+        if (is < count) {
+          const bool seg_first = cs.b != prev_bs;
+          const int slot = static_cast<int>(is % kAuBufs);
+          const int sb = static_cast<int>(is & 1);
+          const bool ready = (!seg_first || sm100::mbar_test_wait(q_full, static_cast<uint32_t>(q_seen & 1))) &&
+                             sm100::mbar_test_wait(&tile_full[slot], static_cast<uint32_t>((is / kAuBufs) & 1)) &&
+                             (is < 2 || sm100::mbar_test_wait(&s_free[sb], static_cast<uint32_t>(((is - 2) >> 1) & 1)));
+          if (ready) {
+            sm100::tc_fence_after();
+            if (seg_first) ++q_seen;
+            prev_bs = cs.b;
+            // S = Q K^T (M = 64 heads) over the nine 64-column chunks
+            const uint32_t ta = smem_u32(ring + slot * kAuTileBytes);
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            sm100::mma_bf16_ss(tm_s, sm100::smem_desc_k_sw128(a0 + 32 * kk), sm100::smem_desc_k_sw128(b0 + 32 * kk),
-                               idesc_s, (cc | kk) != 0);
-          sm100::mma_commit(&chunk_empty[slot]);
-        }
-        if (!ok) { *abort_flag = 1; break; }
-        sm100::mma_commit(s_full);
-        const int this_b = c.b;
-        c.next(seqlens, B, seqlen_cap, k);
-        const bool last_of_req = !c.valid() || c.b != this_b;
-        // O += P V over this CTA's four value chunks
-        if (!sm100::mbar_wait(p_full, ntile & 1)) { *abort_flag = 1; break; }
-        sm100::tc_fence_after();
-        for (int v = 0; v < kAuVChunks && ok; ++v, ++n) {
-          const int slot = static_cast<int>(n % kAuSlots);
-          ok = sm100::mbar_wait(&chunk_full[slot], static_cast<uint32_t>((n / kAuSlots) & 1));
-          if (!ok) break;
-          sm100::tc_fence_after();
-          const uint32_t b0 = smem_u32(ring + slot * kAuSlotBytes + kAuQChunkBytes);
+            for (int cc = 0; cc < kAuChunks; ++cc)
 #pragma unroll
-          for (int i = 0; i < kAuTile / 16; ++i)
-            sm100::mma_bf16_ts(tm_o + 64 * v, tm_s + 8 * i,
-                               sm100::smem_desc_mn_sw128(b0 + i * 2048, kAuChunkBytes, 1024), idesc_pv,
-                               !(seg_first && i == 0));
-          sm100::mma_commit(&chunk_empty[slot]);
+              for (int kk = 0; kk < 4; ++kk)
+                sm100::mma_bf16_ss(tm_s + kAuTile * sb, sm100::smem_desc_k_sw128(qa + cc * kAuQChunkBytes + 32 * kk),
+                                   sm100::smem_desc_k_sw128(ta + cc * kAuChunkBytes + 32 * kk), idesc_s,
+                                   (cc | kk) != 0);
+            sm100::mma_commit(&s_full[sb]);
+            const int this_b = cs.b;
+            cs.next(seqlens, B, seqlen_cap, k);
+            if (is + 1 >= count || cs.b != this_b) sm100::mma_commit(q_empty);
+            ++is;
+            progressed = true;
+          }
         }
-        if (!ok) { *abort_flag = 1; break; }
-        sm100::mma_commit(pv_done);
-        seg_first = last_of_req;
-        ++ntile;
+        if (ip < is && sm100::mbar_test_wait(p_full, static_cast<uint32_t>(ip & 1))) {
+          sm100::tc_fence_after();
+          const bool seg_first = cp.b != prev_bp;
+          prev_bp = cp.b;
+          const int slot = static_cast<int>(ip % kAuBufs);
+          const uint32_t ta = smem_u32(ring + slot * kAuTileBytes);
+          // O^T += V^T P^T (chunks 2v, 2v+1 are value block v)
+#pragma unroll
+          for (int v = 0; v < kAuVBlocks; ++v)
+#pragma unroll
+            for (int kk = 0; kk < kAuTile / 16; ++kk)
+              sm100::mma_bf16_ss(tm_o + 64 * v,
+                                 sm100::smem_desc_mn_sw128(ta + 2 * v * kAuChunkBytes + kk * 2048, kAuChunkBytes, 1024),
+                                 sm100::smem_desc_k_sw128(pa + 32 * kk), idesc_pv, !(seg_first && kk == 0));
+          sm100::mma_commit(&tile_empty[slot]);
+          sm100::mma_commit(pv_done);
+          cp.next(seqlens, B, seqlen_cap, k);
+          ++ip;
+          progressed = true;
+        }
+        if (progressed) {
+          idle = 0;
+        } else if (++idle >= sm100::kWaitLimit || *abort_flag) {
+          if (!*abort_flag) raise_error(SD_DEVERR_TIMEOUT);
+          ok = false;
+        } else {
+          __nanosleep(32);  // leave issue slots to the epilogue warp on this scheduler
+        }
       }
+      if (!ok) *abort_flag = 1;
+      // every issued MMA completes before tensor memory is released
+      sm100::mma_commit(mma_fin);
+      sm100::mbar_wait(mma_fin, 0);
     }
+  } else {
+    // ------------------------------ row ids ------------------------------
+    // Streams each tile's resolved pool rows into a small ring, kAuRidSlots
+    // tiles ahead of the copies and the softmax.
+    AttnCursor c;
+    c.init(seqlens, B, seqlen_cap, k, first, count);
+    long long n = 0;
+    bool ok = true;
+    while (c.valid() && ok) {
+      const int rs = static_cast<int>(n % kAuRidSlots);
+      ok = sm100::mbar_wait(&rid_empty[rs], static_cast<uint32_t>((n / kAuRidSlots) & 1) ^ 1) && !*abort_flag;
+      if (!ok) break;
+      const int32_t* src = rows + (size_t)c.b * kpad + c.tile * kAuTile;
+#pragma unroll
+      for (int w = 0; w < kAuTileWords; ++w) cp_async_4(&rid[rs * kAuTile + 32 * w + lane], src + 32 * w + lane);
+      sm100::cp_async_arrive_noinc(&rid_full[rs]);
+      ++n;
+      c.next(seqlens, B, seqlen_cap, k);
+    }
+    cp_async_wait<0>();
+    if (!ok) *abort_flag = 1;
   }
 
   sm100::tc_fence_before();
@@ -433,11 +564,11 @@ __global__ void __launch_bounds__(kAuThreads, 1) attn_mla_umma_kernel(
 }
 
 // Merges the per-range partials into the bf16 output. One block per (request,
-// group of 8 heads): warp 0 finds the request's segments once (a request has
-// at most ceil(k / 256) tiles, hence at most that many covering ranges: tile i
-// of the list lies in range ((i + 1) * n_ranges - 1) / total), the (m, l) of
-// 8 heads x those segments are staged in shared memory, and each thread merges
-// 4 value columns of all 8 heads, its partial loads all in flight together.
+// group of 8 heads). Warp 0 lists the ranges that cover the request once: a
+// request has at most ceil(k / kAuTile) tiles, and tile i of the list lies in
+// range ((i + 1) * n_ranges - 1) / total. The (m, l) of 8 heads x those ranges
+// are staged in shared memory, and each thread merges 4 value columns of all
+// 8 heads, its partial loads all in flight together.
 constexpr int kAuMaxSeg = kMaxTopK / kAuTile;
 constexpr int kAuCombineHeads = 8;
 
@@ -448,6 +579,7 @@ __global__ void __launch_bounds__(128) attn_mla_umma_combine_kernel(
   const int b = blockIdx.x / HG;
   const int h0 = (blockIdx.x % HG) * kAuCombineHeads;
   __shared__ int seg_r[kAuMaxSeg];
+  __shared__ int nseg_s;
   __shared__ float2 ml_s[kAuCombineHeads][kAuMaxSeg];
   const int tid = threadIdx.x, lane = tid & 31;
   if (tid < 32) {
@@ -467,35 +599,45 @@ __global__ void __launch_bounds__(128) attn_mla_umma_combine_kernel(
       mine += __shfl_xor_sync(0xffffffffu, mine, o);
     }
     const uint32_t nr = static_cast<uint32_t>(n_ranges);
-    const uint32_t r = lane < static_cast<int>(mine) ? ((before + lane + 1) * nr - 1) / total : 0xffffffffu;
-    const uint32_t prev = __shfl_up_sync(0xffffffffu, r, 1);
-    if (lane < kAuMaxSeg) seg_r[lane] = (r != 0xffffffffu && (lane == 0 || r != prev)) ? static_cast<int>(r) : -1;
+    uint32_t carry = 0xffffffffu;  // range of the previous tile
+    int nseg = 0;
+    for (uint32_t base = 0; base < mine; base += 32) {
+      const uint32_t t = base + lane;
+      const bool has = t < mine;
+      const uint32_t r = has ? static_cast<uint32_t>(((unsigned long long)(before + t + 1) * nr - 1) / total)
+                             : 0xffffffffu;
+      uint32_t prev = __shfl_up_sync(0xffffffffu, r, 1);
+      if (lane == 0) prev = carry;
+      const bool head_of_seg = has && r != prev;
+      const uint32_t bal = __ballot_sync(0xffffffffu, head_of_seg);
+      if (head_of_seg) seg_r[nseg + __popc(bal & ((1u << lane) - 1u))] = static_cast<int>(r);
+      nseg += __popc(bal);
+      carry = __shfl_sync(0xffffffffu, r, 31);
+    }
+    if (lane == 0) nseg_s = nseg;
   }
   __syncthreads();
-  if (tid < kAuCombineHeads * kAuMaxSeg) {
-    const int hh = tid / kAuMaxSeg, j = tid % kAuMaxSeg;
-    const int r = seg_r[j];
-    ml_s[hh][j] = r >= 0 ? part_ml[((size_t)r + b) * kAuHeads + h0 + hh] : make_float2(-INFINITY, 0.f);
+  const int nseg = nseg_s;
+  for (int e = tid; e < kAuCombineHeads * nseg; e += 128) {
+    const int hh = e / nseg, jj = e % nseg;
+    ml_s[hh][jj] = part_ml[((size_t)seg_r[jj] + b) * kAuHeads + h0 + hh];
   }
   __syncthreads();
   const int d0 = 4 * tid;  // value columns d0..d0+3
-  const int hf = d0 / (kAuDv / 2), dl = d0 % (kAuDv / 2);
 #pragma unroll 2
   for (int hh = 0; hh < kAuCombineHeads; ++hh) {
     const int h = h0 + hh;
     float M = -INFINITY;
-#pragma unroll
-    for (int j = 0; j < kAuMaxSeg; ++j) M = fmaxf(M, ml_s[hh][j].x);
+    for (int jj = 0; jj < nseg; ++jj) M = fmaxf(M, ml_s[hh][jj].x);
     float denom = 0.f;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-    for (int j = 0; j < kAuMaxSeg; ++j) {
-      const float2 ml = ml_s[hh][j];
+    for (int jj = 0; jj < nseg; ++jj) {
+      const float2 ml = ml_s[hh][jj];
       if (ml.x == -INFINITY) continue;
-      const size_t slot = static_cast<size_t>(seg_r[j]) + b;
+      const size_t slot = static_cast<size_t>(seg_r[jj]) + b;
       const float wgt = exp2f(ml.x - M);
       denom += wgt * ml.y;
-      const float4 o = *reinterpret_cast<const float4*>(part_o + ((slot * 2 + hf) * kAuHeads + h) * (kAuDv / 2) + dl);
+      const float4 o = *reinterpret_cast<const float4*>(part_o + (slot * kAuHeads + h) * kAuDv + d0);
       acc.x += wgt * o.x;
       acc.y += wgt * o.y;
       acc.z += wgt * o.z;
@@ -510,10 +652,15 @@ __global__ void __launch_bounds__(128) attn_mla_umma_combine_kernel(
   }
 }
 
-inline size_t attn_umma_workspace(int B) {
+// Workspace: partial O [slots][128][512] fp32, (m, l) [slots][128], and the
+// resolved row ids [B][attn_kpad(k)] int32.
+inline size_t attn_umma_rows_offset(int B) {
   const size_t slots = static_cast<size_t>(kAuRanges) + B;
-  const size_t o = slots * 2 * kAuHeads * (kAuDv / 2) * sizeof(float);
-  return ((o + 255) / 256) * 256 + slots * kAuHeads * sizeof(float2);
+  const size_t o = ((slots * kAuHeads * kAuDv * sizeof(float) + 255) / 256) * 256;
+  return o + ((slots * kAuHeads * sizeof(float2) + 255) / 256) * 256;
+}
+inline size_t attn_umma_workspace(int B, int k) {
+  return attn_umma_rows_offset(B) + static_cast<size_t>(B) * attn_kpad(k) * sizeof(int32_t);
 }
 
 }  // namespace sd

@@ -87,7 +87,7 @@ size_t attn_bytes(int B, int G, int H, int k, int Dv) {
   const AttnPlan p = attn_plan(B, G, H, k);
   const size_t n = (size_t)B * H * p.n_splits;
   size_t bytes = align_up(sizeof(float) * n * Dv) + align_up(sizeof(float2) * n);
-  if (G == 1 && H == sd::kAuHeads && Dv == sd::kAuDv) bytes = std::max(bytes, align_up(sd::attn_umma_workspace(B)));
+  if (G == 1 && H == sd::kAuHeads && Dv == sd::kAuDv) bytes = std::max(bytes, align_up(sd::attn_umma_workspace(B, k)));
   return bytes;
 }
 
@@ -226,7 +226,7 @@ sd_status launch_indexer_umma(const int8_t* qi, const int32_t* w, const int8_t* 
 
 template <int PER>
 sd_status launch_topk_cluster(const int32_t* scores, const int32_t* seqlens, int32_t* indices, int rows, int G,
-                              int max_seqlen, int cap, int k, int cs, cudaStream_t st) {
+                              int max_seqlen, int cap, int k, int cs, const sd::RowMap& rm, cudaStream_t st) {
   const size_t smem = sizeof(sd::TopkClusterSmem<PER>);
   sd_status s = cuda_check(cudaFuncSetAttribute(sd::topk_cluster_kernel<PER>,
                                                 cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)));
@@ -244,27 +244,27 @@ sd_status launch_topk_cluster(const int32_t* scores, const int32_t* seqlens, int
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   return cuda_check(cudaLaunchKernelEx(&cfg, sd::topk_cluster_kernel<PER>, scores, seqlens, indices, G,
-                                       std::max(max_seqlen, 1), cap, k));
+                                       std::max(max_seqlen, 1), cap, k, rm));
 }
 
 // Top-k: one thread-block cluster per row when the row fits in the cluster's
 // shared memory (max_seqlen <= 8 x 512 x 32), else one CTA per row over L2.
 sd_status launch_topk(const int32_t* scores, const int32_t* seqlens, int32_t* indices, int B, int G,
-                      int max_seqlen, int cap, int k, cudaStream_t st) {
+                      int max_seqlen, int cap, int k, const sd::RowMap& rm, cudaStream_t st) {
   const int rows = B * G;
   const int cs16 = sd::topk_cluster_size(max_seqlen, 16);
   const int cs32 = sd::topk_cluster_size(max_seqlen, 32);
   stage_mark(kStageTopk, 0, st);
   if ((cs16 > 0 || cs32 > 0) && rows <= 65535) {
     // 32 scores per thread measured faster than 16 (fewer CTAs per cluster)
-    const sd_status s = cs32 > 0 ? launch_topk_cluster<32>(scores, seqlens, indices, rows, G, max_seqlen, cap, k, cs32, st)
-                                 : launch_topk_cluster<16>(scores, seqlens, indices, rows, G, max_seqlen, cap, k, cs16, st);
+    const sd_status s = cs32 > 0 ? launch_topk_cluster<32>(scores, seqlens, indices, rows, G, max_seqlen, cap, k, cs32, rm, st)
+                                 : launch_topk_cluster<16>(scores, seqlens, indices, rows, G, max_seqlen, cap, k, cs16, rm, st);
     stage_mark(kStageTopk, 1, st);
     ++t_launches;
     return s;
   }
   sd::topk_radix_kernel<<<rows, sd::kTopkThreads, 0, st>>>(scores, seqlens, indices, G,
-                                                           std::max(max_seqlen, 1), cap, k);
+                                                           std::max(max_seqlen, 1), cap, k, rm);
   stage_mark(kStageTopk, 1, st);
   return after_launch();
 }
@@ -272,7 +272,7 @@ sd_status launch_topk(const int32_t* scores, const int32_t* seqlens, int32_t* in
 sd_status launch_indexer_topk(const int8_t* qi, const int32_t* w, const int8_t* ki, const int32_t* bt,
                               const int32_t* seqlens, const sd_paged_desc& pd, int B, int Hi, int Di,
                               int max_seqlen, int k, int32_t* indices, int32_t* scores,
-                              cudaStream_t st) {
+                              cudaStream_t st, const sd::RowMap& rm = sd::RowMap{}) {
   const int G = pd.kv_heads;
   if (B == 0) return SD_OK;
   bool done = false;
@@ -288,7 +288,7 @@ sd_status launch_indexer_topk(const int8_t* qi, const int32_t* w, const int8_t* 
     if (s != SD_OK) return s;
   }
   const int cap = std::min(max_seqlen, pd.max_pages_per_req * pd.page_size);
-  return launch_topk(scores, seqlens, indices, B, G, max_seqlen, cap, k, st);
+  return launch_topk(scores, seqlens, indices, B, G, max_seqlen, cap, k, rm, st);
 }
 
 template <int DK, int DV, int MT>
@@ -320,27 +320,35 @@ sd_status launch_attn_t(const uint16_t* q, const uint16_t* kp, const uint16_t* v
   return after_launch();
 }
 
+// `rows_ready`: the top-k already resolved the selections to pool rows in the
+// workspace's row array; otherwise a small kernel does it first.
 sd_status launch_attn_umma(const uint16_t* q, const uint16_t* kp, const int32_t* bt, const int32_t* seqlens,
                            const int32_t* indices, const sd_paged_desc& pd, int B, int k, float scale,
-                           uint16_t* out, float* lse, void* ws, int seqlen_cap, cudaStream_t st) {
+                           uint16_t* out, float* lse, void* ws, int seqlen_cap, bool rows_ready, cudaStream_t st) {
   using Lay = sd::AttnUmmaLayout;
   const size_t slots = static_cast<size_t>(sd::kAuRanges) + B;
   float* part_o = static_cast<float*>(ws);
   float2* part_ml = reinterpret_cast<float2*>(
-      static_cast<char*>(ws) + align_up(slots * 2 * sd::kAuHeads * (sd::kAuDv / 2) * sizeof(float)));
-  CUtensorMap tm_q, tm_kv;
-  const uint64_t rows = (uint64_t)pd.num_pages * pd.page_size;
-  if (!encode_bf16_rows(&tm_q, q, sd::kAuDk, (uint64_t)B * sd::kAuHeads, sd::kAuDk * 2, 64, sd::kAuHeads) ||
-      !encode_bf16_rows(&tm_kv, kp, sd::kAuDk, rows, sd::kAuDk * 2, 64, 1) || rows >= (1ull << 31))
+      static_cast<char*>(ws) + align_up(slots * sd::kAuHeads * sd::kAuDv * sizeof(float)));
+  int32_t* rows = reinterpret_cast<int32_t*>(static_cast<char*>(ws) + sd::attn_umma_rows_offset(B));
+  CUtensorMap tm_q;
+  const uint64_t pool_rows = (uint64_t)pd.num_pages * pd.page_size;
+  if (!encode_bf16_rows(&tm_q, q, sd::kAuDk, (uint64_t)B * sd::kAuHeads, sd::kAuDk * 2, 64, sd::kAuHalfHeads) ||
+      (reinterpret_cast<uintptr_t>(kp) & 15u) != 0 || pool_rows >= (1ull << 31))
     return SD_ERR_UNSUPPORTED;
   sd_status s = cuda_check(cudaFuncSetAttribute(sd::attn_mla_umma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                 static_cast<int>(Lay::kSmemAlloc)));
   if (s != SD_OK) return s;
   const float scale_log2 = scale * 1.4426950408889634f;
   stage_mark(kStageAttn, 0, st);
+  if (!rows_ready) {
+    const dim3 grid((sd::attn_kpad(k) + 255) / 256, B);
+    sd::attn_rows_kernel<<<grid, 256, 0, st>>>(indices, bt, seqlens, k, seqlen_cap, pd.page_size,
+                                               pd.max_pages_per_req, pd.num_pages, rows);
+    if ((s = after_launch()) != SD_OK) return s;
+  }
   sd::attn_mla_umma_kernel<<<2 * sd::kAuRanges, sd::kAuThreads, Lay::kSmemAlloc, st>>>(
-      tm_q, tm_kv, reinterpret_cast<const __nv_bfloat16*>(kp), bt, seqlens, indices, B, k, pd.num_pages,
-      pd.page_size, pd.max_pages_per_req, seqlen_cap, scale_log2, part_o, part_ml);
+      tm_q, reinterpret_cast<const __nv_bfloat16*>(kp), seqlens, rows, B, k, seqlen_cap, scale_log2, part_o, part_ml);
   stage_mark(kStageAttn, 1, st);
   if ((s = after_launch()) != SD_OK) return s;
   stage_mark(kStageCombine, 0, st);
@@ -353,10 +361,11 @@ sd_status launch_attn_umma(const uint16_t* q, const uint16_t* kp, const int32_t*
 sd_status launch_attn(const uint16_t* q, const uint16_t* kp, const uint16_t* vp, const int32_t* bt,
                       const int32_t* seqlens, const int32_t* indices, const sd_paged_desc& pd, int B,
                       int H, int Dk, int Dv, int k, float scale, uint16_t* out, float* lse,
-                      void* ws, int seqlen_cap, cudaStream_t st) {
+                      void* ws, int seqlen_cap, cudaStream_t st, bool rows_ready = false) {
   if (B == 0) return SD_OK;
   if (umma_attn_fits(pd.kv_heads, H, Dk, Dv, vp != nullptr)) {
-    const sd_status su = launch_attn_umma(q, kp, bt, seqlens, indices, pd, B, k, scale, out, lse, ws, seqlen_cap, st);
+    const sd_status su =
+        launch_attn_umma(q, kp, bt, seqlens, indices, pd, B, k, scale, out, lse, ws, seqlen_cap, rows_ready, st);
     if (su != SD_ERR_UNSUPPORTED) return su;  // else: pointers the TMA cannot map; take the mma.sync kernel
   }
   const AttnPlan p = attn_plan(B, pd.kv_heads, H, k);
@@ -434,13 +443,23 @@ sd_status sd_decode_step(const int8_t* qi, const int32_t* w, const int8_t* ki_pa
     return SD_ERR_WORKSPACE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   int32_t* sc = scores ? scores : static_cast<int32_t*>(workspace);
+  void* attn_ws = static_cast<char*>(workspace) + sb;
+  // With the tensor-core attention, the top-k also resolves each selection to
+  // its pool row (one block-table load per selected token, off the
+  // attention's gather path).
+  const bool umma = umma_attn_fits(pd.kv_heads, H, Dk, Dv, v_pages != nullptr) && B > 0 &&
+                    (reinterpret_cast<uintptr_t>(q) & 15u) == 0 && (reinterpret_cast<uintptr_t>(k_pages) & 15u) == 0;
+  sd::RowMap rm{};
+  if (umma)
+    rm = sd::RowMap{reinterpret_cast<int32_t*>(static_cast<char*>(attn_ws) + sd::attn_umma_rows_offset(B)),
+                    block_table, pd.page_size, pd.max_pages_per_req, pd.num_pages, sd::attn_kpad(k)};
   s = launch_indexer_topk(qi, w, ki_pages, block_table, seqlens, pd, B, Hi, Di, max_seqlen, k, indices,
-                          sc, st);
+                          sc, st, rm);
   if (s != SD_OK) return s;
   const int launches = t_launches;
   const int cap = std::min(max_seqlen, pd.max_pages_per_req * pd.page_size);
   s = launch_attn(q, k_pages, v_pages, block_table, seqlens, indices, pd, B, H, Dk, Dv, k, scale, out,
-                  lse, static_cast<char*>(workspace) + sb, cap, st);
+                  lse, attn_ws, cap, st, umma);
   t_launches += launches;
   return s;
 }

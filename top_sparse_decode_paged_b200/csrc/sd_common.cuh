@@ -29,12 +29,44 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
+// Optional second output of the top-k: each selected token resolved to its
+// pool row (page * page_size + slot) through the block table, [rows][kpad]
+// with -1 for empty slots, so that the attention's gathers need no dependent
+// block-table load. rows == nullptr disables it.
+struct RowMap {
+  int32_t* rows;
+  const int32_t* block_table;
+  int page_size, max_pages, num_pages, kpad;
+  // `pcache` holds the last (block-table index, page) looked up by this
+  // thread: a thread's selections are ascending and mostly share a page.
+  __device__ __forceinline__ void put(int row, int b, int slot, int token, int2& pcache) const {
+    if (rows == nullptr) return;
+    int r = -1;
+    if (token >= 0) {
+      const int pi = token / page_size;
+      if (pi != pcache.x) pcache = make_int2(pi, block_table[(size_t)b * max_pages + pi]);
+      const int page = pcache.y;
+      if (page >= 0 && page < num_pages) {
+        r = page * page_size + token % page_size;
+      } else {
+        raise_error(SD_DEVERR_PAGE);
+      }
+    }
+    rows[(size_t)row * kpad + slot] = r;
+  }
+};
+
 // 16-byte global->shared async copy; src_bytes = 0 writes zeros.
 __device__ __forceinline__ void cp_async_16(void* smem_dst, const void* gmem_src, int src_bytes) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(smem_u32(smem_dst)),
                "l"(gmem_src), "r"(src_bytes)
                : "memory");
 }
+// 4-byte cp.async (through L1), for small index blocks of any alignment.
+__device__ __forceinline__ void cp_async_4(void* smem_dst, const void* gmem_src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;\n" ::"r"(smem_u32(smem_dst)), "l"(gmem_src) : "memory");
+}
+
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
 template <int N>
 __device__ __forceinline__ void cp_async_wait() {

@@ -100,7 +100,7 @@ __device__ __forceinline__ uint32_t tk_block_reduce(uint32_t v, uint32_t* scratc
 template <int PER>
 __global__ void __launch_bounds__(kTkThreads, 2) topk_cluster_kernel(
     const int32_t* __restrict__ scores, const int32_t* __restrict__ seqlens, int32_t* __restrict__ indices,
-    int G, int max_seqlen, int seqlen_cap, int k) {
+    int G, int max_seqlen, int seqlen_cap, int k, RowMap rm) {
   constexpr int kTkPerThread = PER;
   constexpr int kTkChunkStride = PER + 1;
   extern __shared__ __align__(16) uint8_t tk_smem_raw[];
@@ -113,11 +113,17 @@ __global__ void __launch_bounds__(kTkThreads, 2) topk_cluster_kernel(
   const int tid = threadIdx.x;
   const int L = checked_seqlen(seqlens, b, seqlen_cap);
   int32_t* out = indices + (size_t)row * k;
+  int2 pc = make_int2(-1, 0);  // last block-table lookup (row ids)
 
   if (L <= k) {  // uniform over the cluster: no cluster barrier is reached
-    for (int i = crank * kTkThreads + tid; i < k; i += CS * kTkThreads) out[i] = i < L ? i : -1;
+    const int n = rm.rows != nullptr ? max(k, rm.kpad) : k;
+    for (int i = crank * kTkThreads + tid; i < n; i += CS * kTkThreads) {
+      if (i < k) out[i] = i < L ? i : -1;
+      rm.put(row, b, i, i < L ? i : -1, pc);
+    }
     return;
   }
+
 
   const int slice = ceil_div(ceil_div(L, CS), kTkThreads) * kTkThreads;  // <= kTkSlice by launch
   const int s0 = crank * slice;
@@ -278,6 +284,10 @@ __global__ void __launch_bounds__(kTkThreads, 2) topk_cluster_kernel(
     }
   }
   cluster.sync();  // no CTA leaves while others may still read its shared memory
+  // optional row ids: a separate pass over the finished output (written by
+  // the whole cluster before the barrier), one block-table load per page run
+  if (rm.rows != nullptr)
+    for (int i = crank * kTkThreads + tid; i < rm.kpad; i += CS * kTkThreads) rm.put(row, b, i, i < k ? out[i] : -1, pc);
 }
 
 // Cluster size for rows of up to max_seqlen scores with PER scores per thread

@@ -52,7 +52,7 @@ __device__ __forceinline__ int block_excl_scan_flag(bool flag, uint32_t* warp_su
 
 __global__ void __launch_bounds__(kTopkThreads) topk_radix_kernel(
     const int32_t* __restrict__ scores, const int32_t* __restrict__ seqlens, int32_t* __restrict__ indices,
-    int G, int max_seqlen, int seqlen_cap, int k) {
+    int G, int max_seqlen, int seqlen_cap, int k, RowMap rm) {
   __shared__ uint32_t hist[256];
   __shared__ uint32_t scan_scratch[kTopkWarps + 1];
   __shared__ int sel_digit, sel_remaining;
@@ -62,11 +62,17 @@ __global__ void __launch_bounds__(kTopkThreads) topk_radix_kernel(
   const int L = checked_seqlen(seqlens, b, seqlen_cap);
   const int32_t* s = scores + (size_t)row * max_seqlen;
   int32_t* out = indices + (size_t)row * k;
+  int2 pc = make_int2(-1, 0);  // last block-table lookup (row ids)
 
   if (L <= k) {  // everything is selected: 0..L-1 then -1
-    for (int i = threadIdx.x; i < k; i += kTopkThreads) out[i] = i < L ? i : -1;
+    const int n = rm.rows != nullptr ? max(k, rm.kpad) : k;
+    for (int i = threadIdx.x; i < n; i += kTopkThreads) {
+      if (i < k) out[i] = i < L ? i : -1;
+      rm.put(row, b, i, i < L ? i : -1, pc);
+    }
     return;
   }
+
 
   uint32_t prefix = 0, prefix_mask = 0;
   int remaining = k;  // how many still to take among keys that match `prefix`
@@ -132,6 +138,10 @@ __global__ void __launch_bounds__(kTopkThreads) topk_radix_kernel(
     if (take) out[pos] = i;
     taken_eq += eq_total;
     written += take_total;
+  }
+  if (rm.rows != nullptr) {
+    __syncthreads();  // the output above is complete
+    for (int i = threadIdx.x; i < rm.kpad; i += kTopkThreads) rm.put(row, b, i, i < k ? out[i] : -1, pc);
   }
 }
 

@@ -564,23 +564,20 @@ __global__ void __launch_bounds__(kAuThreads, 1) attn_mla_umma_kernel(
 }
 
 // Merges the per-range partials into the bf16 output. One block per (request,
-// group of 8 heads). Warp 0 lists the ranges that cover the request once: a
-// request has at most ceil(k / kAuTile) tiles, and tile i of the list lies in
-// range ((i + 1) * n_ranges - 1) / total. The (m, l) of 8 heads x those ranges
-// are staged in shared memory, and each thread merges 4 value columns of all
-// 8 heads, its partial loads all in flight together.
+// head), 128 threads of 4 value columns each. Warp 0 lists the ranges that
+// cover the request: a request has at most ceil(k / kAuTile) tiles, and tile
+// i of the list lies in range ((i + 1) * n_ranges - 1) / total. Each thread
+// then issues the loads of all its partials together.
 constexpr int kAuMaxSeg = kMaxTopK / kAuTile;
-constexpr int kAuCombineHeads = 8;
 
 __global__ void __launch_bounds__(128) attn_mla_umma_combine_kernel(
     const float* __restrict__ part_o, const float2* __restrict__ part_ml, const int32_t* __restrict__ seqlens,
     int B, int k, int seqlen_cap, int n_ranges, __nv_bfloat16* __restrict__ out, float* __restrict__ lse) {
-  constexpr int HG = kAuHeads / kAuCombineHeads;
-  const int b = blockIdx.x / HG;
-  const int h0 = (blockIdx.x % HG) * kAuCombineHeads;
+  const int b = blockIdx.x / kAuHeads;
+  const int h = blockIdx.x % kAuHeads;
   __shared__ int seg_r[kAuMaxSeg];
+  __shared__ float2 ml_s[kAuMaxSeg];
   __shared__ int nseg_s;
-  __shared__ float2 ml_s[kAuCombineHeads][kAuMaxSeg];
   const int tid = threadIdx.x, lane = tid & 31;
   if (tid < 32) {
     uint32_t before = 0, total = 0, mine = 0;
@@ -610,7 +607,11 @@ __global__ void __launch_bounds__(128) attn_mla_umma_combine_kernel(
       if (lane == 0) prev = carry;
       const bool head_of_seg = has && r != prev;
       const uint32_t bal = __ballot_sync(0xffffffffu, head_of_seg);
-      if (head_of_seg) seg_r[nseg + __popc(bal & ((1u << lane) - 1u))] = static_cast<int>(r);
+      const int at = nseg + __popc(bal & ((1u << lane) - 1u));
+      if (head_of_seg) {
+        seg_r[at] = static_cast<int>(r);
+        ml_s[at] = part_ml[((size_t)r + b) * kAuHeads + h];
+      }
       nseg += __popc(bal);
       carry = __shfl_sync(0xffffffffu, r, 31);
     }
@@ -618,38 +619,30 @@ __global__ void __launch_bounds__(128) attn_mla_umma_combine_kernel(
   }
   __syncthreads();
   const int nseg = nseg_s;
-  for (int e = tid; e < kAuCombineHeads * nseg; e += 128) {
-    const int hh = e / nseg, jj = e % nseg;
-    ml_s[hh][jj] = part_ml[((size_t)seg_r[jj] + b) * kAuHeads + h0 + hh];
-  }
-  __syncthreads();
   const int d0 = 4 * tid;  // value columns d0..d0+3
-#pragma unroll 2
-  for (int hh = 0; hh < kAuCombineHeads; ++hh) {
-    const int h = h0 + hh;
-    float M = -INFINITY;
-    for (int jj = 0; jj < nseg; ++jj) M = fmaxf(M, ml_s[hh][jj].x);
-    float denom = 0.f;
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int jj = 0; jj < nseg; ++jj) {
-      const float2 ml = ml_s[hh][jj];
-      if (ml.x == -INFINITY) continue;
-      const size_t slot = static_cast<size_t>(seg_r[jj]) + b;
-      const float wgt = exp2f(ml.x - M);
-      denom += wgt * ml.y;
-      const float4 o = *reinterpret_cast<const float4*>(part_o + (slot * kAuHeads + h) * kAuDv + d0);
-      acc.x += wgt * o.x;
-      acc.y += wgt * o.y;
-      acc.z += wgt * o.z;
-      acc.w += wgt * o.w;
-    }
-    const float inv = denom > 0.f ? 1.f / denom : 0.f;
-    __nv_bfloat162* o2 = reinterpret_cast<__nv_bfloat162*>(out + ((size_t)b * kAuHeads + h) * kAuDv + d0);
-    o2[0] = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
-    o2[1] = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
-    if (lse != nullptr && tid == 0)
-      lse[(size_t)b * kAuHeads + h] = denom > 0.f ? (M + log2f(denom)) * 0.69314718055994530942f : -INFINITY;
+  float M = -INFINITY;
+  for (int jj = 0; jj < nseg; ++jj) M = fmaxf(M, ml_s[jj].x);
+  float denom = 0.f;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
+  for (int jj = 0; jj < nseg; ++jj) {
+    const float2 ml = ml_s[jj];
+    if (ml.x == -INFINITY) continue;
+    const size_t slot = static_cast<size_t>(seg_r[jj]) + b;
+    const float wgt = exp2f(ml.x - M);
+    denom += wgt * ml.y;
+    const float4 o = *reinterpret_cast<const float4*>(part_o + (slot * kAuHeads + h) * kAuDv + d0);
+    acc.x += wgt * o.x;
+    acc.y += wgt * o.y;
+    acc.z += wgt * o.z;
+    acc.w += wgt * o.w;
   }
+  const float inv = denom > 0.f ? 1.f / denom : 0.f;
+  __nv_bfloat162* o2 = reinterpret_cast<__nv_bfloat162*>(out + ((size_t)b * kAuHeads + h) * kAuDv + d0);
+  o2[0] = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
+  o2[1] = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
+  if (lse != nullptr && tid == 0)
+    lse[(size_t)b * kAuHeads + h] = denom > 0.f ? (M + log2f(denom)) * 0.69314718055994530942f : -INFINITY;
 }
 
 // Workspace: partial O [slots][128][512] fp32, (m, l) [slots][128], and the

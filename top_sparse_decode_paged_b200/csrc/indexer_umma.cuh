@@ -29,23 +29,30 @@ namespace sd {
 
 constexpr int kUmmaTile = 128;     // tokens per tile (MMA M)
 constexpr int kUmmaRowBytes = 128; // Di = 128 int8
-constexpr int kUmmaStages = 8;
+constexpr int kUmmaStages = 6;
+constexpr int kUmmaTilesPerStage = 2;  // consecutive tiles of one request share a stage
+constexpr int kUmmaAccs = 2;       // accumulators in tensor memory
 constexpr int kUmmaThreads = 192;
 
 template <int HI>
 struct IndexerUmmaLayout {
   static constexpr int kTileBytes = kUmmaTile * kUmmaRowBytes;  // 16 KB
+  static constexpr int kStageBytes = kUmmaTilesPerStage * kTileBytes;
   static constexpr int kQBytes = HI * kUmmaRowBytes;
-  static constexpr int kTmemCols = (2 * HI) <= 32 ? 32 : ((2 * HI) <= 64 ? 64 : ((2 * HI) <= 128 ? 128 : 256));
-  static constexpr int kOffQ = kUmmaStages * kTileBytes;
+  static constexpr int kAccCols = kUmmaAccs * HI;
+  static constexpr int kTmemCols = kAccCols <= 32 ? 32 : (kAccCols <= 64 ? 64 : (kAccCols <= 128 ? 128 : (kAccCols <= 256 ? 256 : 512)));
+  static constexpr int kOffQ = kUmmaStages * kStageBytes;
   static constexpr int kOffBar = kOffQ + 2 * kQBytes;
-  static constexpr int kNumBars = 2 * kUmmaStages + 2 + 2 + 2 + 2;
+  static constexpr int kNumBars = 2 * kUmmaStages + 2 + 2 + 2 * kUmmaAccs;
   static constexpr int kOffMisc = kOffBar + 8 * kNumBars;
   static constexpr int kBytes = kOffMisc + 16;
   static constexpr size_t kSmemAlloc = kBytes + 1024;  // slack to align the base to 1024 B
 };
 
 // Walks a contiguous range of the global tile list (request-major).
+struct TileCursor;
+__device__ __forceinline__ bool stage_pairs(const TileCursor& c);
+
 struct TileCursor {
   int b, tile, tiles_b, L;
   long long remaining;
@@ -76,6 +83,12 @@ struct TileCursor {
   }
 };
 
+// A stage takes the cursor's tile and, when the range continues within the
+// same request, the next one (whose tile is then a full 128 tokens before it).
+__device__ __forceinline__ bool stage_pairs(const TileCursor& c) {
+  return kUmmaTilesPerStage == 2 && c.remaining > 1 && c.tile + 1 < c.tiles_b;
+}
+
 __device__ __forceinline__ long long total_tiles(const int32_t* seqlens, int B, int cap) {
   long long n = 0;
   for (int b = 0; b < B; ++b) {
@@ -104,7 +117,7 @@ __global__ void __launch_bounds__(kUmmaThreads, 1) indexer_umma_kernel(
   uint64_t* qfull = bars + 2 * kUmmaStages;
   uint64_t* qempty = qfull + 2;
   uint64_t* accfull = qempty + 2;
-  uint64_t* accempty = accfull + 2;
+  uint64_t* accempty = accfull + kUmmaAccs;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Lay::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Lay::kOffMisc + 4);
 
@@ -119,6 +132,8 @@ __global__ void __launch_bounds__(kUmmaThreads, 1) indexer_umma_kernel(
     for (int i = 0; i < 2; ++i) {
       sm100::mbar_init(&qfull[i], 1);
       sm100::mbar_init(&qempty[i], 1);
+    }
+    for (int i = 0; i < kUmmaAccs; ++i) {
       sm100::mbar_init(&accfull[i], 1);
       sm100::mbar_init(&accempty[i], 128);
     }
@@ -145,21 +160,29 @@ __global__ void __launch_bounds__(kUmmaThreads, 1) indexer_umma_kernel(
   if (warp == 0) {
     // ---------------- TMA producer (whole warp) ----------------
     // The 32 lanes keep a window of 32 consecutive block-table entries of the
-    // current request, fetched in one coalesced load, so the page lookups of
-    // 16+ tiles cost one memory round trip. Lane j issues the copy of the
-    // tile's j-th page; lane 0 does the barrier bookkeeping.
+    // current request (and the next window, loaded ahead), fetched in one
+    // coalesced load, so the page lookups of 16+ tiles cost one memory round
+    // trip. Windows start at tile boundaries, so the pages of a tile are
+    // consecutive lanes: each such lane copies its own page. A page outside
+    // the pool is copied from past the end of the tensor (zero fill), which
+    // keeps the byte count of every stage fixed; the epilogue marks its
+    // tokens invalid.
     TileCursor c;
     c.init(seqlens, B, cap, first, count);
     int stage = 0;
     uint32_t phase = 0;
     int nq = 0, cur_b = -1;
+    const int pshift = __ffs(page_size) - 1;  // page sizes on this path are powers of two
+    const uint32_t page_bytes = static_cast<uint32_t>(page_size) * kUmmaRowBytes;
+    const int oob_row = num_pages * page_size;
     int win_b = -1, win_p0 = 0, win_val = -1;
-    while (c.valid() && !*abort_flag) {
+    int nxt_p0 = -1, nxt_val = -1;  // the following window of the same request, loaded ahead
+    while (c.valid()) {
       if (c.b != cur_b) {
         const int slot = nq & 1;
         bool ok = true;
         if (lane == 0) {
-          ok = sm100::mbar_wait(&qempty[slot], ((nq >> 1) & 1) ^ 1);
+          ok = sm100::mbar_wait(&qempty[slot], ((nq >> 1) & 1) ^ 1) && !*abort_flag;
           if (ok) {
             sm100::mbar_arrive_expect_tx(&qfull[slot], Lay::kQBytes);
             sm100::tma_load_2d(qbuf + slot * Lay::kQBytes, &tm_q, &qfull[slot], 0, c.b * HI);
@@ -173,31 +196,39 @@ __global__ void __launch_bounds__(kUmmaThreads, 1) indexer_umma_kernel(
         ++nq;
       }
       const int t0 = c.tile * kUmmaTile;
-      const int p_first = t0 / page_size;
-      const int npages = ceil_div(min(kUmmaTile, c.L - t0), page_size);
-      if (c.b != win_b || p_first < win_p0 || p_first + npages > win_p0 + 32) {
+      const int p_first = t0 >> pshift;
+      const bool two = stage_pairs(c);
+      const int npages = (min(kUmmaTile * (two ? 2 : 1), c.L - t0) + page_size - 1) >> pshift;
+      if (c.b != win_b || p_first + npages > win_p0 + 32) {
+        if (c.b == win_b && p_first == nxt_p0) {
+          win_val = nxt_val;  // loaded one window ago: no round trip on this path
+        } else {
+          const int p = p_first + lane;
+          win_val = p < max_pages ? block_table[(size_t)c.b * max_pages + p] : -1;
+        }
         win_b = c.b;
         win_p0 = p_first;
-        const int p = win_p0 + lane;
-        win_val = p < max_pages ? block_table[(size_t)c.b * max_pages + p] : -1;
+        nxt_p0 = win_p0 + 32;
+        const int pn = nxt_p0 + lane;
+        nxt_val = pn < max_pages ? block_table[(size_t)c.b * max_pages + pn] : -1;
       }
-      const int phys = __shfl_sync(0xffffffffu, win_val, min(p_first - win_p0 + lane, 31));
-      const bool mine = lane < npages && phys >= 0 && phys < num_pages;
-      const uint32_t vmask = __ballot_sync(0xffffffffu, mine);
+      const int off = lane - (p_first - win_p0);  // this lane's page within the tile
       bool ok = true;
       if (lane == 0) {
-        ok = sm100::mbar_wait(&empty[stage], phase ^ 1);
-        if (ok) sm100::mbar_arrive_expect_tx(&full[stage], __popc(vmask) * page_size * kUmmaRowBytes);
+        ok = sm100::mbar_wait(&empty[stage], phase ^ 1) && (stage != 0 || !*abort_flag);
+        if (ok) sm100::mbar_arrive_expect_tx(&full[stage], static_cast<uint32_t>(npages) * page_bytes);
       }
       if (!__shfl_sync(0xffffffffu, ok, 0)) {
         if (lane == 0) *abort_flag = 1;
         break;
       }
-      if (mine)
-        sm100::tma_load_2d(kstage + stage * Lay::kTileBytes + lane * page_size * kUmmaRowBytes, &tm_keys,
-                           &full[stage], 0, phys * page_size);
+      if (off >= 0 && off < npages) {
+        const int row = (win_val >= 0 && win_val < num_pages) ? win_val * page_size : oob_row;
+        sm100::tma_load_2d(kstage + stage * Lay::kStageBytes + off * page_bytes, &tm_keys, &full[stage], 0, row);
+      }
       if (++stage == kUmmaStages) { stage = 0; phase ^= 1; }
       c.next(seqlens, B, cap);
+      if (two) c.next(seqlens, B, cap);
     }
   } else if (warp == 1) {
     // ---------------- MMA issuer ----------------
@@ -215,27 +246,37 @@ __global__ void __launch_bounds__(kUmmaThreads, 1) indexer_umma_kernel(
           ++nq;
         }
         const int slot = (nq - 1) & 1;
-        if (!sm100::mbar_wait(&accempty[acc], accphase ^ 1)) { *abort_flag = 1; break; }
+        const int ntiles = stage_pairs(c) ? 2 : 1;
         if (!sm100::mbar_wait(&full[stage], phase)) { *abort_flag = 1; break; }
-        sm100::tc_fence_after();
-        const uint32_t a0 = smem_u32(kstage + stage * Lay::kTileBytes);
         const uint32_t b0 = smem_u32(qbuf + slot * Lay::kQBytes);
-        const uint32_t d = tmem_base + acc * HI;
+        bool ok = true;
+        for (int j = 0; j < ntiles; ++j) {
+          if (!sm100::mbar_wait(&accempty[acc], accphase ^ 1)) { ok = false; break; }
+          sm100::tc_fence_after();
+          const uint32_t a0 = smem_u32(kstage + stage * Lay::kStageBytes + j * Lay::kTileBytes);
+          const uint32_t d = tmem_base + acc * HI;
 #pragma unroll
-        for (int k = 0; k < kUmmaRowBytes / 32; ++k)
-          sm100::mma_i8_ss(d, sm100::smem_desc_k_sw128(a0 + 32 * k), sm100::smem_desc_k_sw128(b0 + 32 * k),
-                           idesc, k > 0);
+          for (int k = 0; k < kUmmaRowBytes / 32; ++k)
+            sm100::mma_i8_ss(d, sm100::smem_desc_k_sw128(a0 + 32 * k), sm100::smem_desc_k_sw128(b0 + 32 * k),
+                             idesc, k > 0);
+          sm100::mma_commit(&accfull[acc]);
+          if (++acc == kUmmaAccs) { acc = 0; accphase ^= 1; }
+        }
+        if (!ok) { *abort_flag = 1; break; }
         sm100::mma_commit(&empty[stage]);
-        sm100::mma_commit(&accfull[acc]);
         const int this_b = c.b;
         c.next(seqlens, B, cap);
+        if (ntiles == 2) c.next(seqlens, B, cap);
         if (!c.valid() || c.b != this_b) sm100::mma_commit(&qempty[slot]);
         if (++stage == kUmmaStages) { stage = 0; phase ^= 1; }
-        if (++acc == 2) { acc = 0; accphase ^= 1; }
       }
     }
   } else {
     // ---------------- epilogue: ReLU, weighted head sum, store ----------------
+    // The accumulator is released as soon as its row is in registers; the
+    // block-table entry that validates this thread's token is loaded one tile
+    // ahead, so neither the tensor-memory round trip nor that load sits
+    // between two accumulators.
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
     TileCursor c;
@@ -244,6 +285,12 @@ __global__ void __launch_bounds__(kUmmaThreads, 1) indexer_umma_kernel(
     uint32_t accphase = 0;
     int cur_b = -1;
     int32_t wreg[HI];
+    const int pshift = __ffs(page_size) - 1;  // page sizes on this path are powers of two
+    auto page_of = [&](const TileCursor& cc) -> int {
+      const int t = cc.tile * kUmmaTile + row;
+      return (cc.valid() && t < cc.L) ? block_table[(size_t)cc.b * max_pages + (t >> pshift)] : 0;
+    };
+    int phys_next = page_of(c);
     while (c.valid() && !*abort_flag) {
       if (c.b != cur_b) {
 #pragma unroll
@@ -251,23 +298,29 @@ __global__ void __launch_bounds__(kUmmaThreads, 1) indexer_umma_kernel(
         cur_b = c.b;
       }
       const int t = c.tile * kUmmaTile + row;
-      int phys = 0;
-      if (t < c.L) phys = block_table[(size_t)c.b * max_pages + t / page_size];  // overlaps the wait
+      const int phys = phys_next;
+      TileCursor cn = c;
+      cn.next(seqlens, B, cap);
+      phys_next = page_of(cn);
       const bool ok = sm100::mbar_wait(&accfull[acc], accphase);
       __syncwarp();  // tcgen05.ld is warp-collective: reconverge after the polling loop
       if (!ok) { *abort_flag = 1; break; }
       sm100::tc_fence_after();
-      int32_t s = 0;
+      uint32_t r[HI];
 #pragma unroll
-      for (int j = 0; j < HI / 32; ++j) {
-        uint32_t r[32];
-        sm100::tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + acc * HI + j * 32, r);
-        sm100::tmem_ld_wait();
-#pragma unroll
-        for (int i = 0; i < 32; ++i) s += wreg[j * 32 + i] * max(static_cast<int32_t>(r[i]), 0);
-      }
+      for (int j = 0; j < HI / 32; ++j)
+        sm100::tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + acc * HI + j * 32,
+                                  *reinterpret_cast<uint32_t(*)[32]>(r + 32 * j));
+      sm100::tmem_ld_wait();
       sm100::tc_fence_before();
       sm100::mbar_arrive(&accempty[acc]);
+      // eight independent partial sums (a single chain would serialize 64 IMADs)
+      int32_t part[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+#pragma unroll
+      for (int i = 0; i < HI; ++i) part[i & 7] += wreg[i] * max(static_cast<int32_t>(r[i]), 0);
+      const int32_t s0 = (part[0] + part[1]) + (part[2] + part[3]);
+      const int32_t s1 = (part[4] + part[5]) + (part[6] + part[7]);
+      int32_t s = s0 + s1;
       if (t < c.L) {
         if (phys < 0 || phys >= num_pages) {
           raise_error(SD_DEVERR_PAGE);
@@ -275,8 +328,8 @@ __global__ void __launch_bounds__(kUmmaThreads, 1) indexer_umma_kernel(
         }
         scores[(size_t)c.b * max_seqlen + t] = s;
       }
-      if (++acc == 2) { acc = 0; accphase ^= 1; }
-      c.next(seqlens, B, cap);
+      if (++acc == kUmmaAccs) { acc = 0; accphase ^= 1; }
+      c = cn;
     }
   }
 

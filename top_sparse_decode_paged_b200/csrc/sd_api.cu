@@ -199,6 +199,7 @@ int sm_count() {
 bool umma_indexer_fits(const sd_paged_desc& pd, int Hi, int Di, const void* qi, const void* ki) {
   const int P = pd.page_size;
   return pd.kv_heads == 1 && Di == 128 && Hi == 64 && P >= 8 && P <= 128 && (128 % P) == 0 &&
+         (long long)(pd.num_pages + 1) * P < (1ll << 31) &&  // TMA row coordinates, one page past the end included
          (reinterpret_cast<uintptr_t>(qi) & 15u) == 0 && (reinterpret_cast<uintptr_t>(ki) & 15u) == 0;
 }
 
@@ -352,7 +353,7 @@ sd_status launch_attn_umma(const uint16_t* q, const uint16_t* kp, const int32_t*
   stage_mark(kStageAttn, 1, st);
   if ((s = after_launch()) != SD_OK) return s;
   stage_mark(kStageCombine, 0, st);
-  sd::attn_mla_umma_combine_kernel<<<B * (sd::kAuHeads / sd::kAuCombineHeads), 128, 0, st>>>(
+  sd::attn_mla_umma_combine_kernel<<<B * sd::kAuHeads, 128, 0, st>>>(
       part_o, part_ml, seqlens, B, k, seqlen_cap, sd::kAuRanges, reinterpret_cast<__nv_bfloat16*>(out), lse);
   stage_mark(kStageCombine, 1, st);
   return after_launch();
@@ -497,7 +498,7 @@ const char* sd_status_str(sd_status status) {
 
 int32_t sd_last_cuda_error(void) { return t_last_cuda_error; }
 int32_t sd_last_launch_count(void) { return t_launches; }
-int32_t sd_version(void) { return (0 << 16) | 2; }
+int32_t sd_version(void) { return (0 << 16) | 3; }
 
 }  // extern "C"
 

@@ -31,8 +31,9 @@ constexpr int kUmmaTile = 128;     // tokens per tile (MMA M)
 constexpr int kUmmaRowBytes = 128; // Di = 128 int8
 constexpr int kUmmaStages = 6;
 constexpr int kUmmaTilesPerStage = 2;  // consecutive tiles of one request share a stage
-constexpr int kUmmaAccs = 2;       // accumulators in tensor memory
-constexpr int kUmmaThreads = 192;
+constexpr int kUmmaAccs = 2;       // accumulators in tensor memory (tile i uses i % 2)
+constexpr int kUmmaEpiSets = 2;   // epilogue warp sets; set e reads the tiles i = e (mod 2)
+constexpr int kUmmaThreads = 64 + 128 * kUmmaEpiSets;
 
 template <int HI>
 struct IndexerUmmaLayout {
@@ -50,8 +51,6 @@ struct IndexerUmmaLayout {
 };
 
 // Walks a contiguous range of the global tile list (request-major).
-struct TileCursor;
-__device__ __forceinline__ bool stage_pairs(const TileCursor& c);
 
 struct TileCursor {
   int b, tile, tiles_b, L;
@@ -83,10 +82,14 @@ struct TileCursor {
   }
 };
 
-// A stage takes the cursor's tile and, when the range continues within the
-// same request, the next one (whose tile is then a full 128 tokens before it).
-__device__ __forceinline__ bool stage_pairs(const TileCursor& c) {
-  return kUmmaTilesPerStage == 2 && c.remaining > 1 && c.tile + 1 < c.tiles_b;
+// A stage takes the cursor's tile and the following ones of the same
+// request within the range, up to kUmmaTilesPerStage and to 32 pages (one
+// block-table window); every tile but the stage's last is then a full 128
+// tokens.
+__device__ __forceinline__ int stage_tiles(const TileCursor& c, int pages_per_tile) {
+  const long long left = c.remaining < (long long)(c.tiles_b - c.tile) ? c.remaining : (long long)(c.tiles_b - c.tile);
+  const int cap = min(kUmmaTilesPerStage, 32 / pages_per_tile);
+  return left < cap ? static_cast<int>(left) : cap;
 }
 
 __device__ __forceinline__ long long total_tiles(const int32_t* seqlens, int B, int cap) {
@@ -123,6 +126,7 @@ __global__ void __launch_bounds__(kUmmaThreads, 1) indexer_umma_kernel(
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int cap = min(max_seqlen, max_pages * page_size);
+  const int pshift = __ffs(page_size) - 1;  // page sizes on this path are powers of two
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kUmmaStages; ++i) {
@@ -172,7 +176,6 @@ __global__ void __launch_bounds__(kUmmaThreads, 1) indexer_umma_kernel(
     int stage = 0;
     uint32_t phase = 0;
     int nq = 0, cur_b = -1;
-    const int pshift = __ffs(page_size) - 1;  // page sizes on this path are powers of two
     const uint32_t page_bytes = static_cast<uint32_t>(page_size) * kUmmaRowBytes;
     const int oob_row = num_pages * page_size;
     int win_b = -1, win_p0 = 0, win_val = -1;
@@ -197,8 +200,8 @@ __global__ void __launch_bounds__(kUmmaThreads, 1) indexer_umma_kernel(
       }
       const int t0 = c.tile * kUmmaTile;
       const int p_first = t0 >> pshift;
-      const bool two = stage_pairs(c);
-      const int npages = (min(kUmmaTile * (two ? 2 : 1), c.L - t0) + page_size - 1) >> pshift;
+      const int nt = stage_tiles(c, kUmmaTile >> pshift);
+      const int npages = (min(kUmmaTile * nt, c.L - t0) + page_size - 1) >> pshift;
       if (c.b != win_b || p_first + npages > win_p0 + 32) {
         if (c.b == win_b && p_first == nxt_p0) {
           win_val = nxt_val;  // loaded one window ago: no round trip on this path
@@ -227,8 +230,7 @@ __global__ void __launch_bounds__(kUmmaThreads, 1) indexer_umma_kernel(
         sm100::tma_load_2d(kstage + stage * Lay::kStageBytes + off * page_bytes, &tm_keys, &full[stage], 0, row);
       }
       if (++stage == kUmmaStages) { stage = 0; phase ^= 1; }
-      c.next(seqlens, B, cap);
-      if (two) c.next(seqlens, B, cap);
+      for (int j = 0; j < nt; ++j) c.next(seqlens, B, cap);
     }
   } else if (warp == 1) {
     // ---------------- MMA issuer ----------------
@@ -246,7 +248,7 @@ __global__ void __launch_bounds__(kUmmaThreads, 1) indexer_umma_kernel(
           ++nq;
         }
         const int slot = (nq - 1) & 1;
-        const int ntiles = stage_pairs(c) ? 2 : 1;
+        const int ntiles = stage_tiles(c, kUmmaTile >> pshift);
         if (!sm100::mbar_wait(&full[stage], phase)) { *abort_flag = 1; break; }
         const uint32_t b0 = smem_u32(qbuf + slot * Lay::kQBytes);
         bool ok = true;
@@ -265,27 +267,29 @@ __global__ void __launch_bounds__(kUmmaThreads, 1) indexer_umma_kernel(
         if (!ok) { *abort_flag = 1; break; }
         sm100::mma_commit(&empty[stage]);
         const int this_b = c.b;
-        c.next(seqlens, B, cap);
-        if (ntiles == 2) c.next(seqlens, B, cap);
+        for (int j = 0; j < ntiles; ++j) c.next(seqlens, B, cap);
         if (!c.valid() || c.b != this_b) sm100::mma_commit(&qempty[slot]);
         if (++stage == kUmmaStages) { stage = 0; phase ^= 1; }
       }
     }
   } else {
     // ---------------- epilogue: ReLU, weighted head sum, store ----------------
-    // The accumulator is released as soon as its row is in registers; the
-    // block-table entry that validates this thread's token is loaded one tile
-    // ahead, so neither the tensor-memory round trip nor that load sits
-    // between two accumulators.
+    // Two sets of four warps take alternate tiles (set e: tiles i = e mod 2,
+    // accumulator e), so each set has two tile periods per tile. A warp reads
+    // its TMEM quadrant (warp % 4); the accumulator is released as soon as
+    // its row is in registers; the block-table entry that validates this
+    // thread's token is loaded one tile of the set ahead.
+    static_assert(kUmmaAccs == kUmmaEpiSets, "one accumulator per epilogue set");
+    const int set = (warp - 2) >> 2;
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
+    const int acc = set;
+    uint32_t accphase = 0;
     TileCursor c;
     c.init(seqlens, B, cap, first, count);
-    int acc = 0;
-    uint32_t accphase = 0;
+    for (int i = 0; i < set; ++i) c.next(seqlens, B, cap);
     int cur_b = -1;
     int32_t wreg[HI];
-    const int pshift = __ffs(page_size) - 1;  // page sizes on this path are powers of two
     auto page_of = [&](const TileCursor& cc) -> int {
       const int t = cc.tile * kUmmaTile + row;
       return (cc.valid() && t < cc.L) ? block_table[(size_t)cc.b * max_pages + (t >> pshift)] : 0;
@@ -300,7 +304,7 @@ __global__ void __launch_bounds__(kUmmaThreads, 1) indexer_umma_kernel(
       const int t = c.tile * kUmmaTile + row;
       const int phys = phys_next;
       TileCursor cn = c;
-      cn.next(seqlens, B, cap);
+      for (int i = 0; i < kUmmaEpiSets; ++i) cn.next(seqlens, B, cap);
       phys_next = page_of(cn);
       const bool ok = sm100::mbar_wait(&accfull[acc], accphase);
       __syncwarp();  // tcgen05.ld is warp-collective: reconverge after the polling loop
@@ -328,7 +332,7 @@ __global__ void __launch_bounds__(kUmmaThreads, 1) indexer_umma_kernel(
         }
         scores[(size_t)c.b * max_seqlen + t] = s;
       }
-      if (++acc == kUmmaAccs) { acc = 0; accphase ^= 1; }
+      accphase ^= 1;
       c = cn;
     }
   }

@@ -41,8 +41,8 @@ L2_FLUSH_BYTES = 256 << 20
 # Valid only for the library version they were taken on; any other version
 # reports traffic as null.
 NCU_TRAFFIC = {
-    ("b32_l65536_mla", "indexer"): (0x00000002, 269.063936e6 + 9.028864e6),
-    ("b32_l65536_mla", "attn"): (0x00000002, 104.638464e6 + 4.646656e6),
+    ("b32_l65536_mla", "indexer"): (0x00000004, 269.090560e6 + 8.853760e6),
+    ("b32_l65536_mla", "attn"): (0x00000004, 81.054208e6 + 4.387584e6),
 }
 
 

@@ -498,7 +498,7 @@ const char* sd_status_str(sd_status status) {
 
 int32_t sd_last_cuda_error(void) { return t_last_cuda_error; }
 int32_t sd_last_launch_count(void) { return t_launches; }
-int32_t sd_version(void) { return (0 << 16) | 3; }
+int32_t sd_version(void) { return (0 << 16) | 4; }
 
 }  // extern "C"
 

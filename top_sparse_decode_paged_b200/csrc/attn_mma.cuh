@@ -55,6 +55,9 @@ __global__ void __launch_bounds__(AttnMmaCfg<DK, DV, MT>::THREADS) attn_split_mm
     int page_size, int max_pages, int G, int H, int k, int seqlen_cap, float scale_log2,
     int n_head_blocks, int n_splits, int slots_per_split, float* __restrict__ part_o,
     float2* __restrict__ part_ml) {
+  pdl_wait();  // inputs come from earlier work in the stream
+  pdl_trigger();
+
   using C = AttnMmaCfg<DK, DV, MT>;
   constexpr int HB = C::HB, KS = C::KS, VS = C::VS, PS = C::PS;
   const bool separate_v = v_pages != nullptr;
@@ -297,6 +300,9 @@ __global__ void __launch_bounds__(128) attn_combine_kernel(const float* __restri
                                                            const float2* __restrict__ part_ml,
                                                            int n_splits, __nv_bfloat16* __restrict__ out,
                                                            float* __restrict__ lse) {
+  pdl_wait();  // inputs come from earlier work in the stream
+  pdl_trigger();
+
   const int bh = blockIdx.x;
   const float2* ml = part_ml + (size_t)bh * n_splits;
   float M = -INFINITY;

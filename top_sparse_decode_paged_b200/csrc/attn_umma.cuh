@@ -158,6 +158,9 @@ __global__ void __launch_bounds__(256) attn_rows_kernel(const int32_t* __restric
                                                         const int32_t* __restrict__ seqlens, int k, int seqlen_cap,
                                                         int page_size, int max_pages, int num_pages,
                                                         int32_t* __restrict__ rows) {
+  pdl_wait();  // inputs come from earlier work in the stream
+  pdl_trigger();
+
   const int b = blockIdx.y;
   const int s = blockIdx.x * 256 + threadIdx.x;
   const int kpad = attn_kpad(k);
@@ -230,6 +233,9 @@ __global__ void __launch_bounds__(kAuThreads, 1) attn_mla_umma_kernel(
   sm100::tc_fence_before();
   __syncthreads();
   sm100::tc_fence_after();
+  // the set-up above reads no input: the previous kernel may still be running
+  pdl_wait();
+  pdl_trigger();
   const uint32_t tmem = *tmem_slot;
   const uint32_t tm_o = tmem;          // cols [0,256): O^T, block j at 64j
   const uint32_t tm_s = tmem + 256;    // S, two buffers of kAuTile columns
@@ -573,6 +579,9 @@ constexpr int kAuMaxSeg = kMaxTopK / kAuTile;
 __global__ void __launch_bounds__(128) attn_mla_umma_combine_kernel(
     const float* __restrict__ part_o, const float2* __restrict__ part_ml, const int32_t* __restrict__ seqlens,
     int B, int k, int seqlen_cap, int n_ranges, __nv_bfloat16* __restrict__ out, float* __restrict__ lse) {
+  pdl_wait();  // inputs come from earlier work in the stream
+  pdl_trigger();
+
   const int b = blockIdx.x / kAuHeads;
   const int h = blockIdx.x % kAuHeads;
   __shared__ int seg_r[kAuMaxSeg];

@@ -27,6 +27,9 @@ __global__ void __launch_bounds__(kIdxThreads) indexer_dp4a_kernel(
     const int32_t* __restrict__ block_table, const int32_t* __restrict__ seqlens,
     int32_t* __restrict__ scores, int num_pages, int page_size, int max_pages, int G, int Hi,
     int max_seqlen) {
+  pdl_wait();  // inputs come from earlier work in the stream
+  pdl_trigger();
+
   constexpr int W4 = DI / 4;      // int32 words per key row
   extern __shared__ int32_t smem_i32[];
   const int b = blockIdx.y;

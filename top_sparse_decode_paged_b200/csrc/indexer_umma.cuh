@@ -155,6 +155,9 @@ __global__ void __launch_bounds__(kUmmaThreads, 1) indexer_umma_kernel(
   sm100::tc_fence_before();
   __syncthreads();
   sm100::tc_fence_after();
+  // the set-up above reads no input: the previous kernel may still be running
+  pdl_wait();
+  pdl_trigger();
   const uint32_t tmem_base = *tmem_slot;
 
   const long long total = total_tiles(seqlens, B, cap);

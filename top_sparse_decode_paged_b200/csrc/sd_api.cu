@@ -53,6 +53,27 @@ sd_status after_launch() {
   return cuda_check(cudaGetLastError());
 }
 
+// Launches a kernel with programmatic dependent launch allowed, so that its
+// launch and set-up overlap the tail of the previous kernel in the stream
+// (every kernel of this library waits in pdl_wait() before reading earlier
+// results). Off while stage events are armed: an event between two kernels
+// must see the first one complete.
+template <typename... KArgs, typename... Args>
+sd_status launch_k(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = t_stage_count == 0 ? 1 : 0;
+  ++t_launches;
+  return cuda_check(cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...));
+}
+
 struct AttnPlan {
   int mt, hb, n_hb, n_splits, slots_per_split;
 };
@@ -133,11 +154,11 @@ sd_status launch_indexer_t(const int8_t* qi, const int32_t* w, const int8_t* ki,
   const size_t smem = sd::indexer_dp4a_smem(pd.kv_heads, Hi, DI);
   dim3 grid(sd::ceil_div(max_seqlen, sd::kIdxTokensPerCta), B);
   stage_mark(kStageIndexer, 0, st);
-  sd::indexer_dp4a_kernel<DI><<<grid, sd::kIdxThreads, smem, st>>>(
-      qi, w, ki, bt, seqlens, scores, pd.num_pages, pd.page_size, pd.max_pages_per_req,
-      pd.kv_heads, Hi, max_seqlen);
+  const sd_status s = launch_k(sd::indexer_dp4a_kernel<DI>, grid, dim3(sd::kIdxThreads), smem, st, qi, w, ki, bt,
+                               seqlens, scores, pd.num_pages, pd.page_size, pd.max_pages_per_req, pd.kv_heads, Hi,
+                               max_seqlen);
   stage_mark(kStageIndexer, 1, st);
-  return after_launch();
+  return s;
 }
 
 // cuTensorMapEncodeTiled through the runtime's driver entry point (no link
@@ -217,12 +238,11 @@ sd_status launch_indexer_umma(const int8_t* qi, const int32_t* w, const int8_t* 
                                                 static_cast<int>(Lay::kSmemAlloc)));
   if (s != SD_OK) return s;
   stage_mark(kStageIndexer, 0, st);
-  kern<<<sm_count(), sd::kUmmaThreads, Lay::kSmemAlloc, st>>>(tm_keys, tm_q, w, bt, seqlens, scores, B,
-                                                              pd.num_pages, pd.page_size,
-                                                              pd.max_pages_per_req, max_seqlen);
+  s = launch_k(kern, dim3(sm_count()), dim3(sd::kUmmaThreads), Lay::kSmemAlloc, st, tm_keys, tm_q, w, bt, seqlens,
+               scores, B, pd.num_pages, pd.page_size, pd.max_pages_per_req, max_seqlen);
   stage_mark(kStageIndexer, 1, st);
   *launched = true;
-  return after_launch();
+  return s;
 }
 
 template <int PER>
@@ -237,13 +257,15 @@ sd_status launch_topk_cluster(const int32_t* scores, const int32_t* seqlens, int
   cfg.blockDim = dim3(sd::kTkThreads, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = cs;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = t_stage_count == 0 ? 2 : 1;  // see launch_k
   return cuda_check(cudaLaunchKernelEx(&cfg, sd::topk_cluster_kernel<PER>, scores, seqlens, indices, G,
                                        std::max(max_seqlen, 1), cap, k, rm));
 }
@@ -264,10 +286,10 @@ sd_status launch_topk(const int32_t* scores, const int32_t* seqlens, int32_t* in
     ++t_launches;
     return s;
   }
-  sd::topk_radix_kernel<<<rows, sd::kTopkThreads, 0, st>>>(scores, seqlens, indices, G,
-                                                           std::max(max_seqlen, 1), cap, k, rm);
+  const sd_status s = launch_k(sd::topk_radix_kernel, dim3(rows), dim3(sd::kTopkThreads), 0, st, scores, seqlens,
+                               indices, G, std::max(max_seqlen, 1), cap, k, rm);
   stage_mark(kStageTopk, 1, st);
-  return after_launch();
+  return s;
 }
 
 sd_status launch_indexer_topk(const int8_t* qi, const int32_t* w, const int8_t* ki, const int32_t* bt,
@@ -307,18 +329,17 @@ sd_status launch_attn_t(const uint16_t* q, const uint16_t* kp, const uint16_t* v
   const float scale_log2 = scale * 1.4426950408889634f;
   dim3 grid(p.n_splits, p.n_hb, B * pd.kv_heads);
   stage_mark(kStageAttn, 0, st);
-  kern<<<grid, C::THREADS, smem, st>>>(
-      reinterpret_cast<const __nv_bfloat16*>(q), reinterpret_cast<const __nv_bfloat16*>(kp),
-      reinterpret_cast<const __nv_bfloat16*>(vp), bt, seqlens, indices, pd.num_pages, pd.page_size,
-      pd.max_pages_per_req, pd.kv_heads, H, k, seqlen_cap, scale_log2, p.n_hb, p.n_splits,
-      p.slots_per_split, part_o, part_ml);
+  s = launch_k(kern, grid, dim3(C::THREADS), smem, st, reinterpret_cast<const __nv_bfloat16*>(q),
+               reinterpret_cast<const __nv_bfloat16*>(kp), reinterpret_cast<const __nv_bfloat16*>(vp), bt, seqlens,
+               indices, pd.num_pages, pd.page_size, pd.max_pages_per_req, pd.kv_heads, H, k, seqlen_cap, scale_log2,
+               p.n_hb, p.n_splits, p.slots_per_split, part_o, part_ml);
   stage_mark(kStageAttn, 1, st);
-  if ((s = after_launch()) != SD_OK) return s;
+  if (s != SD_OK) return s;
   stage_mark(kStageCombine, 0, st);
-  sd::attn_combine_kernel<DV><<<B * H, 128, 0, st>>>(part_o, part_ml, p.n_splits,
-                                                      reinterpret_cast<__nv_bfloat16*>(out), lse);
+  s = launch_k(sd::attn_combine_kernel<DV>, dim3(B * H), dim3(128), 0, st, static_cast<const float*>(part_o),
+               static_cast<const float2*>(part_ml), p.n_splits, reinterpret_cast<__nv_bfloat16*>(out), lse);
   stage_mark(kStageCombine, 1, st);
-  return after_launch();
+  return s;
 }
 
 // `rows_ready`: the top-k already resolved the selections to pool rows in the
@@ -344,19 +365,21 @@ sd_status launch_attn_umma(const uint16_t* q, const uint16_t* kp, const int32_t*
   stage_mark(kStageAttn, 0, st);
   if (!rows_ready) {
     const dim3 grid((sd::attn_kpad(k) + 255) / 256, B);
-    sd::attn_rows_kernel<<<grid, 256, 0, st>>>(indices, bt, seqlens, k, seqlen_cap, pd.page_size,
-                                               pd.max_pages_per_req, pd.num_pages, rows);
-    if ((s = after_launch()) != SD_OK) return s;
+    if ((s = launch_k(sd::attn_rows_kernel, grid, dim3(256), 0, st, indices, bt, seqlens, k, seqlen_cap, pd.page_size,
+                      pd.max_pages_per_req, pd.num_pages, rows)) != SD_OK)
+      return s;
   }
-  sd::attn_mla_umma_kernel<<<2 * sd::kAuRanges, sd::kAuThreads, Lay::kSmemAlloc, st>>>(
-      tm_q, reinterpret_cast<const __nv_bfloat16*>(kp), seqlens, rows, B, k, seqlen_cap, scale_log2, part_o, part_ml);
+  s = launch_k(sd::attn_mla_umma_kernel, dim3(2 * sd::kAuRanges), dim3(sd::kAuThreads), Lay::kSmemAlloc, st, tm_q,
+               reinterpret_cast<const __nv_bfloat16*>(kp), seqlens, static_cast<const int32_t*>(rows), B, k,
+               seqlen_cap, scale_log2, part_o, part_ml);
   stage_mark(kStageAttn, 1, st);
-  if ((s = after_launch()) != SD_OK) return s;
+  if (s != SD_OK) return s;
   stage_mark(kStageCombine, 0, st);
-  sd::attn_mla_umma_combine_kernel<<<B * sd::kAuHeads, 128, 0, st>>>(
-      part_o, part_ml, seqlens, B, k, seqlen_cap, sd::kAuRanges, reinterpret_cast<__nv_bfloat16*>(out), lse);
+  s = launch_k(sd::attn_mla_umma_combine_kernel, dim3(B * sd::kAuHeads), dim3(128), 0, st,
+               static_cast<const float*>(part_o), static_cast<const float2*>(part_ml), seqlens, B, k, seqlen_cap,
+               sd::kAuRanges, reinterpret_cast<__nv_bfloat16*>(out), lse);
   stage_mark(kStageCombine, 1, st);
-  return after_launch();
+  return s;
 }
 
 sd_status launch_attn(const uint16_t* q, const uint16_t* kp, const uint16_t* vp, const int32_t* bt,

@@ -25,6 +25,14 @@ __device__ __forceinline__ int checked_seqlen(const int32_t* seqlens, int b, int
   return L;
 }
 
+// Programmatic dependent launch. pdl_wait() blocks until the grids this one
+// depends on in its stream have completed and their writes are visible; call
+// it before reading anything earlier work produced. pdl_trigger() lets the
+// next grid in the stream start launching (it still waits in pdl_wait()).
+// Both are no-ops for a grid launched without the programmatic attribute.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" :::); }
+
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }

@@ -101,6 +101,9 @@ template <int PER>
 __global__ void __launch_bounds__(kTkThreads, 2) topk_cluster_kernel(
     const int32_t* __restrict__ scores, const int32_t* __restrict__ seqlens, int32_t* __restrict__ indices,
     int G, int max_seqlen, int seqlen_cap, int k, RowMap rm) {
+  pdl_wait();  // inputs come from earlier work in the stream
+  pdl_trigger();
+
   constexpr int kTkPerThread = PER;
   constexpr int kTkChunkStride = PER + 1;
   extern __shared__ __align__(16) uint8_t tk_smem_raw[];

@@ -53,6 +53,9 @@ __device__ __forceinline__ int block_excl_scan_flag(bool flag, uint32_t* warp_su
 __global__ void __launch_bounds__(kTopkThreads) topk_radix_kernel(
     const int32_t* __restrict__ scores, const int32_t* __restrict__ seqlens, int32_t* __restrict__ indices,
     int G, int max_seqlen, int seqlen_cap, int k, RowMap rm) {
+  pdl_wait();  // inputs come from earlier work in the stream
+  pdl_trigger();
+
   __shared__ uint32_t hist[256];
   __shared__ uint32_t scan_scratch[kTopkWarps + 1];
   __shared__ int sel_digit, sel_remaining;

@@ -316,7 +316,8 @@ def bench_ours(args, rank, world, local):
     e_steps = max(3, min(args.steps, 50))
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     torch.cuda.synchronize()
-    e_ms = 0.0
+    # (a) one step at a time: copies in, step, copies out, then wait
+    e_ms_serial = 0.0
     for i in range(e_steps):
         flush_l2()
         e0.record(stream)
@@ -330,8 +331,55 @@ def bench_ours(args, rank, world, local):
         h_out.copy_(out.view(torch.int16), non_blocking=True)
         e1.record(stream)
         e1.synchronize()
-        e_ms += e0.elapsed_time(e1)
-    e_ms = max_over_ranks(e_ms / e_steps, world)
+        e_ms_serial += e0.elapsed_time(e1)
+    e_ms_serial = max_over_ranks(e_ms_serial / e_steps, world)
+    # (b) as a serving loop runs it: step i's inputs go up while step i-1
+    # computes and step i-2's results come down (two buffer sets, three
+    # streams); every step still pays both copies. No flush: the inputs
+    # (indexer keys and latent cache) are larger than L2.
+    bufs = []
+    for _ in range(2):
+        bufs.append(dict(qi=torch.empty_like(qi), w=torch.empty_like(w), q=torch.empty_like(q), bt=torch.empty_like(bt),
+                         sl=torch.empty_like(sl), idx=torch.empty_like(idx), out=torch.empty_like(out),
+                         h_idx=torch.empty_like(h_idx).pin_memory(), h_out=torch.empty_like(h_out).pin_memory(),
+                         up=torch.cuda.Event(), done=torch.cuda.Event(), down=torch.cuda.Event()))
+    s_up, s_comp, s_down = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+
+    def pipelined(n):
+        for i in range(n):
+            bb = bufs[i % 2]
+            with torch.cuda.stream(s_up):
+                if i >= 2:
+                    s_up.wait_event(bb["done"])  # step i-2 has consumed this buffer set
+                bb["qi"].copy_(h_qi, non_blocking=True)
+                bb["w"].copy_(h_w, non_blocking=True)
+                bb["q"].view(torch.int16).copy_(h_q, non_blocking=True)
+                bb["bt"].copy_(h_bt, non_blocking=True)
+                bb["sl"].copy_(h_sl, non_blocking=True)
+                bb["up"].record(s_up)
+            with torch.cuda.stream(s_comp):
+                s_comp.wait_event(bb["up"])
+                if i >= 2:
+                    s_comp.wait_event(bb["down"])  # step i-2's results are out of this buffer set
+                sd.sd_decode_step(bb["qi"], bb["w"], ki, bb["q"], kp, vp, bb["bt"], bb["sl"], s.k, Lmax, s.scale,
+                                  s.Dv, indices=bb["idx"], out=bb["out"], workspace=ws)
+                bb["done"].record(s_comp)
+            with torch.cuda.stream(s_down):
+                s_down.wait_event(bb["done"])
+                bb["h_idx"].copy_(bb["idx"], non_blocking=True)
+                bb["h_out"].copy_(bb["out"].view(torch.int16), non_blocking=True)
+                bb["down"].record(s_down)
+
+    pipelined(4)
+    torch.cuda.synchronize()
+    p0, p1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    p0.record(s_up)
+    pipelined(e_steps)
+    for st_ in (s_up, s_comp):
+        s_down.wait_stream(st_)
+    p1.record(s_down)
+    p1.synchronize()
+    e_ms = max_over_ranks(p0.elapsed_time(p1) / e_steps, world)
 
     alg = W.algorithmic_bytes(s, wl.seqlens)
     lens = wl.seqlens.astype(np.int64)
@@ -370,7 +418,9 @@ def bench_ours(args, rank, world, local):
         "roofline": rooflines[dominant],
         "rooflines": rooflines,
         "e2e": {"value": world * B / (e_ms * 1e-3), "unit": "queries/s",
-                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "mode": "pipelined: step i's inputs go up while step i-1 computes and step i-2's results come down",
+                "serial_value": world * B / (e_ms_serial * 1e-3)},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks.summary(),
         "library_version": lib_version,

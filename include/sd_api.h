@@ -127,6 +127,29 @@ sd_status sd_sparse_attn(const uint16_t* q, const uint16_t* k_pages, const uint1
                          int32_t Dk, int32_t Dv, int32_t k, float scale, uint16_t* out,
                          float* lse, void* workspace, size_t workspace_bytes, void* stream);
 
+/* Steps 3 + 4 for n_layers layers that share one selection: the
+ * shared-indexer decode of "Overlap DSA heuristic prev_topk write-back on the
+ * aux stream" (Description: layers without their own indexer reuse the top-k
+ * buffer) and of "Add DSA Vanilla sparse attention" (the persistent index
+ * buffer read by every layer).
+ *   q        bf16 [n_layers, B, H, Dk], layer-major
+ *   k_pages  HOST array of n_layers device pointers, each a latent / key pool
+ *            laid out as for sd_sparse_attn (all with the geometry `pd`)
+ *   v_pages  HOST array of n_layers value pools, or NULL (V inside K)
+ *   block_table, seqlens, indices: one set, shared by every layer
+ *   out      bf16 [n_layers, B, H, Dv]; lse fp32 [n_layers, B, H] or NULL
+ * With MLA rows (G = 1, H = 128, Dk = 576, Dv = 512, V inside K), up to 16
+ * layers run in one launch, so the selections are resolved to pool rows once
+ * per group of layers and small batches fill the GPU; other shapes run layer
+ * after layer. Workspace: sd_attn_layers_workspace_size(). Errors as for
+ * sd_sparse_attn; SD_ERR_INVALID_ARG also for n_layers < 1 or a NULL pool. */
+size_t sd_attn_layers_workspace_size(int32_t n_layers, int32_t B, int32_t G, int32_t k, int32_t H, int32_t Dv);
+sd_status sd_sparse_attn_layers(const uint16_t* q, const uint16_t* const* k_pages, const uint16_t* const* v_pages,
+                                int32_t n_layers, const int32_t* block_table, const int32_t* seqlens,
+                                const int32_t* indices, sd_paged_desc pd, int32_t B, int32_t H, int32_t Dk,
+                                int32_t Dv, int32_t k, float scale, uint16_t* out, float* lse, void* workspace,
+                                size_t workspace_bytes, void* stream);
+
 /* Steps 1 + 2 + 3 in one call on one stream (arguments as above). */
 sd_status sd_decode_step(const int8_t* qi, const int32_t* w, const int8_t* ki_pages,
                          const uint16_t* q, const uint16_t* k_pages, const uint16_t* v_pages,

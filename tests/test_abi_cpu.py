@@ -80,3 +80,23 @@ def test_attention_argument_errors(lib):
     # non-finite scale
     assert f(256, 256, None, 256, 256, 256, desc, 1, 4, 64, 64, 8, ctypes.c_float(float("nan")), 256,
              None, None, 0, None) == 1
+
+
+def test_layers_argument_errors(lib):
+    desc = api.PagedDesc(4, 16, 4, 1)
+    f = lib.sd_sparse_attn_layers
+    pools = (ctypes.c_void_p * 2)(256, 256)
+    holes = (ctypes.c_void_p * 2)(256, None)
+    args = lambda kp, n, Dk=64, Dv=64: (256, ctypes.cast(kp, ctypes.c_void_p), None, n, 256, 256, 256, desc,  # noqa: E731
+                                         1, 4, Dk, Dv, 8, ctypes.c_float(0.1), 256, None, None, 0, None)
+    assert f(*args(pools, 0)) == 1          # no layers
+    assert f(*args(holes, 2)) == 1          # a NULL pool
+    assert f(*args(pools, 2, 96, 96)) == 2  # unsupported head width
+    assert f(*args(pools, 2)) == 3          # no workspace
+    assert lib.sd_attn_layers_workspace_size(0, 1, 1, 8, 4, 64) == 0
+    one = lib.sd_attn_layers_workspace_size(1, 32, 1, 2048, 128, 512)
+    assert lib.sd_attn_layers_workspace_size(4, 32, 1, 2048, 128, 512) > one > 0
+    # layers beyond the 16 of one launch reuse the workspace of 16
+    assert lib.sd_attn_layers_workspace_size(40, 32, 1, 2048, 128, 512) == \
+        lib.sd_attn_layers_workspace_size(16, 32, 1, 2048, 128, 512)
+    assert lib.sd_last_launch_count() == 0

@@ -22,7 +22,7 @@ SD_DEVERR_PAGE = 0x2
 SD_DEVERR_INDEX = 0x4
 
 EXPORTED = ("sd_workspace_size", "sd_indexer_topk", "sd_indexer_topk_noalloc", "sd_sparse_attn",
-            "sd_decode_step",
+            "sd_attn_layers_workspace_size", "sd_sparse_attn_layers", "sd_decode_step",
             "sd_set_stage_events", "sd_get_device_errors", "sd_status_str", "sd_last_cuda_error",
             "sd_last_launch_count", "sd_version")
 
@@ -62,6 +62,11 @@ def load_library(path: str = LIB_PATH):
     lib.sd_sparse_attn.restype = i32
     lib.sd_sparse_attn.argtypes = [p, p, p, p, p, p, PagedDesc, i32, i32, i32, i32, i32,
                                    ctypes.c_float, p, p, p, sz, p]
+    lib.sd_attn_layers_workspace_size.restype = sz
+    lib.sd_attn_layers_workspace_size.argtypes = [i32] * 6
+    lib.sd_sparse_attn_layers.restype = i32
+    lib.sd_sparse_attn_layers.argtypes = [p, p, p, i32, p, p, p, PagedDesc, i32, i32, i32, i32, i32,
+                                          ctypes.c_float, p, p, p, sz, p]
     lib.sd_decode_step.restype = i32
     lib.sd_decode_step.argtypes = [p, p, p, p, p, p, p, p, PagedDesc, i32, i32, i32, i32, i32, i32,
                                    i32, i32, ctypes.c_float, p, p, p, p, p, sz, p]
@@ -178,6 +183,35 @@ def sd_sparse_attn(q, k_pages, v_pages, block_table, seqlens, indices, scale: fl
     _check(lib.sd_sparse_attn(_ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(block_table), _ptr(seqlens),
                               _ptr(indices), _desc(k_pages, block_table), B, H, Dk, Dv, k, float(scale),
                               _ptr(out), _ptr(lse), _ptr(workspace), workspace.numel(), _stream(stream)))
+    return out
+
+
+def sd_sparse_attn_layers(q, k_pages, v_pages, block_table, seqlens, indices, scale: float, Dv: int,
+                          out=None, lse=None, workspace=None, stream=None):
+    """Attention + combine for several layers sharing one selection.
+
+    ``q`` is [n_layers, B, H, Dk]; ``k_pages`` (and ``v_pages``, or None) are
+    sequences of one pool per layer. Returns ``out`` [n_layers, B, H, Dv] bf16.
+    """
+    lib = load_library()
+    q = _bits(q)
+    kps = [_bits(t) for t in k_pages]
+    vps = None if v_pages is None else [_bits(t) for t in v_pages]
+    L, B, H, Dk = q.shape
+    G = kps[0].shape[2]
+    k = indices.shape[-1]
+    if out is None:
+        out = torch.empty((L, B, H, Dv), dtype=torch.bfloat16, device=q.device)
+    if workspace is None:
+        nbytes = int(lib.sd_attn_layers_workspace_size(L, B, G, k, H, Dv))
+        workspace = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=q.device)
+    karr = (ctypes.c_void_p * L)(*[t.data_ptr() for t in kps])
+    varr = None if vps is None else (ctypes.c_void_p * L)(*[t.data_ptr() for t in vps])
+    _check(lib.sd_sparse_attn_layers(_ptr(q), ctypes.cast(karr, ctypes.c_void_p),
+                                     None if varr is None else ctypes.cast(varr, ctypes.c_void_p), L,
+                                     _ptr(block_table), _ptr(seqlens), _ptr(indices), _desc(kps[0], block_table),
+                                     B, H, Dk, Dv, k, float(scale), _ptr(out), _ptr(lse), _ptr(workspace),
+                                     workspace.numel(), _stream(stream)))
     return out
 
 

@@ -94,15 +94,20 @@ struct AttnUmmaLayout {
 static_assert(AttnUmmaLayout::kSmemAlloc <= 232448, "attention shared memory");
 
 // Walks a contiguous range of the attention tile list (request-major).
+// Requests are "virtual": vb = layer * breq + b when several layers share one
+// selection (the row ids, seqlens and block table of request b), vb = b
+// otherwise.
 struct AttnCursor {
   int b, tile, tiles_b, L;
   long long remaining;
+  int breq;
   __device__ static int tiles_of(int L, int k) { return ceil_div(min(k, L), kAuTile); }
-  __device__ void init(const int32_t* seqlens, int B, int cap, int k, long long first, long long count) {
+  __device__ void init(const int32_t* seqlens, int B, int cap, int k, long long first, long long count, int nreq) {
     remaining = count;
+    breq = nreq;
     long long skip = first;
     for (b = 0; b < B; ++b) {
-      L = checked_seqlen(seqlens, b, cap);
+      L = checked_seqlen(seqlens, b % breq, cap);
       tiles_b = tiles_of(L, k);
       if (skip < tiles_b) break;
       skip -= tiles_b;
@@ -116,16 +121,22 @@ struct AttnCursor {
     tile = 0;
     do {
       ++b;
-      L = checked_seqlen(seqlens, b, cap);
+      L = checked_seqlen(seqlens, b % breq, cap);
       tiles_b = tiles_of(L, k);
     } while (tiles_b == 0 && b < B - 1);
   }
 };
 
-__device__ __forceinline__ long long attn_total_tiles(const int32_t* seqlens, int B, int cap, int k) {
+// Base pointers of the latent caches of the layers one launch serves.
+constexpr int kAuMaxLayers = 16;
+struct AttnLayerKV {
+  const __nv_bfloat16* p[kAuMaxLayers];
+};
+
+__device__ __forceinline__ long long attn_total_tiles(const int32_t* seqlens, int B, int cap, int k, int breq) {
   long long n = 0;
   for (int b = 0; b < B; ++b) {
-    int L = seqlens[b];
+    int L = seqlens[b % breq];
     L = L < 0 ? 0 : (L > cap ? cap : L);
     n += ceil_div(min(k, L), kAuTile);
   }
@@ -170,9 +181,11 @@ __global__ void __launch_bounds__(256) attn_rows_kernel(const int32_t* __restric
       attn_row_of(indices, block_table, b, s, min(k, L), k, L, page_size, max_pages, num_pages));
 }
 
+// B counts virtual requests (layers x breq); q, out and the partials are
+// indexed by them, seqlens and the row ids by the real request.
 __global__ void __launch_bounds__(kAuThreads, 1) attn_mla_umma_kernel(
-    const __grid_constant__ CUtensorMap tm_q, const __nv_bfloat16* __restrict__ kv,
-    const int32_t* __restrict__ seqlens, const int32_t* __restrict__ rows, int B, int k, int seqlen_cap,
+    const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ AttnLayerKV kvl,
+    const int32_t* __restrict__ seqlens, const int32_t* __restrict__ rows, int B, int breq, int k, int seqlen_cap,
     float scale_log2, float* __restrict__ part_o, float2* __restrict__ part_ml) {
   using Lay = AttnUmmaLayout;
   extern __shared__ uint8_t smem_dyn[];
@@ -240,7 +253,7 @@ __global__ void __launch_bounds__(kAuThreads, 1) attn_mla_umma_kernel(
   const uint32_t tm_o = tmem;          // cols [0,256): O^T, block j at 64j
   const uint32_t tm_s = tmem + 256;    // S, two buffers of kAuTile columns
 
-  const long long total = attn_total_tiles(seqlens, B, seqlen_cap, k);
+  const long long total = attn_total_tiles(seqlens, B, seqlen_cap, k, breq);
   const long long first = total * range / n_ranges;
   const long long count = total * (range + 1) / n_ranges - first;
 
@@ -252,7 +265,7 @@ __global__ void __launch_bounds__(kAuThreads, 1) attn_mla_umma_kernel(
     const int pt = threadIdx.x;  // 0..127
     const int seg = lane & 7;
     AttnCursor c;
-    c.init(seqlens, B, seqlen_cap, k, first, count);
+    c.init(seqlens, B, seqlen_cap, k, first, count, breq);
     long long n = 0;
     int q_issued = 0, prev_b = -1;
     bool ok = true;
@@ -286,6 +299,7 @@ __global__ void __launch_bounds__(kAuThreads, 1) attn_mla_umma_kernel(
       ok = ok && sm100::mbar_wait(&tile_empty[slot], static_cast<uint32_t>((n / kAuBufs) & 1) ^ 1) && !*abort_flag;
       if (!ok) break;
       uint8_t* tb = ring + slot * kAuTileBytes;
+      const __nv_bfloat16* kv = kvl.p[c.b / breq];
 #pragma unroll
       for (int i = 0; i < kAuTile / 16; ++i) {
         const int t = (pt >> 3) + 16 * i;
@@ -317,7 +331,7 @@ __global__ void __launch_bounds__(kAuThreads, 1) attn_mla_umma_kernel(
     const int vrow = quarter * 32 + lane;       // value row of O^T within a block
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
     AttnCursor c;
-    c.init(seqlens, B, seqlen_cap, k, first, count);
+    c.init(seqlens, B, seqlen_cap, k, first, count, breq);
     long long j = 0;
     int prev_b = -1;
     float m_ref[2] = {-INFINITY, -INFINITY}, l_sum[2] = {0.f, 0.f};
@@ -467,8 +481,8 @@ __global__ void __launch_bounds__(kAuThreads, 1) attn_mla_umma_kernel(
       // next tile's rows, so a tile buffer is released as soon as its own
       // P V is done.
       AttnCursor cs, cp;
-      cs.init(seqlens, B, seqlen_cap, k, first, count);
-      cp.init(seqlens, B, seqlen_cap, k, first, count);
+      cs.init(seqlens, B, seqlen_cap, k, first, count, breq);
+      cp.init(seqlens, B, seqlen_cap, k, first, count, breq);
       long long is = 0, ip = 0;
       int q_seen = 0, prev_bs = -1, prev_bp = -1;
       uint32_t idle = 0;
@@ -542,14 +556,14 @@ __global__ void __launch_bounds__(kAuThreads, 1) attn_mla_umma_kernel(
     // Streams each tile's resolved pool rows into a small ring, kAuRidSlots
     // tiles ahead of the copies and the softmax.
     AttnCursor c;
-    c.init(seqlens, B, seqlen_cap, k, first, count);
+    c.init(seqlens, B, seqlen_cap, k, first, count, breq);
     long long n = 0;
     bool ok = true;
     while (c.valid() && ok) {
       const int rs = static_cast<int>(n % kAuRidSlots);
       ok = sm100::mbar_wait(&rid_empty[rs], static_cast<uint32_t>((n / kAuRidSlots) & 1) ^ 1) && !*abort_flag;
       if (!ok) break;
-      const int32_t* src = rows + (size_t)c.b * kpad + c.tile * kAuTile;
+      const int32_t* src = rows + (size_t)(c.b % breq) * kpad + c.tile * kAuTile;
 #pragma unroll
       for (int w = 0; w < kAuTileWords; ++w) cp_async_4(&rid[rs * kAuTile + 32 * w + lane], src + 32 * w + lane);
       sm100::cp_async_arrive_noinc(&rid_full[rs]);
@@ -570,28 +584,29 @@ __global__ void __launch_bounds__(kAuThreads, 1) attn_mla_umma_kernel(
 }
 
 // Merges the per-range partials into the bf16 output. One block per (request,
-// head), 128 threads of 4 value columns each. Warp 0 lists the ranges that
-// cover the request: a request has at most ceil(k / kAuTile) tiles, and tile
-// i of the list lies in range ((i + 1) * n_ranges - 1) / total. Each thread
-// then issues the loads of all its partials together.
+// pair of heads), 128 threads per head of 4 value columns each. Warp 0 lists
+// the ranges that cover the request: a request has at most ceil(k / kAuTile)
+// tiles, and tile i of the list lies in range ((i + 1) * n_ranges - 1) /
+// total. Each thread then issues the loads of all its partials together.
 constexpr int kAuMaxSeg = kMaxTopK / kAuTile;
+constexpr int kAuCombineHeads = 2;
 
-__global__ void __launch_bounds__(128) attn_mla_umma_combine_kernel(
+__global__ void __launch_bounds__(128 * kAuCombineHeads) attn_mla_umma_combine_kernel(
     const float* __restrict__ part_o, const float2* __restrict__ part_ml, const int32_t* __restrict__ seqlens,
-    int B, int k, int seqlen_cap, int n_ranges, __nv_bfloat16* __restrict__ out, float* __restrict__ lse) {
+    int B, int breq, int k, int seqlen_cap, int n_ranges, __nv_bfloat16* __restrict__ out, float* __restrict__ lse) {
   pdl_wait();  // inputs come from earlier work in the stream
   pdl_trigger();
-
-  const int b = blockIdx.x / kAuHeads;
-  const int h = blockIdx.x % kAuHeads;
+  constexpr int HG = kAuHeads / kAuCombineHeads;
+  const int b = blockIdx.x / HG;
+  const int h = (blockIdx.x % HG) * kAuCombineHeads + (threadIdx.x >> 7);
   __shared__ int seg_r[kAuMaxSeg];
-  __shared__ float2 ml_s[kAuMaxSeg];
+  __shared__ float2 ml_s[kAuCombineHeads][kAuMaxSeg];
   __shared__ int nseg_s;
-  const int tid = threadIdx.x, lane = tid & 31;
-  if (tid < 32) {
+  const int tid = threadIdx.x & 127, lane = threadIdx.x & 31;
+  if (threadIdx.x < 32) {
     uint32_t before = 0, total = 0, mine = 0;
     for (int i = lane; i < B; i += 32) {
-      int L = seqlens[i];
+      int L = seqlens[i % breq];
       L = L < 0 ? 0 : (L > seqlen_cap ? seqlen_cap : L);
       const uint32_t n = static_cast<uint32_t>(ceil_div(min(k, L), kAuTile));
       before += i < b ? n : 0;
@@ -605,6 +620,7 @@ __global__ void __launch_bounds__(128) attn_mla_umma_combine_kernel(
       mine += __shfl_xor_sync(0xffffffffu, mine, o);
     }
     const uint32_t nr = static_cast<uint32_t>(n_ranges);
+    const int h0 = (blockIdx.x % HG) * kAuCombineHeads;
     uint32_t carry = 0xffffffffu;  // range of the previous tile
     int nseg = 0;
     for (uint32_t base = 0; base < mine; base += 32) {
@@ -619,7 +635,8 @@ __global__ void __launch_bounds__(128) attn_mla_umma_combine_kernel(
       const int at = nseg + __popc(bal & ((1u << lane) - 1u));
       if (head_of_seg) {
         seg_r[at] = static_cast<int>(r);
-        ml_s[at] = part_ml[((size_t)r + b) * kAuHeads + h];
+#pragma unroll
+        for (int hh = 0; hh < kAuCombineHeads; ++hh) ml_s[hh][at] = part_ml[((size_t)r + b) * kAuHeads + h0 + hh];
       }
       nseg += __popc(bal);
       carry = __shfl_sync(0xffffffffu, r, 31);
@@ -628,18 +645,19 @@ __global__ void __launch_bounds__(128) attn_mla_umma_combine_kernel(
   }
   __syncthreads();
   const int nseg = nseg_s;
+  const float2* ml = ml_s[threadIdx.x >> 7];
   const int d0 = 4 * tid;  // value columns d0..d0+3
   float M = -INFINITY;
-  for (int jj = 0; jj < nseg; ++jj) M = fmaxf(M, ml_s[jj].x);
+  for (int jj = 0; jj < nseg; ++jj) M = fmaxf(M, ml[jj].x);
   float denom = 0.f;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll 4
   for (int jj = 0; jj < nseg; ++jj) {
-    const float2 ml = ml_s[jj];
-    if (ml.x == -INFINITY) continue;
+    const float2 m_l = ml[jj];
+    if (m_l.x == -INFINITY) continue;
     const size_t slot = static_cast<size_t>(seg_r[jj]) + b;
-    const float wgt = exp2f(ml.x - M);
-    denom += wgt * ml.y;
+    const float wgt = exp2f(m_l.x - M);
+    denom += wgt * m_l.y;
     const float4 o = *reinterpret_cast<const float4*>(part_o + (slot * kAuHeads + h) * kAuDv + d0);
     acc.x += wgt * o.x;
     acc.y += wgt * o.y;

@@ -343,21 +343,33 @@ sd_status launch_attn_t(const uint16_t* q, const uint16_t* kp, const uint16_t* v
 }
 
 // `rows_ready`: the top-k already resolved the selections to pool rows in the
-// workspace's row array; otherwise a small kernel does it first.
-sd_status launch_attn_umma(const uint16_t* q, const uint16_t* kp, const int32_t* bt, const int32_t* seqlens,
-                           const int32_t* indices, const sd_paged_desc& pd, int B, int k, float scale,
-                           uint16_t* out, float* lse, void* ws, int seqlen_cap, bool rows_ready, cudaStream_t st) {
+// workspace's row array; otherwise a small kernel does it first. With
+// n_layers > 1, q / out / lse hold n_layers x B requests (layer-major) that
+// share the selection, seqlens and block table of the B real requests, and
+// kp_layers[l] is layer l's latent cache; requests are "virtual" (layer * B +
+// b) inside the kernels.
+sd_status launch_attn_umma(const uint16_t* q, const uint16_t* const* kp_layers, int n_layers, const int32_t* bt,
+                           const int32_t* seqlens, const int32_t* indices, const sd_paged_desc& pd, int B, int k,
+                           float scale, uint16_t* out, float* lse, void* ws, int seqlen_cap, bool rows_ready,
+                           cudaStream_t st) {
   using Lay = sd::AttnUmmaLayout;
-  const size_t slots = static_cast<size_t>(sd::kAuRanges) + B;
+  if (n_layers < 1 || n_layers > sd::kAuMaxLayers) return SD_ERR_UNSUPPORTED;
+  const int Bv = n_layers * B;
+  const size_t slots = static_cast<size_t>(sd::kAuRanges) + Bv;
   float* part_o = static_cast<float*>(ws);
   float2* part_ml = reinterpret_cast<float2*>(
       static_cast<char*>(ws) + align_up(slots * sd::kAuHeads * sd::kAuDv * sizeof(float)));
-  int32_t* rows = reinterpret_cast<int32_t*>(static_cast<char*>(ws) + sd::attn_umma_rows_offset(B));
+  int32_t* rows = reinterpret_cast<int32_t*>(static_cast<char*>(ws) + sd::attn_umma_rows_offset(Bv));
   CUtensorMap tm_q;
   const uint64_t pool_rows = (uint64_t)pd.num_pages * pd.page_size;
-  if (!encode_bf16_rows(&tm_q, q, sd::kAuDk, (uint64_t)B * sd::kAuHeads, sd::kAuDk * 2, 64, sd::kAuHalfHeads) ||
-      (reinterpret_cast<uintptr_t>(kp) & 15u) != 0 || pool_rows >= (1ull << 31))
+  if (!encode_bf16_rows(&tm_q, q, sd::kAuDk, (uint64_t)Bv * sd::kAuHeads, sd::kAuDk * 2, 64, sd::kAuHalfHeads) ||
+      pool_rows >= (1ull << 31))
     return SD_ERR_UNSUPPORTED;
+  sd::AttnLayerKV kvl{};
+  for (int l = 0; l < n_layers; ++l) {
+    if (kp_layers[l] == nullptr || (reinterpret_cast<uintptr_t>(kp_layers[l]) & 15u) != 0) return SD_ERR_UNSUPPORTED;
+    kvl.p[l] = reinterpret_cast<const __nv_bfloat16*>(kp_layers[l]);
+  }
   sd_status s = cuda_check(cudaFuncSetAttribute(sd::attn_mla_umma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                 static_cast<int>(Lay::kSmemAlloc)));
   if (s != SD_OK) return s;
@@ -370,14 +382,14 @@ sd_status launch_attn_umma(const uint16_t* q, const uint16_t* kp, const int32_t*
       return s;
   }
   s = launch_k(sd::attn_mla_umma_kernel, dim3(2 * sd::kAuRanges), dim3(sd::kAuThreads), Lay::kSmemAlloc, st, tm_q,
-               reinterpret_cast<const __nv_bfloat16*>(kp), seqlens, static_cast<const int32_t*>(rows), B, k,
-               seqlen_cap, scale_log2, part_o, part_ml);
+               kvl, seqlens, static_cast<const int32_t*>(rows), Bv, B, k, seqlen_cap, scale_log2, part_o, part_ml);
   stage_mark(kStageAttn, 1, st);
   if (s != SD_OK) return s;
   stage_mark(kStageCombine, 0, st);
-  s = launch_k(sd::attn_mla_umma_combine_kernel, dim3(B * sd::kAuHeads), dim3(128), 0, st,
-               static_cast<const float*>(part_o), static_cast<const float2*>(part_ml), seqlens, B, k, seqlen_cap,
-               sd::kAuRanges, reinterpret_cast<__nv_bfloat16*>(out), lse);
+  s = launch_k(sd::attn_mla_umma_combine_kernel, dim3(Bv * (sd::kAuHeads / sd::kAuCombineHeads)),
+               dim3(128 * sd::kAuCombineHeads), 0, st, static_cast<const float*>(part_o),
+               static_cast<const float2*>(part_ml), seqlens, Bv, B, k, seqlen_cap, sd::kAuRanges,
+               reinterpret_cast<__nv_bfloat16*>(out), lse);
   stage_mark(kStageCombine, 1, st);
   return s;
 }
@@ -389,7 +401,7 @@ sd_status launch_attn(const uint16_t* q, const uint16_t* kp, const uint16_t* vp,
   if (B == 0) return SD_OK;
   if (umma_attn_fits(pd.kv_heads, H, Dk, Dv, vp != nullptr)) {
     const sd_status su =
-        launch_attn_umma(q, kp, bt, seqlens, indices, pd, B, k, scale, out, lse, ws, seqlen_cap, rows_ready, st);
+        launch_attn_umma(q, &kp, 1, bt, seqlens, indices, pd, B, k, scale, out, lse, ws, seqlen_cap, rows_ready, st);
     if (su != SD_ERR_UNSUPPORTED) return su;  // else: pointers the TMA cannot map; take the mma.sync kernel
   }
   const AttnPlan p = attn_plan(B, pd.kv_heads, H, k);
@@ -447,6 +459,53 @@ sd_status sd_sparse_attn(const uint16_t* q, const uint16_t* k_pages, const uint1
   const int cap = pd.max_pages_per_req * pd.page_size;
   return launch_attn(q, k_pages, v_pages, block_table, seqlens, indices, pd, B, H, Dk, Dv, k, scale,
                      out, lse, workspace, cap, static_cast<cudaStream_t>(stream));
+}
+
+size_t sd_attn_layers_workspace_size(int32_t n_layers, int32_t B, int32_t G, int32_t k, int32_t H, int32_t Dv) {
+  if (n_layers < 1 || B < 0 || G <= 0 || k <= 0 || H <= 0 || Dv <= 0) return 0;
+  size_t bytes = attn_bytes(B, G, H, k, Dv);
+  if (G == 1 && H == sd::kAuHeads && Dv == sd::kAuDv)
+    bytes = std::max(bytes, align_up(sd::attn_umma_workspace(std::min(n_layers, (int32_t)sd::kAuMaxLayers) * B, k)));
+  return bytes;
+}
+
+sd_status sd_sparse_attn_layers(const uint16_t* q, const uint16_t* const* k_pages, const uint16_t* const* v_pages,
+                                int32_t n_layers, const int32_t* block_table, const int32_t* seqlens,
+                                const int32_t* indices, sd_paged_desc pd, int32_t B, int32_t H, int32_t Dk,
+                                int32_t Dv, int32_t k, float scale, uint16_t* out, float* lse, void* workspace,
+                                size_t workspace_bytes, void* stream) {
+  t_launches = 0;
+  if (n_layers < 1 || k_pages == nullptr) return SD_ERR_INVALID_ARG;
+  for (int l = 0; l < n_layers; ++l)
+    if (k_pages[l] == nullptr || (v_pages != nullptr && v_pages[l] == nullptr)) return SD_ERR_INVALID_ARG;
+  sd_status s = check_attn_args(q, k_pages[0], block_table, seqlens, indices, pd, B, H, Dk, Dv, k, scale, out,
+                                v_pages != nullptr);
+  if (s != SD_OK) return s;
+  if (!ws_ok(workspace, workspace_bytes, sd_attn_layers_workspace_size(n_layers, B, pd.kv_heads, k, H, Dv)))
+    return SD_ERR_WORKSPACE;
+  if (B == 0) return SD_OK;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int cap = pd.max_pages_per_req * pd.page_size;
+  const size_t q_layer = (size_t)B * H * Dk, o_layer = (size_t)B * H * Dv, l_layer = (size_t)B * H;
+  int l0 = 0;
+  if (v_pages == nullptr && umma_attn_fits(pd.kv_heads, H, Dk, Dv, false)) {
+    // layers share the selection: one launch per group of up to kAuMaxLayers
+    for (; l0 < n_layers; l0 += sd::kAuMaxLayers) {
+      const int nl = std::min(n_layers - l0, (int)sd::kAuMaxLayers);
+      s = launch_attn_umma(q + l0 * q_layer, k_pages + l0, nl, block_table, seqlens, indices, pd, B, k, scale,
+                           out + l0 * o_layer, lse ? lse + l0 * l_layer : nullptr, workspace, cap, false, st);
+      if (s == SD_ERR_UNSUPPORTED) break;  // pointers the TMA cannot map: one layer at a time below
+      if (s != SD_OK) return s;
+    }
+  }
+  const int launches = t_launches;
+  for (int l = l0; l < n_layers; ++l) {
+    s = launch_attn(q + l * q_layer, k_pages[l], v_pages ? v_pages[l] : nullptr, block_table, seqlens, indices, pd, B,
+                    H, Dk, Dv, k, scale, out + l * o_layer, lse ? lse + l * l_layer : nullptr, workspace, cap, st);
+    if (s != SD_OK) return s;
+  }
+  t_launches += launches;
+  return SD_OK;
 }
 
 sd_status sd_decode_step(const int8_t* qi, const int32_t* w, const int8_t* ki_pages, const uint16_t* q,

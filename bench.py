@@ -432,6 +432,99 @@ def bench_ours(args, rank, world, local):
         print(json.dumps(line), flush=True)
 
 
+def bench_layers(args, rank, world, local):
+    """Attention-only decode over args.layers layers that share one selection
+    (sd_sparse_attn_layers), against the same layers as separate
+    sd_sparse_attn calls. Layer l uses the workload's queries with the heads
+    rolled by l and its cache scaled by 1 + (l mod 4)/4 (one pool per layer in
+    HBM). L2 is flushed before every timed replay, as in the decode-step bench."""
+    import torch
+    import top_sparse_decode_paged_b200 as sd
+
+    torch.cuda.set_device(local)
+    wl = W.make(rank_spec(args.config, rank))
+    s = wl.spec
+    n = args.layers
+    dev = "cuda"
+    t = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(dev)  # noqa: E731
+    qi, w, ki = t(wl.qi), t(wl.w), t(wl.ki_pages)
+    bt, sl = t(wl.block_table), t(wl.seqlens)
+    q0 = t(wl.q.view(np.int16)).view(torch.bfloat16)
+    kp0 = t(wl.k_pages.view(np.int16)).view(torch.bfloat16)
+    vp0 = None if wl.v_pages is None else t(wl.v_pages.view(np.int16)).view(torch.bfloat16)
+    B = wl.seqlens.shape[0]
+    idx = sd.sd_indexer_topk(qi, w, ki, bt, sl, s.k, wl.max_seqlen)
+    del ki
+    q = torch.stack([torch.roll(q0, l, dims=1) for l in range(n)]).contiguous()
+    kps = [kp0] + [(kp0.float() * (1 + (l % 4) / 4)).to(torch.bfloat16) for l in range(1, n)]
+    vps = None if vp0 is None else [vp0] + [(vp0.float() * (1 + (l % 4) / 4)).to(torch.bfloat16) for l in range(1, n)]
+    out = torch.empty((n, B, s.H, s.Dv), dtype=torch.bfloat16, device=dev)
+    lib = sd.load_library()
+    ws_l = torch.empty(int(lib.sd_attn_layers_workspace_size(n, B, s.G, s.k, s.H, s.Dv)), dtype=torch.uint8, device=dev)
+    ws_1 = sd.alloc_workspace(B, s.G, 0, s.k, s.H, s.Dv)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    clean = torch.zeros(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def flush_l2():
+        flush.zero_()
+        clean.max()
+
+    def together():
+        sd.sd_sparse_attn_layers(q, kps, vps, bt, sl, idx, s.scale, s.Dv, out=out, workspace=ws_l)
+
+    def apart():
+        for l in range(n):
+            sd.sd_sparse_attn(q[l], kps[l], None if vps is None else vps[l], bt, sl, idx, s.scale, s.Dv,
+                              out=out[l], workspace=ws_1)
+
+    def timed(fn):
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            fn()
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=side):
+            fn()
+        for _ in range(args.warmup):
+            flush_l2()
+            g.replay()
+        torch.cuda.synchronize()
+        stream = torch.cuda.current_stream()
+        tot = 0.0
+        for _ in range(args.steps):
+            flush_l2()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            g.replay()
+            b.record(stream)
+            b.synchronize()
+            tot += a.elapsed_time(b)
+        del g
+        return max_over_ranks(tot / args.steps, world)
+
+    ms_together = timed(together)
+    ms_apart = timed(apart)
+    lens = wl.seqlens.astype(np.int64)
+    row_bytes = s.Dk * 2 if s.v_in_k else (s.Dk + s.Dv) * 2
+    nbytes = n * int(np.minimum(lens, s.k).sum()) * s.G * row_bytes
+    peak, peak_kind = _peaks()
+    achieved = nbytes / (ms_together * 1e-3) / 1e9
+    line = {
+        "metric": "attention-only decode layer-queries/s (layers sharing one selection), 1 B200",
+        "value": world * n * B / (ms_together * 1e-3), "unit": "layer-queries/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "layers": n,
+        "ms_per_step": ms_together, "ms_per_step_separate_calls": ms_apart,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": _config(s, "flushed before every step (256 MiB write, then 256 MiB read; outside the timed events)"),
+        "roofline": {"kernel": "attn (all layers, with combine)", "bound": "hbm", "achieved": achieved, "peak": peak,
+                     "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak, "traffic": None,
+                     "algorithmic_bytes_per_launch": nbytes, "ms_per_launch": ms_together},
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -441,6 +534,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="time eager calls instead of a CUDA graph replay")
+    ap.add_argument("--layers", type=int, default=0,
+                    help="time attention-only decode over this many layers sharing one selection instead")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     rank, world, local = _dist_env()
@@ -455,6 +550,8 @@ def main():
     try:
         if args.impl == "reference":
             bench_reference(args, rank, world)
+        elif args.layers > 0:
+            bench_layers(args, rank, world, local)
         else:
             bench_ours(args, rank, world, local)
     finally:

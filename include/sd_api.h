@@ -150,6 +150,31 @@ sd_status sd_sparse_attn_layers(const uint16_t* q, const uint16_t* const* k_page
                                 int32_t Dv, int32_t k, float scale, uint16_t* out, float* lse, void* workspace,
                                 size_t workspace_bytes, void* stream);
 
+/* Steps 3 + 4 with the selection given in the packed forms of the unified
+ * sparse runtime ("Unify sparse attention framework with clean backend
+ * interfaces", runtime parameters sparse_attn_offsets and
+ * sparse_attn_indices_block_size):
+ *   indices     int32, all rows' entries packed (may be NULL if every row is
+ *               empty); row r = b * G + g owns indices[offsets[r] ..
+ *               offsets[r + 1]).
+ *   offsets     int32 [B * G + 1], non-decreasing.
+ *   block_size  0 or 1: an entry is a token; bs > 1: entry e selects tokens
+ *               e*bs .. e*bs + bs - 1.
+ *   max_selected  1 .. 2048: the most tokens any row keeps.
+ * Row r attends over the valid tokens of its expansion, in list order: entries
+ * < 0 are skipped, tokens at or past seqlens[b] are dropped, and only the
+ * first min(max_selected, seqlens[b]) are kept. An entry whose whole block is
+ * past the seqlen, decreasing offsets, or more valid tokens than kept set
+ * SD_DEVERR_INDEX. Duplicates are attended as listed. Other arguments,
+ * outputs and errors as for sd_sparse_attn. Workspace:
+ * sd_csr_workspace_size(). */
+size_t sd_csr_workspace_size(int32_t B, int32_t G, int32_t max_selected, int32_t H, int32_t Dv);
+sd_status sd_sparse_attn_csr(const uint16_t* q, const uint16_t* k_pages, const uint16_t* v_pages,
+                             const int32_t* block_table, const int32_t* seqlens, const int32_t* indices,
+                             const int32_t* offsets, int32_t block_size, int32_t max_selected, sd_paged_desc pd,
+                             int32_t B, int32_t H, int32_t Dk, int32_t Dv, float scale, uint16_t* out, float* lse,
+                             void* workspace, size_t workspace_bytes, void* stream);
+
 /* Steps 1 + 2 + 3 in one call on one stream (arguments as above). */
 sd_status sd_decode_step(const int8_t* qi, const int32_t* w, const int8_t* ki_pages,
                          const uint16_t* q, const uint16_t* k_pages, const uint16_t* v_pages,

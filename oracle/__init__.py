@@ -8,9 +8,11 @@ from .sd_oracle import (  # noqa: F401
     bf16_bits_to_f64,
     decode_step,
     dense_attention,
+    expand_csr,
     gather_token_rows,
     indexer_scores,
     sparse_attention,
+    sparse_attention_csr,
     topk_indices,
     topk_row,
 )

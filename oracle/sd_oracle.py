@@ -20,6 +20,9 @@ attend over the selected tokens):
 3. ``sparse_attention`` for every query head h (KV head g = h // (H/G)):
    o = sum_j softmax_j(scale * q_h . K_j) V_j over the selected rows j.
 4. ``dense_attention``  the same over every cached token (the dense golden case).
+5. ``expand_csr`` / ``sparse_attention_csr``  the selection given as CSR
+   offsets and block-sized indices ("Unify sparse attention framework with
+   clean backend interfaces", runtime parameters), expanded to tokens.
 
 Readings where the pages are silent (the pages never write the formulas):
 the per-head ReLU and integer head weights of the indexer; ties broken toward
@@ -145,6 +148,50 @@ def sparse_attention(q, k_pages, v_pages, Dv, block_table, seqlens, indices, sca
             for h in range(g * qpk, (g + 1) * qpk):
                 out[i, h], lse[i, h] = attend_rows(bf16_bits_to_f64(q[b, h]), K, V, scale)
     return out, lse
+
+
+def expand_csr(indices_flat, offsets, block_size, seqlens, G, max_selected):
+    """The packed selection of the unified sparse runtime ("Unify sparse
+    attention framework with clean backend interfaces", runtime parameters
+    sparse_attn_offsets / sparse_attn_indices_block_size), in the padded form.
+
+    Row r = b*G + g owns entries offsets[r] .. offsets[r+1]-1. Entry e covers
+    tokens e*bs .. e*bs+bs-1 with bs = max(block_size, 1); entries < 0 are
+    skipped and tokens at or past L_b dropped; the valid tokens keep list order
+    and the first min(max_selected, L_b) are kept. Returns, per request, int64
+    [G, max_selected] padded with -1."""
+    bs = max(int(block_size), 1)
+    out = []
+    for b in range(len(seqlens)):
+        L = int(seqlens[b])
+        cap = min(int(max_selected), L)
+        rows = np.full((G, int(max_selected)), -1, dtype=np.int64)
+        for g in range(G):
+            r = b * G + g
+            toks = []
+            for j in range(int(offsets[r]), int(offsets[r + 1])):
+                e = int(indices_flat[j])
+                if e < 0:
+                    continue
+                for u in range(bs):
+                    t = e * bs + u
+                    if t < L:
+                        toks.append(t)
+            toks = toks[:cap]
+            rows[g, :len(toks)] = toks
+        out.append(rows)
+    return out
+
+
+def sparse_attention_csr(q, k_pages, v_pages, Dv, block_table, seqlens, indices_flat, offsets, block_size,
+                         max_selected, scale, requests=None):
+    """Selected-token attention with the selection in CSR / block form
+    (``expand_csr``); duplicates are attended as listed."""
+    G = k_pages.shape[2]
+    sel = expand_csr(indices_flat, offsets, block_size, seqlens, G, max_selected)
+    req = list(range(len(seqlens))) if requests is None else list(requests)
+    return sparse_attention(q, k_pages, v_pages, Dv, block_table, seqlens, [sel[b] for b in req], scale,
+                            requests=req)
 
 
 def dense_attention(q, k_pages, v_pages, Dv, block_table, seqlens, G, scale, requests=None):

@@ -377,3 +377,49 @@ def test_planted_mistakes_are_caught():
     rng = np.random.default_rng(0)
     row = rng.integers(0, 3, size=30)
     assert m["ties_high"](row, 8).tolist() != _brute_topk(row.tolist(), 8)
+
+
+# ----------------------------------------------------------------------------
+# CSR offsets and block-sized indices
+# ----------------------------------------------------------------------------
+def test_csr_expansion_hand_worked():
+    """Blocks of 4 tokens, two requests (L = 22 and 9), G = 1:
+    request 0 lists blocks 5 and 0 -> tokens 20, 21 (22, 23 are past L) then
+    0..3; request 1 lists block 2 -> token 8 (9..11 past L); a negative entry
+    is skipped."""
+    out = oracle.expand_csr(np.array([5, 0, -3, 2]), np.array([0, 3, 4]), 4, np.array([22, 9]), 1, 8)
+    assert out[0].tolist() == [[20, 21, 0, 1, 2, 3, -1, -1]]
+    assert out[1].tolist() == [[8, -1, -1, -1, -1, -1, -1, -1]]
+    # at most min(max_selected, L) tokens are kept, in list order
+    out = oracle.expand_csr(np.array([1, 4, 6]), np.array([0, 3]), 1, np.array([10]), 1, 2)
+    assert out[0].tolist() == [[1, 4]]
+    out = oracle.expand_csr(np.array([1, 4, 6]), np.array([0, 3]), 0, np.array([5]), 1, 8)
+    assert out[0].tolist() == [[1, 4, -1, -1, -1, -1, -1, -1]]
+
+
+def test_csr_of_a_padded_selection_is_the_same_attention():
+    d = _tiny_paged(21, B=3, G=2, lens=(5, 11, 1), separate_v=True)
+    sc = oracle.indexer_scores(d["qi"], d["w"], d["ki"], d["bt"], d["seqlens"])
+    idx = oracle.topk_indices(sc, 3)
+    flat, offs = [], [0]
+    for b in range(3):
+        for g in range(2):
+            row = [int(t) for t in idx[b][g] if t >= 0]
+            flat += row
+            offs.append(offs[-1] + len(row))
+    a = oracle.sparse_attention(d["q"], d["kp"], d["vp"], d["Dv"], d["bt"], d["seqlens"], idx, 0.7)
+    c = oracle.sparse_attention_csr(d["q"], d["kp"], d["vp"], d["Dv"], d["bt"], d["seqlens"], np.array(flat),
+                                    np.array(offs), 1, 3, 0.7)
+    assert np.array_equal(a[0], c[0]) and np.array_equal(a[1], c[1])
+
+
+def test_csr_duplicates_weigh_twice():
+    """q = 0: the output is the mean over the listed rows, with a duplicate
+    counted twice: (2 v3 + v7) / 3."""
+    d = _tiny_paged(22, B=1, G=1, H=2, lens=(9,), separate_v=True)
+    d["q"][:] = 0
+    out, _ = oracle.sparse_attention_csr(d["q"], d["kp"], d["vp"], d["Dv"], d["bt"], d["seqlens"],
+                                         np.array([3, 7, 3]), np.array([0, 3]), 1, 8, 1.0)
+    P = d["P"]
+    v = lambda t: np.array([_bf16_to_float(x) for x in d["vp"][d["bt"][0][t // P]][t % P][0]])  # noqa: E731
+    np.testing.assert_allclose(out[0, 0], (2 * v(3) + v(7)) / 3, rtol=1e-13, atol=1e-15)

@@ -20,11 +20,13 @@ from .api import (  # noqa: F401
     sd_indexer_topk,
     sd_indexer_topk_noalloc,
     sd_sparse_attn,
+    sd_sparse_attn_csr,
     sd_sparse_attn_layers,
     workspace_size,
 )
 
 __all__ = [
-    "sd_indexer_topk", "sd_indexer_topk_noalloc", "sd_sparse_attn", "sd_sparse_attn_layers", "sd_decode_step",
+    "sd_indexer_topk", "sd_indexer_topk_noalloc", "sd_sparse_attn", "sd_sparse_attn_layers", "sd_sparse_attn_csr",
+    "sd_decode_step",
     "workspace_size", "alloc_workspace", "device_errors", "load_library", "SdError", "StageTimer",
 ]

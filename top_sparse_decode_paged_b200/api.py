@@ -22,7 +22,8 @@ SD_DEVERR_PAGE = 0x2
 SD_DEVERR_INDEX = 0x4
 
 EXPORTED = ("sd_workspace_size", "sd_indexer_topk", "sd_indexer_topk_noalloc", "sd_sparse_attn",
-            "sd_attn_layers_workspace_size", "sd_sparse_attn_layers", "sd_decode_step",
+            "sd_attn_layers_workspace_size", "sd_sparse_attn_layers", "sd_csr_workspace_size",
+            "sd_sparse_attn_csr", "sd_decode_step",
             "sd_set_stage_events", "sd_get_device_errors", "sd_status_str", "sd_last_cuda_error",
             "sd_last_launch_count", "sd_version")
 
@@ -67,6 +68,11 @@ def load_library(path: str = LIB_PATH):
     lib.sd_sparse_attn_layers.restype = i32
     lib.sd_sparse_attn_layers.argtypes = [p, p, p, i32, p, p, p, PagedDesc, i32, i32, i32, i32, i32,
                                           ctypes.c_float, p, p, p, sz, p]
+    lib.sd_csr_workspace_size.restype = sz
+    lib.sd_csr_workspace_size.argtypes = [i32] * 5
+    lib.sd_sparse_attn_csr.restype = i32
+    lib.sd_sparse_attn_csr.argtypes = [p, p, p, p, p, p, p, i32, i32, PagedDesc, i32, i32, i32, i32,
+                                       ctypes.c_float, p, p, p, sz, p]
     lib.sd_decode_step.restype = i32
     lib.sd_decode_step.argtypes = [p, p, p, p, p, p, p, p, PagedDesc, i32, i32, i32, i32, i32, i32,
                                    i32, i32, ctypes.c_float, p, p, p, p, p, sz, p]
@@ -212,6 +218,29 @@ def sd_sparse_attn_layers(q, k_pages, v_pages, block_table, seqlens, indices, sc
                                      _ptr(block_table), _ptr(seqlens), _ptr(indices), _desc(kps[0], block_table),
                                      B, H, Dk, Dv, k, float(scale), _ptr(out), _ptr(lse), _ptr(workspace),
                                      workspace.numel(), _stream(stream)))
+    return out
+
+
+def sd_sparse_attn_csr(q, k_pages, v_pages, block_table, seqlens, indices, offsets, block_size: int,
+                       max_selected: int, scale: float, Dv: int, out=None, lse=None, workspace=None, stream=None):
+    """Attention + combine with the selection in CSR form (``offsets`` [B*G+1],
+    ``indices`` packed, each entry a block of ``block_size`` tokens when > 1).
+    Returns ``out`` [B, H, Dv] bf16."""
+    lib = load_library()
+    q, k_pages = _bits(q), _bits(k_pages)
+    v_pages = _bits(v_pages) if v_pages is not None else None
+    B, H, Dk = q.shape
+    G = k_pages.shape[2]
+    if out is None:
+        out = torch.empty((B, H, Dv), dtype=torch.bfloat16, device=q.device)
+    if workspace is None:
+        nbytes = int(lib.sd_csr_workspace_size(B, G, max_selected, H, Dv))
+        workspace = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=q.device)
+    idx = indices if indices is not None and indices.numel() > 0 else None
+    _check(lib.sd_sparse_attn_csr(_ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(block_table), _ptr(seqlens),
+                                  _ptr(idx), _ptr(offsets), int(block_size), int(max_selected),
+                                  _desc(k_pages, block_table), B, H, Dk, Dv, float(scale), _ptr(out), _ptr(lse),
+                                  _ptr(workspace), workspace.numel(), _stream(stream)))
     return out
 
 

@@ -16,6 +16,7 @@
 #include "indexer_dp4a.cuh"
 #include "indexer_umma.cuh"
 #include "sd_common.cuh"
+#include "sparse_index.cuh"
 #include "topk_cluster.cuh"
 #include "topk_radix.cuh"
 
@@ -506,6 +507,39 @@ sd_status sd_sparse_attn_layers(const uint16_t* q, const uint16_t* const* k_page
   }
   t_launches += launches;
   return SD_OK;
+}
+
+size_t sd_csr_workspace_size(int32_t B, int32_t G, int32_t max_selected, int32_t H, int32_t Dv) {
+  if (B < 0 || G <= 0 || max_selected <= 0 || H <= 0 || Dv <= 0) return 0;
+  return align_up((size_t)B * G * max_selected * sizeof(int32_t)) + attn_bytes(B, G, H, max_selected, Dv);
+}
+
+sd_status sd_sparse_attn_csr(const uint16_t* q, const uint16_t* k_pages, const uint16_t* v_pages,
+                             const int32_t* block_table, const int32_t* seqlens, const int32_t* indices,
+                             const int32_t* offsets, int32_t block_size, int32_t max_selected, sd_paged_desc pd,
+                             int32_t B, int32_t H, int32_t Dk, int32_t Dv, float scale, uint16_t* out, float* lse,
+                             void* workspace, size_t workspace_bytes, void* stream) {
+  t_launches = 0;
+  if (offsets == nullptr || block_size < 0) return SD_ERR_INVALID_ARG;
+  // the packed entries may be empty: check the attention arguments with a placeholder for them
+  sd_status s = check_attn_args(q, k_pages, block_table, seqlens, indices ? indices : offsets, pd, B, H, Dk, Dv,
+                                max_selected, scale, out, v_pages != nullptr);
+  if (s != SD_OK) return s;
+  if (!ws_ok(workspace, workspace_bytes, sd_csr_workspace_size(B, pd.kv_heads, max_selected, H, Dv)))
+    return SD_ERR_WORKSPACE;
+  if (B == 0) return SD_OK;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int cap = pd.max_pages_per_req * pd.page_size;
+  int32_t* padded = static_cast<int32_t*>(workspace);
+  void* attn_ws = static_cast<char*>(workspace) + align_up((size_t)B * pd.kv_heads * max_selected * sizeof(int32_t));
+  s = launch_k(sd::csr_expand_kernel, dim3(B * pd.kv_heads), dim3(sd::kCsrThreads), 0, st,
+               indices ? indices : offsets, offsets, block_size, seqlens, pd.kv_heads, max_selected, cap, padded);
+  if (s != SD_OK) return s;
+  const int launches = t_launches;
+  s = launch_attn(q, k_pages, v_pages, block_table, seqlens, padded, pd, B, H, Dk, Dv, max_selected, scale, out, lse,
+                  attn_ws, cap, st);
+  t_launches += launches;
+  return s;
 }
 
 sd_status sd_decode_step(const int8_t* qi, const int32_t* w, const int8_t* ki_pages, const uint16_t* q,

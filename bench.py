@@ -525,6 +525,105 @@ def bench_layers(args, rank, world, local):
         print(json.dumps(line), flush=True)
 
 
+def bench_csr(args, rank, world, local):
+    """Attention with the selection in CSR form (sd_sparse_attn_csr): the
+    decode step's top-k selection packed per request (block size 1), or, with
+    --csr-block bs > 1, the blocks of bs tokens that hold the first 2048 / bs
+    selected tokens' blocks. Timed like the decode step (graph replay, L2
+    flushed), beside sd_sparse_attn on the padded top-k selection."""
+    import torch
+    import top_sparse_decode_paged_b200 as sd
+
+    torch.cuda.set_device(local)
+    wl = W.make(rank_spec(args.config, rank))
+    s = wl.spec
+    dev = "cuda"
+    t = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(dev)  # noqa: E731
+    qi, w, ki = t(wl.qi), t(wl.w), t(wl.ki_pages)
+    bt, sl = t(wl.block_table), t(wl.seqlens)
+    q = t(wl.q.view(np.int16)).view(torch.bfloat16)
+    kp = t(wl.k_pages.view(np.int16)).view(torch.bfloat16)
+    vp = None if wl.v_pages is None else t(wl.v_pages.view(np.int16)).view(torch.bfloat16)
+    B = wl.seqlens.shape[0]
+    idx = sd.sd_indexer_topk(qi, w, ki, bt, sl, s.k, wl.max_seqlen)
+    del ki
+    bs = max(args.csr_block, 1)
+    ix = idx.cpu().numpy().reshape(B * s.G, s.k)
+    flat, offs = [], [0]
+    for r in range(B * s.G):
+        row = ix[r][ix[r] >= 0]
+        if bs > 1:
+            row = np.unique(row // bs)[: max(s.k // bs, 1)]
+        flat.append(row.astype(np.int32))
+        offs.append(offs[-1] + len(row))
+    flat_t = t(np.concatenate(flat))
+    offs_t = t(np.asarray(offs, dtype=np.int32))
+    max_sel = s.k
+    out = torch.empty((B, s.H, s.Dv), dtype=torch.bfloat16, device=dev)
+    lib = sd.load_library()
+    ws_c = torch.empty(int(lib.sd_csr_workspace_size(B, s.G, max_sel, s.H, s.Dv)), dtype=torch.uint8, device=dev)
+    ws_p = sd.alloc_workspace(B, s.G, 0, s.k, s.H, s.Dv)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    clean = torch.zeros(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def flush_l2():
+        flush.zero_()
+        clean.max()
+
+    def csr():
+        sd.sd_sparse_attn_csr(q, kp, vp, bt, sl, flat_t, offs_t, bs, max_sel, s.scale, s.Dv, out=out, workspace=ws_c)
+
+    def padded():
+        sd.sd_sparse_attn(q, kp, vp, bt, sl, idx, s.scale, s.Dv, out=out, workspace=ws_p)
+
+    def timed(fn):
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            fn()
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=side):
+            fn()
+        for _ in range(args.warmup):
+            flush_l2()
+            g.replay()
+        torch.cuda.synchronize()
+        stream = torch.cuda.current_stream()
+        tot = 0.0
+        for _ in range(args.steps):
+            flush_l2()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            g.replay()
+            b.record(stream)
+            b.synchronize()
+            tot += a.elapsed_time(b)
+        del g
+        return max_over_ranks(tot / args.steps, world)
+
+    ms_csr = timed(csr)
+    ms_pad = timed(padded)
+    sel_tokens = int(sum(min(len(f) * bs, int(wl.seqlens[r // s.G]), max_sel) for r, f in enumerate(flat)))
+    row_bytes = s.Dk * 2 if s.v_in_k else (s.Dk + s.Dv) * 2
+    nbytes = sel_tokens * row_bytes
+    peak, peak_kind = _peaks()
+    achieved = nbytes / (ms_csr * 1e-3) / 1e9
+    line = {
+        "metric": "attention-only decode queries/s, selection as CSR offsets / block-sized indices, 1 B200",
+        "value": world * B / (ms_csr * 1e-3), "unit": "queries/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "block_size": bs, "selected_tokens": sel_tokens,
+        "ms_per_step": ms_csr, "ms_per_step_padded_topk_selection": ms_pad,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": _config(s, "flushed before every step (256 MiB write, then 256 MiB read; outside the timed events)"),
+        "roofline": {"kernel": "csr expansion + attn + combine", "bound": "hbm", "achieved": achieved, "peak": peak,
+                     "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak, "traffic": None,
+                     "algorithmic_bytes_per_launch": nbytes, "ms_per_launch": ms_csr},
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -534,6 +633,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="time eager calls instead of a CUDA graph replay")
+    ap.add_argument("--csr-block", type=int, default=0,
+                    help="time attention with the selection as CSR offsets, blocks of this many tokens (1: tokens)")
     ap.add_argument("--layers", type=int, default=0,
                     help="time attention-only decode over this many layers sharing one selection instead")
     args = ap.parse_args()
@@ -552,6 +653,8 @@ def main():
             bench_reference(args, rank, world)
         elif args.layers > 0:
             bench_layers(args, rank, world, local)
+        elif args.csr_block > 0:
+            bench_csr(args, rank, world, local)
         else:
             bench_ours(args, rank, world, local)
     finally:

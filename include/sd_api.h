@@ -127,6 +127,32 @@ sd_status sd_sparse_attn(const uint16_t* q, const uint16_t* k_pages, const uint1
                          int32_t Dk, int32_t Dv, int32_t k, float scale, uint16_t* out,
                          float* lse, void* workspace, size_t workspace_bytes, void* stream);
 
+/* Steps 1 + 2, and the whole decode step, with the previous step's selection
+ * as a hint: the "heuristic_prev_topk" feedback of "Overlap DSA heuristic
+ * prev_topk write-back on the aux stream" (Description: each decode step's
+ * top-k is the next step's pre_idx hint).
+ *   hint  int32 [B, G, k] request-local tokens (-1 and tokens >= seqlen are
+ *         ignored), typically the previous call's `indices`; NULL = no hint.
+ *         It must not be the same buffer as `indices`.
+ * The result is identical to the unhinted call for any hint. A good hint (the
+ * previous selection of a slowly changing query) narrows the radix passes of
+ * the top-k to the range between the hint's lowest current score and the best
+ * score outside it; an exact hint needs no radix pass at all. The write-back
+ * of the pages (a copy into the hint buffer) is not needed: alternate two
+ * `indices` buffers between steps and pass the other as the hint. Other
+ * arguments and errors as for sd_indexer_topk / sd_decode_step. */
+sd_status sd_indexer_topk_hinted(const int8_t* qi, const int32_t* w, const int8_t* ki_pages,
+                                 const int32_t* block_table, const int32_t* seqlens, sd_paged_desc pd, int32_t B,
+                                 int32_t Hi, int32_t Di, int32_t max_seqlen, int32_t k, const int32_t* hint,
+                                 int32_t* indices, int32_t* scores, void* workspace, size_t workspace_bytes,
+                                 void* stream);
+sd_status sd_decode_step_hinted(const int8_t* qi, const int32_t* w, const int8_t* ki_pages, const uint16_t* q,
+                                const uint16_t* k_pages, const uint16_t* v_pages, const int32_t* block_table,
+                                const int32_t* seqlens, sd_paged_desc pd, int32_t B, int32_t Hi, int32_t Di,
+                                int32_t H, int32_t Dk, int32_t Dv, int32_t max_seqlen, int32_t k, float scale,
+                                const int32_t* hint, int32_t* indices, int32_t* scores, uint16_t* out, float* lse,
+                                void* workspace, size_t workspace_bytes, void* stream);
+
 /* Steps 3 + 4 for n_layers layers that share one selection: the
  * shared-indexer decode of "Overlap DSA heuristic prev_topk write-back on the
  * aux stream" (Description: layers without their own indexer reuse the top-k

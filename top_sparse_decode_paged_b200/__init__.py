@@ -17,7 +17,9 @@ from .api import (  # noqa: F401
     last_launch_count,
     load_library,
     sd_decode_step,
+    sd_decode_step_hinted,
     sd_indexer_topk,
+    sd_indexer_topk_hinted,
     sd_indexer_topk_noalloc,
     sd_sparse_attn,
     sd_sparse_attn_csr,
@@ -26,7 +28,7 @@ from .api import (  # noqa: F401
 )
 
 __all__ = [
-    "sd_indexer_topk", "sd_indexer_topk_noalloc", "sd_sparse_attn", "sd_sparse_attn_layers", "sd_sparse_attn_csr",
+    "sd_indexer_topk", "sd_indexer_topk_hinted", "sd_indexer_topk_noalloc", "sd_decode_step_hinted", "sd_sparse_attn", "sd_sparse_attn_layers", "sd_sparse_attn_csr",
     "sd_decode_step",
     "workspace_size", "alloc_workspace", "device_errors", "load_library", "SdError", "StageTimer",
 ]

@@ -23,7 +23,7 @@ SD_DEVERR_INDEX = 0x4
 
 EXPORTED = ("sd_workspace_size", "sd_indexer_topk", "sd_indexer_topk_noalloc", "sd_sparse_attn",
             "sd_attn_layers_workspace_size", "sd_sparse_attn_layers", "sd_csr_workspace_size",
-            "sd_sparse_attn_csr", "sd_decode_step",
+            "sd_sparse_attn_csr", "sd_indexer_topk_hinted", "sd_decode_step_hinted", "sd_decode_step",
             "sd_set_stage_events", "sd_get_device_errors", "sd_status_str", "sd_last_cuda_error",
             "sd_last_launch_count", "sd_version")
 
@@ -73,6 +73,11 @@ def load_library(path: str = LIB_PATH):
     lib.sd_sparse_attn_csr.restype = i32
     lib.sd_sparse_attn_csr.argtypes = [p, p, p, p, p, p, p, i32, i32, PagedDesc, i32, i32, i32, i32,
                                        ctypes.c_float, p, p, p, sz, p]
+    lib.sd_indexer_topk_hinted.restype = i32
+    lib.sd_indexer_topk_hinted.argtypes = [p, p, p, p, p, PagedDesc, i32, i32, i32, i32, i32, p, p, p, p, sz, p]
+    lib.sd_decode_step_hinted.restype = i32
+    lib.sd_decode_step_hinted.argtypes = [p, p, p, p, p, p, p, p, PagedDesc, i32, i32, i32, i32, i32, i32,
+                                          i32, i32, ctypes.c_float, p, p, p, p, p, p, sz, p]
     lib.sd_decode_step.restype = i32
     lib.sd_decode_step.argtypes = [p, p, p, p, p, p, p, p, PagedDesc, i32, i32, i32, i32, i32, i32,
                                    i32, i32, ctypes.c_float, p, p, p, p, p, sz, p]
@@ -151,6 +156,23 @@ def sd_indexer_topk(qi, w, ki_pages, block_table, seqlens, k: int, max_seqlen: i
     return indices
 
 
+def sd_indexer_topk_hinted(qi, w, ki_pages, block_table, seqlens, k: int, max_seqlen: int, hint,
+                           indices=None, scores=None, workspace=None, stream=None):
+    """``sd_indexer_topk`` with the previous selection ``hint`` [B, G, k] (not
+    the output buffer); the result is the same for any hint."""
+    lib = load_library()
+    B, G, Hi, Di = qi.shape
+    if indices is None:
+        indices = torch.empty((B, G, k), dtype=torch.int32, device=qi.device)
+    if workspace is None and scores is None:
+        workspace = alloc_workspace(B, G, max_seqlen, k, G, 1, qi.device)
+    ws_bytes = workspace.numel() if workspace is not None else 0
+    _check(lib.sd_indexer_topk_hinted(_ptr(qi), _ptr(w), _ptr(ki_pages), _ptr(block_table), _ptr(seqlens),
+                                      _desc(ki_pages, block_table), B, Hi, Di, max_seqlen, k, _ptr(hint),
+                                      _ptr(indices), _ptr(scores), _ptr(workspace), ws_bytes, _stream(stream)))
+    return indices
+
+
 NOALLOC_MAX_SCORES = 4 << 20
 
 
@@ -190,6 +212,30 @@ def sd_sparse_attn(q, k_pages, v_pages, block_table, seqlens, indices, scale: fl
                               _ptr(indices), _desc(k_pages, block_table), B, H, Dk, Dv, k, float(scale),
                               _ptr(out), _ptr(lse), _ptr(workspace), workspace.numel(), _stream(stream)))
     return out
+
+
+def sd_decode_step_hinted(qi, w, ki_pages, q, k_pages, v_pages, block_table, seqlens, k: int, max_seqlen: int,
+                          scale: float, Dv: int, hint, indices=None, scores=None, out=None, lse=None,
+                          workspace=None, stream=None):
+    """``sd_decode_step`` with the previous selection ``hint`` [B, G, k] (not
+    the ``indices`` buffer). Returns (indices, out)."""
+    lib = load_library()
+    q, k_pages = _bits(q), _bits(k_pages)
+    v_pages = _bits(v_pages) if v_pages is not None else None
+    B, G, Hi, Di = qi.shape
+    H, Dk = q.shape[1], q.shape[2]
+    if indices is None:
+        indices = torch.empty((B, G, k), dtype=torch.int32, device=q.device)
+    if out is None:
+        out = torch.empty((B, H, Dv), dtype=torch.bfloat16, device=q.device)
+    if workspace is None:
+        workspace = alloc_workspace(B, G, max_seqlen, k, H, Dv, q.device)
+    _check(lib.sd_decode_step_hinted(_ptr(qi), _ptr(w), _ptr(ki_pages), _ptr(q), _ptr(k_pages), _ptr(v_pages),
+                                     _ptr(block_table), _ptr(seqlens), _desc(k_pages, block_table), B, Hi, Di,
+                                     H, Dk, Dv, max_seqlen, k, float(scale), _ptr(hint), _ptr(indices),
+                                     _ptr(scores), _ptr(out), _ptr(lse), _ptr(workspace), workspace.numel(),
+                                     _stream(stream)))
+    return indices, out
 
 
 def sd_sparse_attn_layers(q, k_pages, v_pages, block_table, seqlens, indices, scale: float, Dv: int,

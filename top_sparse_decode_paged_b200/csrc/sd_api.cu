@@ -248,7 +248,8 @@ sd_status launch_indexer_umma(const int8_t* qi, const int32_t* w, const int8_t* 
 
 template <int PER>
 sd_status launch_topk_cluster(const int32_t* scores, const int32_t* seqlens, int32_t* indices, int rows, int G,
-                              int max_seqlen, int cap, int k, int cs, const sd::RowMap& rm, cudaStream_t st) {
+                              int max_seqlen, int cap, int k, int cs, const sd::RowMap& rm, const int32_t* hint,
+                              cudaStream_t st) {
   const size_t smem = sizeof(sd::TopkClusterSmem<PER>);
   sd_status s = cuda_check(cudaFuncSetAttribute(sd::topk_cluster_kernel<PER>,
                                                 cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)));
@@ -268,21 +269,22 @@ sd_status launch_topk_cluster(const int32_t* scores, const int32_t* seqlens, int
   cfg.attrs = attr;
   cfg.numAttrs = t_stage_count == 0 ? 2 : 1;  // see launch_k
   return cuda_check(cudaLaunchKernelEx(&cfg, sd::topk_cluster_kernel<PER>, scores, seqlens, indices, G,
-                                       std::max(max_seqlen, 1), cap, k, rm));
+                                       std::max(max_seqlen, 1), cap, k, rm, hint));
 }
 
 // Top-k: one thread-block cluster per row when the row fits in the cluster's
 // shared memory (max_seqlen <= 8 x 512 x 32), else one CTA per row over L2.
 sd_status launch_topk(const int32_t* scores, const int32_t* seqlens, int32_t* indices, int B, int G,
-                      int max_seqlen, int cap, int k, const sd::RowMap& rm, cudaStream_t st) {
+                      int max_seqlen, int cap, int k, const sd::RowMap& rm, const int32_t* hint, cudaStream_t st) {
   const int rows = B * G;
   const int cs16 = sd::topk_cluster_size(max_seqlen, 16);
   const int cs32 = sd::topk_cluster_size(max_seqlen, 32);
   stage_mark(kStageTopk, 0, st);
   if ((cs16 > 0 || cs32 > 0) && rows <= 65535) {
     // 32 scores per thread measured faster than 16 (fewer CTAs per cluster)
-    const sd_status s = cs32 > 0 ? launch_topk_cluster<32>(scores, seqlens, indices, rows, G, max_seqlen, cap, k, cs32, rm, st)
-                                 : launch_topk_cluster<16>(scores, seqlens, indices, rows, G, max_seqlen, cap, k, cs16, rm, st);
+    const sd_status s =
+        cs32 > 0 ? launch_topk_cluster<32>(scores, seqlens, indices, rows, G, max_seqlen, cap, k, cs32, rm, hint, st)
+                 : launch_topk_cluster<16>(scores, seqlens, indices, rows, G, max_seqlen, cap, k, cs16, rm, hint, st);
     stage_mark(kStageTopk, 1, st);
     ++t_launches;
     return s;
@@ -296,7 +298,7 @@ sd_status launch_topk(const int32_t* scores, const int32_t* seqlens, int32_t* in
 sd_status launch_indexer_topk(const int8_t* qi, const int32_t* w, const int8_t* ki, const int32_t* bt,
                               const int32_t* seqlens, const sd_paged_desc& pd, int B, int Hi, int Di,
                               int max_seqlen, int k, int32_t* indices, int32_t* scores,
-                              cudaStream_t st, const sd::RowMap& rm = sd::RowMap{}) {
+                              cudaStream_t st, const sd::RowMap& rm = sd::RowMap{}, const int32_t* hint = nullptr) {
   const int G = pd.kv_heads;
   if (B == 0) return SD_OK;
   bool done = false;
@@ -312,7 +314,7 @@ sd_status launch_indexer_topk(const int8_t* qi, const int32_t* w, const int8_t* 
     if (s != SD_OK) return s;
   }
   const int cap = std::min(max_seqlen, pd.max_pages_per_req * pd.page_size);
-  return launch_topk(scores, seqlens, indices, B, G, max_seqlen, cap, k, rm, st);
+  return launch_topk(scores, seqlens, indices, B, G, max_seqlen, cap, k, rm, hint, st);
 }
 
 template <int DK, int DV, int MT>
@@ -429,22 +431,32 @@ size_t sd_workspace_size(int32_t B, int32_t G, int32_t max_seqlen, int32_t k, in
   return scores_bytes(B, G, max_seqlen) + attn_bytes(B, G, H, k, Dv);
 }
 
-sd_status sd_indexer_topk(const int8_t* qi, const int32_t* w, const int8_t* ki_pages,
-                          const int32_t* block_table, const int32_t* seqlens, sd_paged_desc pd,
-                          int32_t B, int32_t Hi, int32_t Di, int32_t max_seqlen, int32_t k,
-                          int32_t* indices, int32_t* scores, void* workspace, size_t workspace_bytes,
-                          void* stream) {
+sd_status sd_indexer_topk_hinted(const int8_t* qi, const int32_t* w, const int8_t* ki_pages,
+                                 const int32_t* block_table, const int32_t* seqlens, sd_paged_desc pd, int32_t B,
+                                 int32_t Hi, int32_t Di, int32_t max_seqlen, int32_t k, const int32_t* hint,
+                                 int32_t* indices, int32_t* scores, void* workspace, size_t workspace_bytes,
+                                 void* stream) {
   t_launches = 0;
   sd_status s = check_indexer_args(qi, w, ki_pages, block_table, seqlens, pd, B, Hi, Di, max_seqlen,
                                    k, indices);
   if (s != SD_OK) return s;
+  if (hint != nullptr && hint == indices) return SD_ERR_INVALID_ARG;
   if (scores == nullptr) {
     if (!ws_ok(workspace, workspace_bytes, scores_bytes(B, pd.kv_heads, max_seqlen)))
       return SD_ERR_WORKSPACE;
     scores = static_cast<int32_t*>(workspace);
   }
   return launch_indexer_topk(qi, w, ki_pages, block_table, seqlens, pd, B, Hi, Di, max_seqlen, k,
-                             indices, scores, static_cast<cudaStream_t>(stream));
+                             indices, scores, static_cast<cudaStream_t>(stream), sd::RowMap{}, hint);
+}
+
+sd_status sd_indexer_topk(const int8_t* qi, const int32_t* w, const int8_t* ki_pages,
+                          const int32_t* block_table, const int32_t* seqlens, sd_paged_desc pd,
+                          int32_t B, int32_t Hi, int32_t Di, int32_t max_seqlen, int32_t k,
+                          int32_t* indices, int32_t* scores, void* workspace, size_t workspace_bytes,
+                          void* stream) {
+  return sd_indexer_topk_hinted(qi, w, ki_pages, block_table, seqlens, pd, B, Hi, Di, max_seqlen, k, nullptr,
+                                indices, scores, workspace, workspace_bytes, stream);
 }
 
 sd_status sd_sparse_attn(const uint16_t* q, const uint16_t* k_pages, const uint16_t* v_pages,
@@ -542,10 +554,10 @@ sd_status sd_sparse_attn_csr(const uint16_t* q, const uint16_t* k_pages, const u
   return s;
 }
 
-sd_status sd_decode_step(const int8_t* qi, const int32_t* w, const int8_t* ki_pages, const uint16_t* q,
+sd_status sd_decode_step_hinted(const int8_t* qi, const int32_t* w, const int8_t* ki_pages, const uint16_t* q,
                          const uint16_t* k_pages, const uint16_t* v_pages, const int32_t* block_table,
                          const int32_t* seqlens, sd_paged_desc pd, int32_t B, int32_t Hi, int32_t Di,
-                         int32_t H, int32_t Dk, int32_t Dv, int32_t max_seqlen, int32_t k, float scale,
+                         int32_t H, int32_t Dk, int32_t Dv, int32_t max_seqlen, int32_t k, float scale, const int32_t* hint,
                          int32_t* indices, int32_t* scores, uint16_t* out, float* lse, void* workspace,
                          size_t workspace_bytes, void* stream) {
   t_launches = 0;
@@ -555,6 +567,7 @@ sd_status sd_decode_step(const int8_t* qi, const int32_t* w, const int8_t* ki_pa
   s = check_attn_args(q, k_pages, block_table, seqlens, indices, pd, B, H, Dk, Dv, k, scale, out,
                       v_pages != nullptr);
   if (s != SD_OK) return s;
+  if (hint != nullptr && hint == indices) return SD_ERR_INVALID_ARG;
   const size_t sb = scores_bytes(B, pd.kv_heads, max_seqlen);
   if (!ws_ok(workspace, workspace_bytes, sd_workspace_size(B, pd.kv_heads, max_seqlen, k, H, Dv)))
     return SD_ERR_WORKSPACE;
@@ -571,7 +584,7 @@ sd_status sd_decode_step(const int8_t* qi, const int32_t* w, const int8_t* ki_pa
     rm = sd::RowMap{reinterpret_cast<int32_t*>(static_cast<char*>(attn_ws) + sd::attn_umma_rows_offset(B)),
                     block_table, pd.page_size, pd.max_pages_per_req, pd.num_pages, sd::attn_kpad(k)};
   s = launch_indexer_topk(qi, w, ki_pages, block_table, seqlens, pd, B, Hi, Di, max_seqlen, k, indices,
-                          sc, st, rm);
+                          sc, st, rm, hint);
   if (s != SD_OK) return s;
   const int launches = t_launches;
   const int cap = std::min(max_seqlen, pd.max_pages_per_req * pd.page_size);
@@ -579,6 +592,17 @@ sd_status sd_decode_step(const int8_t* qi, const int32_t* w, const int8_t* ki_pa
                   lse, attn_ws, cap, st, umma);
   t_launches += launches;
   return s;
+}
+
+sd_status sd_decode_step(const int8_t* qi, const int32_t* w, const int8_t* ki_pages, const uint16_t* q,
+                         const uint16_t* k_pages, const uint16_t* v_pages, const int32_t* block_table,
+                         const int32_t* seqlens, sd_paged_desc pd, int32_t B, int32_t Hi, int32_t Di,
+                         int32_t H, int32_t Dk, int32_t Dv, int32_t max_seqlen, int32_t k, float scale,
+                         int32_t* indices, int32_t* scores, uint16_t* out, float* lse, void* workspace,
+                         size_t workspace_bytes, void* stream) {
+  return sd_decode_step_hinted(qi, w, ki_pages, q, k_pages, v_pages, block_table, seqlens, pd, B, Hi, Di, H, Dk, Dv,
+                               max_seqlen, k, scale, nullptr, indices, scores, out, lse, workspace, workspace_bytes,
+                               stream);
 }
 
 sd_status sd_set_stage_events(void* const* events, int32_t n) {

@@ -41,6 +41,8 @@ struct TopkClusterSmem {
   uint32_t red[kTkThreads / 32 * 2 + 8];        // block reduction / scan scratch
   uint32_t cta_vals[4];                         // values this CTA publishes to the cluster
   uint32_t found[2];                            // threshold digit, remaining
+  uint32_t mark[kTkThreads * PER / 32];         // hint tokens of this CTA's slice (one bit each)
+  uint32_t hvals[4];                            // hint bounds this CTA publishes
 };
 
 // Block-wide exclusive scan of 32-bit values (512 threads); returns the prefix,
@@ -100,7 +102,7 @@ __device__ __forceinline__ uint32_t tk_block_reduce(uint32_t v, uint32_t* scratc
 template <int PER>
 __global__ void __launch_bounds__(kTkThreads, 2) topk_cluster_kernel(
     const int32_t* __restrict__ scores, const int32_t* __restrict__ seqlens, int32_t* __restrict__ indices,
-    int G, int max_seqlen, int seqlen_cap, int k, RowMap rm) {
+    int G, int max_seqlen, int seqlen_cap, int k, RowMap rm, const int32_t* __restrict__ hint) {
   pdl_wait();  // inputs come from earlier work in the stream
   pdl_trigger();
 
@@ -147,6 +149,8 @@ __global__ void __launch_bounds__(kTkThreads, 2) topk_cluster_kernel(
     }
     sm.keys[(e / kTkPerThread) * kTkChunkStride + (e % kTkPerThread)] = u;
   }
+  if (hint != nullptr)
+    for (int i = tid; i < kTkThreads * PER / 32; i += kTkThreads) sm.mark[i] = 0u;
   kmin = tk_block_reduce(kmin, sm.red, false);
   kmax = tk_block_reduce(kmax, sm.red, true);
   if (tid == 0) {
@@ -172,19 +176,106 @@ __global__ void __launch_bounds__(kTkThreads, 2) topk_cluster_kernel(
     }
   }
   __syncthreads();
-  const uint32_t gmin = sm.found[0], gmax = sm.found[1];
+  uint32_t gmin = sm.found[0], gmax = sm.found[1];
+  uint32_t hi_cut = 0xffffffffu;              // keys above it are all selected
+  uint32_t remaining0 = static_cast<uint32_t>(k);
+
+  // ---- previous selection as a hint (exact for any hint) ----
+  // P = the hint's distinct tokens below L. If |P| = k, the k-th largest key
+  // T* is at least lo = min over P, and at most max(lo, hi) with hi = max over
+  // the other tokens (if T* exceeded both, the top-k would be P itself and
+  // T* = lo). So the radix passes only resolve [lo, max(lo, hi)], after
+  // taking every key above that range.
+  if (hint != nullptr) {
+    const int32_t* hr = hint + (size_t)row * k;
+    for (int i = crank * kTkThreads + tid; i < k; i += CS * kTkThreads) {
+      const int t = hr[i];
+      if (t >= 0 && t < L) {
+        const int owner = t / slice, off = t - owner * slice;
+        atomicOr(cluster.map_shared_rank(sm.mark, owner) + (off >> 5), 1u << (off & 31));
+      }
+    }
+    cluster.sync();  // every hint bit is set
+    uint32_t lo = 0xffffffffu, hi = 0u, np = 0u;
+    {
+      const uint32_t* chunk = sm.keys + tid * kTkChunkStride;
+      for (int j = 0; j < nvalid; ++j) {
+        const int e = tid * kTkPerThread + j;
+        const uint32_t u = chunk[j];
+        if ((sm.mark[e >> 5] >> (e & 31)) & 1u) {
+          lo = min(lo, u);
+          ++np;
+        } else {
+          hi = max(hi, u);
+        }
+      }
+    }
+    lo = tk_block_reduce(lo, sm.red, false);
+    hi = tk_block_reduce(hi, sm.red, true);
+    uint32_t np_tot;
+    tk_block_excl_scan(np, sm.red, &np_tot);
+    if (tid == 0) {
+      sm.hvals[0] = lo;
+      sm.hvals[1] = hi;
+      sm.hvals[2] = np_tot;
+    }
+    cluster.sync();
+    if (tid < 32) {
+      uint32_t l = 0xffffffffu, h = 0u, n = 0u;
+      if (tid < CS) {
+        const uint32_t* rv = cluster.map_shared_rank(sm.hvals, tid);
+        l = rv[0];
+        h = rv[1];
+        n = rv[2];
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        l = min(l, __shfl_xor_sync(0xffffffffu, l, o));
+        h = max(h, __shfl_xor_sync(0xffffffffu, h, o));
+        n += __shfl_xor_sync(0xffffffffu, n, o);
+      }
+      if (tid == 0) {
+        sm.found[0] = l;
+        sm.found[1] = n >= static_cast<uint32_t>(k) ? max(h, l) : 0xffffffffu;  // 0xffffffff: no bound
+      }
+    }
+    __syncthreads();
+    const uint32_t lo_all = sm.found[0], x = sm.found[1];
+    __syncthreads();
+    if (x != 0xffffffffu) {
+      uint32_t above = 0u;
+      const uint32_t* chunk = sm.keys + tid * kTkChunkStride;
+      for (int j = 0; j < nvalid; ++j) above += chunk[j] > x;
+      uint32_t above_cta;
+      tk_block_excl_scan(above, sm.red, &above_cta);
+      if (tid == 0) sm.hvals[3] = above_cta;
+      cluster.sync();
+      if (tid < 32) {
+        uint32_t n = tid < CS ? cluster.map_shared_rank(sm.hvals, tid)[3] : 0u;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) n += __shfl_xor_sync(0xffffffffu, n, o);
+        if (tid == 0) sm.found[0] = n;
+      }
+      __syncthreads();
+      remaining0 = static_cast<uint32_t>(k) - sm.found[0];
+      gmin = lo_all;
+      gmax = x;
+      hi_cut = x;
+      __syncthreads();
+    }
+  }
 
   // ---- radix passes from the highest differing bit ----
   uint32_t T;                 // threshold key
   uint32_t need_eq;           // keys == T to take (in token order)
   if (gmin == gmax) {
     T = gmax;
-    need_eq = static_cast<uint32_t>(k);
+    need_eq = remaining0;
   } else {
     const int hb = 31 - __clz(gmin ^ gmax);       // highest differing bit
     uint32_t prefix = hb == 31 ? 0u : (gmax >> (hb + 1)) << (hb + 1);
     uint32_t pmask = hb == 31 ? 0u : ~((2u << hb) - 1u);
-    uint32_t remaining = static_cast<uint32_t>(k);
+    uint32_t remaining = remaining0;
     int top = hb;                                   // highest unresolved bit
     bool settled = false;
     T = 0;
@@ -198,7 +289,7 @@ __global__ void __launch_bounds__(kTkThreads, 2) topk_cluster_kernel(
       const uint32_t* chunk = sm.keys + tid * kTkChunkStride;
       for (int j = 0; j < nvalid; ++j) {
         const uint32_t u = chunk[j];
-        if ((u & pmask) == prefix) atomicAdd(&sm.hist[(u >> shift) & dmask], 1u);
+        if ((u & pmask) == prefix && u <= hi_cut) atomicAdd(&sm.hist[(u >> shift) & dmask], 1u);
       }
       cluster.sync();  // every CTA's histogram is complete
       for (int i = tid; i < kTkBins; i += kTkThreads) {

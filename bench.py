@@ -624,6 +624,93 @@ def bench_csr(args, rank, world, local):
         print(json.dumps(line), flush=True)
 
 
+def bench_hint(args, rank, world, local):
+    """The decode step with the previous selection as the top-k hint, against
+    the same step without it. The hint is the selection of a slightly
+    different indexer query (10% of qi entries moved by up to 3), as between
+    consecutive decode steps; the exact hint (the selection itself) is timed
+    too. Each variant is a CUDA graph with stage events, so the top-k time is
+    read directly."""
+    import torch
+    import top_sparse_decode_paged_b200 as sd
+    from top_sparse_decode_paged_b200.api import StageTimer
+
+    torch.cuda.set_device(local)
+    wl = W.make(rank_spec(args.config, rank))
+    s = wl.spec
+    dev = "cuda"
+    t = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(dev)  # noqa: E731
+    rng = np.random.default_rng(1234)
+    qi_p = wl.qi.astype(np.int16)
+    m = rng.random(qi_p.shape) < 0.1
+    qi_p[m] += rng.integers(-3, 4, size=int(m.sum())).astype(np.int16)
+    qi_p = np.clip(qi_p, -64, 64).astype(np.int8)
+    qi, qip, w, ki = t(wl.qi), t(qi_p), t(wl.w), t(wl.ki_pages)
+    bt, sl = t(wl.block_table), t(wl.seqlens)
+    q = t(wl.q.view(np.int16)).view(torch.bfloat16)
+    kp = t(wl.k_pages.view(np.int16)).view(torch.bfloat16)
+    vp = None if wl.v_pages is None else t(wl.v_pages.view(np.int16)).view(torch.bfloat16)
+    B = wl.seqlens.shape[0]
+    Lmax = wl.max_seqlen
+    exact = sd.sd_indexer_topk(qi, w, ki, bt, sl, s.k, Lmax)
+    perturbed = sd.sd_indexer_topk(qip, w, ki, bt, sl, s.k, Lmax)
+    torch.cuda.synchronize()
+    same = float((exact == perturbed).float().mean().item())
+    idx = torch.empty_like(exact)
+    out = torch.empty((B, s.H, s.Dv), dtype=torch.bfloat16, device=dev)
+    ws = sd.alloc_workspace(B, s.G, Lmax, s.k, s.H, s.Dv)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    clean = torch.zeros(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def run(hint):
+        if hint is None:
+            sd.sd_decode_step(qi, w, ki, q, kp, vp, bt, sl, s.k, Lmax, s.scale, s.Dv, indices=idx, out=out,
+                              workspace=ws)
+        else:
+            sd.sd_decode_step_hinted(qi, w, ki, q, kp, vp, bt, sl, s.k, Lmax, s.scale, s.Dv, hint, indices=idx,
+                                     out=out, workspace=ws)
+
+    res = {}
+    for name, hint in (("none", None), ("perturbed", perturbed), ("exact", exact)):
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            run(hint)
+        torch.cuda.synchronize()
+        timer = StageTimer()
+        g = torch.cuda.CUDAGraph()
+        timer.arm()
+        with torch.cuda.graph(g, stream=side):
+            run(hint)
+        StageTimer.disarm()
+        ev = timer._pairs[0]
+        for _ in range(args.warmup):
+            flush.zero_()
+            clean.max()
+            g.replay()
+        torch.cuda.synchronize()
+        tot = dict.fromkeys(StageTimer.STAGES, 0.0)
+        for _ in range(args.steps):
+            flush.zero_()
+            clean.max()
+            g.replay()
+            torch.cuda.synchronize()
+            for j, nm in enumerate(StageTimer.STAGES):
+                tot[nm] += ev[2 * j].elapsed_time(ev[2 * j + 1])
+        res[name] = {k_: v / args.steps for k_, v in tot.items()}
+        del g
+        assert torch.equal(idx, exact), "hinted selection differs"
+    line = {
+        "metric": "top-k stage time of the decode step with and without the previous-selection hint, 1 B200",
+        "value": res["perturbed"]["topk"], "unit": "ms", "higher_is_better": False, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "hint_overlap_with_selection": same,
+        "stage_ms": res, "data": "synthetic",
+        "config": _config(s, "flushed before every step (256 MiB write, then 256 MiB read; outside the timed events)"),
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -633,6 +720,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="time eager calls instead of a CUDA graph replay")
+    ap.add_argument("--hint", action="store_true",
+                    help="time the decode step with the previous selection as the top-k hint instead")
     ap.add_argument("--csr-block", type=int, default=0,
                     help="time attention with the selection as CSR offsets, blocks of this many tokens (1: tokens)")
     ap.add_argument("--layers", type=int, default=0,
@@ -655,6 +744,8 @@ def main():
             bench_layers(args, rank, world, local)
         elif args.csr_block > 0:
             bench_csr(args, rank, world, local)
+        elif args.hint:
+            bench_hint(args, rank, world, local)
         else:
             bench_ours(args, rank, world, local)
     finally:

@@ -242,7 +242,10 @@ __global__ void __launch_bounds__(kTkThreads, 2) topk_cluster_kernel(
     __syncthreads();
     const uint32_t lo_all = sm.found[0], x = sm.found[1];
     __syncthreads();
-    if (x != 0xffffffffu) {
+    // narrow only when it saves a radix pass (the count above x costs one
+    // cluster round trip); bound-less hints fall through to the full range
+    auto passes = [](uint32_t a, uint32_t c) { return a == c ? 0 : (32 - __clz(a ^ c) + kTkBinsBits - 1) / kTkBinsBits; };
+    if (x != 0xffffffffu && passes(lo_all, x) < passes(gmin, gmax)) {
       uint32_t above = 0u;
       const uint32_t* chunk = sm.keys + tid * kTkChunkStride;
       for (int j = 0; j < nvalid; ++j) above += chunk[j] > x;

@@ -711,6 +711,106 @@ def bench_hint(args, rank, world, local):
         print(json.dumps(line), flush=True)
 
 
+def bench_tri(args, rank, world, local):
+    """TriAttention-style eviction of one layer (sd_tri_compact): score the
+    evictable region with calibrated queries, select the budget, compact K and
+    V in place. The pools are restored from pristine copies and L2 is flushed
+    before every step, outside the timed events; the call is replayed from a
+    CUDA graph."""
+    import torch
+    import top_sparse_decode_paged_b200 as sd
+
+    torch.cuda.set_device(local)
+    base = W.tri_spec(args.tri)
+    s = W.tri_spec(args.tri, seed=base.seed + 1000 * rank) if rank else base
+    w = W.make_tri(s)
+    mode = sd.TRI_PER_HEAD if args.tri_per_head else sd.TRI_UNION
+    dev = "cuda"
+    t = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(dev)  # noqa: E731
+    kp0 = t(w.k_pages.view(np.int16)).view(torch.bfloat16)
+    vp0 = t(w.v_pages.view(np.int16)).view(torch.bfloat16)
+    kp, vp = kp0.clone(), vp0.clone()
+    q_cal, bt, sl = t(w.q_cal), t(w.block_table), t(w.seqlens)
+    B = int(w.seqlens.shape[0])
+    lib = sd.load_library()
+    ws = torch.empty(int(lib.sd_tri_workspace_size(B, s.G, s.H, s.D, w.max_seqlen, s.n_sink, s.n_recent, s.budget,
+                                                     mode, 1)), dtype=torch.uint8, device=dev)
+    nl = torch.empty((B,), dtype=torch.int32, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    clean = torch.zeros(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def prepare():
+        kp.copy_(kp0)
+        vp.copy_(vp0)
+        flush.zero_()
+        clean.max()
+
+    def call():
+        sd.sd_tri_compact(q_cal, kp, vp, bt, sl, w.max_seqlen, s.n_sink, s.n_recent, s.budget, mode,
+                          new_seqlens=nl, workspace=ws)
+
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        call()
+    torch.cuda.synchronize()
+    launches = sd.last_launch_count()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=side):
+        call()
+    for _ in range(args.warmup):
+        prepare()
+        g.replay()
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    tot = 0.0
+    with ClockSampler(local) as clk:
+        for _ in range(args.steps):
+            prepare()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            g.replay()
+            b.record(stream)
+            b.synchronize()
+            tot += a.elapsed_time(b)
+    del g
+    ms = max_over_ranks(tot / args.steps, world)
+    nbytes = W.tri_algorithmic_bytes(s, w.seqlens, mode)
+    peak, peak_kind = _peaks()
+    achieved = nbytes / (ms * 1e-3) / 1e9
+    line = {
+        "metric": "KV-cache eviction (score, select, compact one layer) requests/s, 1 B200",
+        "value": world * B / (ms * 1e-3), "unit": "requests/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32 scores, bf16 rows", "data": "synthetic",
+        "config": {"workload": s.name, "B": B, "H": s.H, "kv_heads": s.G, "D": s.D, "page_size": s.page_size,
+                   "n_sink": s.n_sink, "n_recent": s.n_recent, "budget": s.budget,
+                   "mode": "per_head" if mode else "union", "max_seqlen": w.max_seqlen,
+                   "l2": "pools restored, then flushed (256 MiB write, 256 MiB read) before every step, "
+                         "outside the timed events"},
+        "gpu_launches": launches,
+        "clocks": clk.summary(),
+        "roofline": {"kernel": "score + reduce + top-k + gather + scatter", "bound": "hbm", "achieved": achieved,
+                     "peak": peak, "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak,
+                     "traffic": None, "algorithmic_bytes_per_launch": nbytes, "ms_per_launch": ms},
+    }
+    if rank == 0 and not args.no_cpu_baseline:
+        sys.path.insert(0, ROOT)
+        from oracle import tri_oracle as T
+        # the host pools are not used again: the oracle compacts them in place
+        t0 = time.perf_counter()
+        n = 0
+        while n < B and (n == 0 or time.perf_counter() - t0 < 15.0):
+            T.tri_evict(w.q_cal, w.k_pages, w.v_pages, w.block_table[n:n + 1], w.seqlens[n:n + 1], s.n_sink,
+                        s.n_recent, s.budget, mode, inplace=True)
+            n += 1
+        el = time.perf_counter() - t0
+        line["cpu_baseline"] = {"value": n / el, "unit": "requests/s", "cores": 1, "kind": "oracle",
+                                "sample": f"{n} of the {B} requests, one at a time"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -726,6 +826,9 @@ def main():
                     help="time attention with the selection as CSR offsets, blocks of this many tokens (1: tokens)")
     ap.add_argument("--layers", type=int, default=0,
                     help="time attention-only decode over this many layers sharing one selection instead")
+    ap.add_argument("--tri", default="", choices=[""] + list(W.TRI_SPECS),
+                    help="time one layer's KV-cache eviction (score, select, compact) on this workload instead")
+    ap.add_argument("--tri-per-head", action="store_true", help="with --tri: one selection per KV head")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     rank, world, local = _dist_env()
@@ -740,6 +843,8 @@ def main():
     try:
         if args.impl == "reference":
             bench_reference(args, rank, world)
+        elif args.tri:
+            bench_tri(args, rank, world, local)
         elif args.layers > 0:
             bench_layers(args, rank, world, local)
         elif args.csr_block > 0:

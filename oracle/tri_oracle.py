@@ -1,0 +1,157 @@
+"""CPU oracle for TriAttention-style decode-time eviction of one layer.
+
+TEST INFRASTRUCTURE ONLY. Only ``tests/``, ``__graft_entry__.smoke()`` and the
+``cpu_baseline`` / ``--impl reference`` legs of ``bench.py`` may import this
+module. The library never calls it and shares no code with it.
+
+What it computes ("Add TriAttention KV-cache compression method", Summary and
+Key Design Decisions: score the evictable decode region with per-head
+calibrated queries, keep ``budget`` tokens, compact the kept K/V entries in
+place inside the same paged pools, keep prompt and protected tails; union and
+per-head modes; deterministic tie settlement):
+
+1. ``tri_scores``   for request b with length L, evictable positions
+   p < E = max(0, L - n_sink - n_recent) (token n_sink + p):
+     z[h, p]  = q_cal[h] . K[n_sink + p, g(h)]
+     s[g, p]  = max over the query heads h of KV head g of (z[h, p] - max_p' z[h, p'])
+     union:     s[p] = max_g s[g, p]
+2. ``tri_select``   the ``budget`` largest scores, ties to the lower position,
+   in ascending position order (nothing is selected when E <= budget).
+3. ``tri_compact``  kept token i takes logical position i: the protected
+   prefix [0, n_sink) stays, then the selected positions, then the tail
+   [L - n_recent, L); the new length is n_sink + budget + n_recent. Union mode
+   moves whole rows, per-head mode each KV head's part by its own selection.
+
+Precision: the scores only decide an integer selection, so they are taken in
+the same precision as the library: fp32, every product and every partial sum
+rounded to fp32, summed over d in index order, with no fused multiply-add;
+z - max is one fp32 subtraction. (A score is never -0.0: the sums start at
++0.0 and x - x rounds to +0.0, so the comparison of fp32 values below is the
+same order as any total order on them.)
+
+Readings where the pages are silent (they name the steps, not the formulas):
+the score is the plain dot product with the calibrated query; each head is
+shifted by its own maximum before the maximum over heads; the protected prefix
+and tail are uniform sizes. The design notes list them.
+
+Parity pins: ``tests/test_tri_pins.py`` (one-hot queries against a closed form
+and an independent sort, an fp64 error bound, shift invariance of the per-head
+normalisation, a hand-worked compaction across pages, the degenerate cases).
+"""
+
+from __future__ import annotations
+
+import numpy as np
+
+from .sd_oracle import bf16_bits_to_f64, gather_token_rows
+
+UNION = 0
+PER_HEAD = 1
+
+
+def _evictable(L: int, n_sink: int, n_recent: int) -> int:
+    return max(0, L - n_sink - n_recent)
+
+
+def tri_logits(q_cal: np.ndarray, K: np.ndarray, G: int) -> np.ndarray:
+    """z[h, p] = q_cal[h] . K[p, h * G // H] in fp32, summed over d in index
+    order with each product and partial sum rounded (no fused multiply-add).
+
+    q_cal: fp32 [H, D]; K: fp32 [E, G, D] (bf16 values). Returns fp32 [H, E]."""
+    q_cal = np.asarray(q_cal, dtype=np.float32)
+    H, D = q_cal.shape
+    E = K.shape[0]
+    z = np.zeros((H, E), dtype=np.float32)
+    for h in range(H):
+        g = h * G // H
+        Kg = K[:, g, :].astype(np.float32)
+        acc = np.zeros(E, dtype=np.float32)
+        for d in range(D):
+            prod = (Kg[:, d] * q_cal[h, d]).astype(np.float32)
+            acc = (acc + prod).astype(np.float32)
+        z[h] = acc
+    return z
+
+
+def tri_scores(q_cal, k_pages, block_table, seqlens, n_sink: int, n_recent: int, mode: int):
+    """Per request, its selection rows' scores: fp32 [rows, E_b] with rows = 1
+    (union) or G (per-head). k_pages: uint16 bf16 bits [num_pages, P, G, D]."""
+    G = k_pages.shape[2]
+    H = q_cal.shape[0]
+    qpk = H // G
+    out = []
+    for b, L in enumerate(np.asarray(seqlens)):
+        E = _evictable(int(L), n_sink, n_recent)
+        tokens = np.arange(n_sink, n_sink + E)
+        K = bf16_bits_to_f64(gather_token_rows(k_pages, block_table[b], tokens)).astype(np.float32)
+        z = tri_logits(q_cal, K, G)
+        if E > 0:
+            zs = (z - z.max(axis=1, keepdims=True)).astype(np.float32)
+        else:
+            zs = z
+        per_g = np.stack([zs[g * qpk:(g + 1) * qpk].max(axis=0) if E > 0 else np.zeros(0, np.float32)
+                          for g in range(G)])
+        out.append(per_g if mode == PER_HEAD else per_g.max(axis=0, keepdims=True))
+    return out
+
+
+def tri_select(scores_b: np.ndarray, budget: int) -> np.ndarray:
+    """Kept evictable positions per selection row: int64 [rows, budget]
+    ascending, or [rows, 0] when the region holds at most ``budget`` tokens."""
+    rows, E = scores_b.shape
+    if E <= budget:
+        return np.zeros((rows, 0), dtype=np.int64)
+    out = np.zeros((rows, budget), dtype=np.int64)
+    for r in range(rows):
+        # full sort by (score descending, position ascending); lexsort keys go last-first
+        order = np.lexsort((np.arange(E), -scores_b[r].astype(np.float64)))
+        out[r] = np.sort(order[:budget])
+    return out
+
+
+def tri_kept_tokens(L: int, sel_row: np.ndarray, n_sink: int, n_recent: int, budget: int) -> np.ndarray:
+    """Old logical positions of the kept tokens, in their new order."""
+    if _evictable(L, n_sink, n_recent) <= budget:
+        return np.arange(L)
+    return np.concatenate([np.arange(n_sink), n_sink + np.asarray(sel_row), np.arange(L - n_recent, L)])
+
+
+def tri_compact(k_pages, v_pages, block_table, seqlens, selections, n_sink: int, n_recent: int, budget: int,
+                mode: int, inplace: bool = False):
+    """Compaction on copies of the pools (or, with ``inplace``, on the pools
+    given). Returns (k, v, new_seqlens); every byte outside the kept positions
+    is left as it was."""
+    k = k_pages if inplace else np.array(k_pages, copy=True)
+    v = None if v_pages is None else (v_pages if inplace else np.array(v_pages, copy=True))
+    P, G = k.shape[1], k.shape[2]
+    new_len = np.zeros(len(seqlens), dtype=np.int32)
+    for b, L in enumerate(np.asarray(seqlens)):
+        L = int(L)
+        if _evictable(L, n_sink, n_recent) <= budget:
+            new_len[b] = L
+            continue
+        new_len[b] = n_sink + budget + n_recent
+        bt = np.asarray(block_table[b], dtype=np.int64)
+        heads = [list(range(G))] if mode == UNION else [[g] for g in range(G)]
+        for r, hs in enumerate(heads):
+            src = tri_kept_tokens(L, selections[b][r], n_sink, n_recent, budget)
+            dst = np.arange(len(src))
+            sp, ss = bt[src // P], src % P
+            dp, ds = bt[dst // P], dst % P
+            for pool in (k, v):
+                if pool is None:
+                    continue
+                rows = pool[sp, ss][:, hs].copy()  # all reads before any write
+                for j in range(len(dst)):
+                    pool[dp[j], ds[j], hs] = rows[j]
+    return k, v, new_len
+
+
+def tri_evict(q_cal, k_pages, v_pages, block_table, seqlens, n_sink: int, n_recent: int, budget: int, mode: int,
+              inplace: bool = False):
+    """Scores, selection and compaction of one layer: (k, v, new_seqlens, selections)."""
+    scores = tri_scores(q_cal, k_pages, block_table, seqlens, n_sink, n_recent, mode)
+    selections = [tri_select(s, budget) for s in scores]
+    k, v, new_len = tri_compact(k_pages, v_pages, block_table, seqlens, selections, n_sink, n_recent, budget, mode,
+                                inplace)
+    return k, v, new_len, selections

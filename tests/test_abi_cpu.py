@@ -100,3 +100,26 @@ def test_layers_argument_errors(lib):
     assert lib.sd_attn_layers_workspace_size(40, 32, 1, 2048, 128, 512) == \
         lib.sd_attn_layers_workspace_size(16, 32, 1, 2048, 128, 512)
     assert lib.sd_last_launch_count() == 0
+
+
+def test_tri_compact_argument_errors(lib):
+    """sd_tri_compact: 1 = invalid, 2 = unsupported, 3 = workspace, all before
+    any launch; the workspace grows with the budget."""
+    desc = api.PagedDesc(64, 16, 8, 2)
+    f = lib.sd_tri_compact
+    ws = lambda *a: lib.sd_tri_workspace_size(*a)  # noqa: E731
+    args = lambda H=4, D=64, budget=8, mode=0, nws=0, B=2: (256, 256, None, 256, 256, desc, B, H, D, 100, 4,  # noqa: E731
+                                                              8, budget, mode, 256, 256 if nws else None, nws, None)
+    assert f(*args(H=5)) == 1            # H not a multiple of G
+    assert f(*args(budget=0)) == 1       # empty budget
+    assert f(*args(mode=2)) == 1         # unknown mode
+    assert f(*args(D=96)) == 2           # head width
+    assert f(*args(H=32)) == 2           # 16 query heads per KV head
+    assert f(*args(budget=4096)) == 2    # above the top-k limit
+    assert f(*args()) == 3               # no workspace
+    assert f(*args(nws=16)) == 3         # too small
+    assert ws(2, 2, 4, 64, 100, 4, 8, 0, 0, 1) == 0
+    a = ws(2, 2, 4, 64, 100, 4, 8, 24, 0, 0)
+    assert ws(2, 2, 4, 64, 100, 4, 8, 24, 0, 1) >= a > 0
+    assert ws(2, 2, 4, 64, 100, 4, 8, 48, 0, 0) > a
+    assert lib.sd_last_launch_count() == 0

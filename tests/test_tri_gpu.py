@@ -1,0 +1,144 @@
+"""GPU parity of the TriAttention eviction (sd_tri_compact) against the oracle.
+
+Scores decide an integer selection, so both sides take them in the same fp32
+arithmetic and everything is compared exactly: the new lengths, and every byte
+of the K and V pools after the in-place compaction ("Add TriAttention KV-cache
+compression method", Summary and Test Plan: union and per-head modes, ragged
+lengths and unaligned final tokens, heavy ties).
+"""
+import dataclasses
+
+import numpy as np
+import pytest
+
+from oracle import tri_oracle as T
+from top_sparse_decode_paged_b200.workloads import bf16_bits_from_f32, make_tri, tri_spec
+
+pytestmark = pytest.mark.gpu
+
+
+def _dev(a):
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(a)).cuda()
+
+
+def _bf16(a):
+    import torch
+    return _dev(a.view(np.int16)).view(torch.bfloat16)
+
+
+def _bits(t):
+    import torch
+    return t.view(torch.int16).cpu().numpy().view(np.uint16)
+
+
+def _run_gpu(w, mode, budget=None):
+    import torch
+    import top_sparse_decode_paged_b200 as sd
+    s = w.spec
+    budget = s.budget if budget is None else budget
+    kp, vp = _bf16(w.k_pages), None if w.v_pages is None else _bf16(w.v_pages)
+    nl = sd.sd_tri_compact(_dev(w.q_cal), kp, vp, _dev(w.block_table), _dev(w.seqlens), w.max_seqlen, s.n_sink,
+                           s.n_recent, budget, mode)
+    torch.cuda.synchronize()
+    assert sd.device_errors() == 0
+    return _bits(kp), None if vp is None else _bits(vp), nl.cpu().numpy()
+
+
+def _check(w, mode, budget=None):
+    s = w.spec
+    budget = s.budget if budget is None else budget
+    k_ref, v_ref, nl_ref, _ = T.tri_evict(w.q_cal, w.k_pages, w.v_pages, w.block_table, w.seqlens, s.n_sink,
+                                          s.n_recent, budget, mode)
+    k, v, nl = _run_gpu(w, mode, budget)
+    assert np.array_equal(nl, nl_ref)
+    assert np.array_equal(k, k_ref)
+    if v_ref is not None:
+        assert np.array_equal(v, v_ref)
+    return nl
+
+
+@pytest.mark.parametrize("mode", [T.UNION, T.PER_HEAD])
+@pytest.mark.parametrize("with_v", [True, False])
+def test_tiny_ragged(mode, with_v):
+    """Lengths 100, 20, 37 (region 88, 8, 25 against budget 24): one request
+    keeps everything, one evicts a single token, pages end unaligned."""
+    w = make_tri(tri_spec("tri_tiny", with_v=with_v))
+    nl = _check(w, mode)
+    assert nl.tolist() == [4 + 24 + 8, 20, 4 + 24 + 8]
+
+
+@pytest.mark.parametrize("H,G,D", [(32, 8, 128), (8, 8, 64), (16, 8, 64), (16, 2, 128)])
+@pytest.mark.parametrize("mode", [T.UNION, T.PER_HEAD])
+def test_shapes_span_tiles(H, G, D, mode):
+    """Regions of several 128-position score tiles with ragged tails, every
+    supported query-heads-per-KV-head ratio (4, 1, 2, 8) and both widths."""
+    s = tri_spec("tri_ragged_b16", B=5, H=H, G=G, D=D, page_size=16, n_sink=40, n_recent=9, budget=200,
+                 ragged=(0, 700), seed=20 + H + G + D)
+    _check(make_tri(s), mode)
+
+
+def test_heavy_ties_on_gpu():
+    """Every key row equal: all scores tie at 0 and the lowest positions stay."""
+    s = tri_spec("tri_tiny", B=2, seqlens=(300, 129), budget=50, n_sink=3, n_recent=5, seed=30)
+    w = make_tri(s)
+    for b, L in enumerate(w.seqlens):
+        for t in range(int(L)):
+            w.k_pages[w.block_table[b, t // s.page_size], t % s.page_size] = bf16_bits_from_f32(
+                np.full((s.G, s.D), 0.5, np.float32))
+    for mode in (T.UNION, T.PER_HEAD):
+        _check(dataclasses.replace(w, k_pages=w.k_pages.copy(),
+                                   v_pages=None if w.v_pages is None else w.v_pages.copy()), mode)
+
+
+@pytest.mark.parametrize("budget", [1, 2048])
+def test_budget_extremes(budget):
+    s = tri_spec("tri_tiny", B=3, seqlens=(2100, 64, 5), n_sink=2, n_recent=3, budget=budget, seed=31)
+    _check(make_tri(s), T.UNION)
+
+
+def test_nothing_evictable_and_empty_batch():
+    import torch
+    import top_sparse_decode_paged_b200 as sd
+    s = tri_spec("tri_tiny", B=3, seqlens=(0, 12, 30), budget=24, seed=32)  # regions 0, 0, 18
+    w = make_tri(s)
+    k, v, nl = _run_gpu(w, T.UNION)
+    assert nl.tolist() == [0, 12, 30]
+    assert np.array_equal(k, w.k_pages) and np.array_equal(v, w.v_pages)
+    kp = _bf16(w.k_pages)
+    empty = torch.zeros((0,), dtype=torch.int32, device="cuda")
+    out = sd.sd_tri_compact(_dev(w.q_cal), kp, None, _dev(w.block_table[:0]), empty, 0, 4, 8, 24)
+    torch.cuda.synchronize()
+    assert out.numel() == 0
+
+
+def test_bad_page_is_reported_without_fault():
+    import torch
+    import top_sparse_decode_paged_b200 as sd
+    w = make_tri(tri_spec("tri_tiny"))
+    bt = w.block_table.copy()
+    bt[0, 2] = w.k_pages.shape[0] + 5  # out of the pool, inside the request
+    kp = _bf16(w.k_pages)
+    sd.sd_tri_compact(_dev(w.q_cal), kp, None, _dev(bt), _dev(w.seqlens), w.max_seqlen, 4, 8, 24)
+    torch.cuda.synchronize()
+    assert sd.device_errors() & sd.SD_DEVERR_PAGE
+
+
+def test_full_size_sampled_requests():
+    """The measured workload (32 requests, Qwen3-8B attention shape, region
+    4096, budget 2048) in the launch configuration the benchmark times; the
+    oracle recomputes sampled requests, compared page by page."""
+    w = make_tri(tri_spec("tri_b32_qwen3_8b"))
+    s = w.spec
+    k, v, nl = _run_gpu(w, T.UNION)
+    assert np.all(nl == s.n_sink + s.budget + s.n_recent)
+    P = s.page_size
+    k_ref, v_ref = w.k_pages, w.v_pages  # requests own disjoint pages: one in-place copy serves all
+    for b in (0, 13, 31):
+        n = (int(w.seqlens[b]) + P - 1) // P
+        pages = w.block_table[b, :n]
+        _, _, nl_ref, _ = T.tri_evict(w.q_cal, k_ref, v_ref, w.block_table[b:b + 1], w.seqlens[b:b + 1],
+                                      s.n_sink, s.n_recent, s.budget, T.UNION, inplace=True)
+        assert nl_ref[0] == nl[b]
+        assert np.array_equal(k[pages], k_ref[pages])
+        assert np.array_equal(v[pages], v_ref[pages])

@@ -1,0 +1,185 @@
+"""Pins of the TriAttention eviction oracle to facts outside itself.
+
+The steps follow "Add TriAttention KV-cache compression method" (Summary: score
+the evictable decode region with per-head calibrated queries, keep `budget`
+tokens, compact in place; Key Design Decisions: in-place compaction inside the
+same pools, prompt and protected tails preserved; Test Plan: union and
+per-head modes, ragged lengths, deterministic heavy-tie settlement).
+"""
+import itertools
+
+import numpy as np
+import pytest
+
+from oracle import tri_oracle as T
+from top_sparse_decode_paged_b200.workloads import bf16_bits_from_f32, make_tri, tri_spec
+
+
+def _pool_from_values(vals: np.ndarray, P: int, perm=None):
+    """Pages [n_pages, P, G, D] holding token rows vals [L, G, D] (bf16 bits),
+    with a page permutation; returns (pool, block_table_row)."""
+    L = vals.shape[0]
+    n = (L + P - 1) // P
+    perm = np.arange(n) if perm is None else np.asarray(perm)
+    pool = np.zeros((n, P) + vals.shape[1:], dtype=np.uint16)
+    for t in range(L):
+        pool[perm[t // P], t % P] = vals[t]
+    return pool, perm.astype(np.int32)
+
+
+def test_logits_within_fp32_bound_of_fp64_dot():
+    """z agrees with the exact fp64 dot product (head h reads KV head h // (H/G))
+    within the recursive-summation bound (D + 1) u sum|q k|; a transposed
+    operand, a wrong head map or a dropped term breaks the bound."""
+    rng = np.random.default_rng(0)
+    H, G, D, E = 6, 3, 64, 40
+    q = rng.standard_normal((H, D), dtype=np.float32)
+    K = bf16_bits_from_f32(rng.standard_normal((E, G, D), dtype=np.float32))
+    Kf = (K.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    z = T.tri_logits(q, Kf.astype(np.float32), G)
+    u = 2.0 ** -24
+    for h in range(H):
+        g = h // (H // G)
+        exact = Kf[:, g, :] @ q[h].astype(np.float64)
+        bound = (D + 1) * u * (np.abs(Kf[:, g, :]) @ np.abs(q[h].astype(np.float64)))
+        assert np.all(np.abs(z[h] - exact) <= bound)
+
+
+def test_one_hot_queries_closed_form_and_independent_sort():
+    """q_cal[h] = 2 e_{d_h}: z[h, p] = 2 K[p, g, d_h] exactly; with one head the
+    selection is the `budget` largest K[., d_0], ties to the lower position."""
+    rng = np.random.default_rng(1)
+    E, D, budget = 50, 64, 17
+    vals = rng.integers(-6, 7, size=(E, 1, D)).astype(np.float32)  # many ties
+    K = bf16_bits_from_f32(vals)
+    q = np.zeros((1, D), dtype=np.float32)
+    q[0, 5] = 2.0
+    z = T.tri_logits(q, vals, 1)
+    assert np.array_equal(z[0], 2.0 * vals[:, 0, 5])
+    pool, bt = _pool_from_values(K, P=8, perm=[3, 0, 6, 1, 5, 2, 4])
+    s = T.tri_scores(q, pool, bt[None], np.array([E]), 0, 0, T.UNION)[0]
+    sel = T.tri_select(s, budget)[0]
+    expect = sorted(sorted(range(E), key=lambda p: (-vals[p, 0, 5], p))[:budget])
+    assert sel.tolist() == expect
+
+
+def test_each_head_normalised_by_its_own_maximum():
+    """A constant key column seen by one head only shifts that head's logits;
+    after the per-head shift the union selection is unchanged, and each head's
+    best token (score 0, the maximum) is kept. Without the shift the offset
+    head would take every slot."""
+    rng = np.random.default_rng(2)
+    E, D, H = 24, 64, 2
+    vals = rng.integers(-4, 5, size=(E, 1, D)).astype(np.float32)
+    vals[:, 0, 63] = 8.0  # constant column
+    q = np.zeros((H, D), dtype=np.float32)
+    q[0, 3] = 1.0
+    q[1, 7] = 1.0
+    q_shift = q.copy()
+    q_shift[1, 63] = 16.0  # head 1 logits + 128 everywhere
+    pool, bt = _pool_from_values(bf16_bits_from_f32(vals), P=8)
+    budget = 6
+    sel = T.tri_select(T.tri_scores(q, pool, bt[None], np.array([E]), 0, 0, T.UNION)[0], budget)[0]
+    sel2 = T.tri_select(T.tri_scores(q_shift, pool, bt[None], np.array([E]), 0, 0, T.UNION)[0], budget)[0]
+    assert sel.tolist() == sel2.tolist()
+    for h, d in ((0, 3), (1, 7)):
+        best = min(range(E), key=lambda p: (-vals[p, 0, d], p))
+        assert best in sel.tolist()
+
+
+def test_union_is_max_of_per_head_and_selection_is_a_threshold_set():
+    w = make_tri(tri_spec("tri_tiny"))
+    s = w.spec
+    per = T.tri_scores(w.q_cal, w.k_pages, w.block_table, w.seqlens, s.n_sink, s.n_recent, T.PER_HEAD)
+    uni = T.tri_scores(w.q_cal, w.k_pages, w.block_table, w.seqlens, s.n_sink, s.n_recent, T.UNION)
+    for a, b in zip(per, uni):
+        assert np.array_equal(a.max(axis=0), b[0])
+        for row in a:
+            if row.size:
+                assert row.max() == 0.0 and np.all(row <= 0.0)
+    # every kept score >= every dropped score; among equal scores the lower position is kept
+    for sc in per:
+        sel = T.tri_select(sc, s.budget)
+        for r in range(sel.shape[0]):
+            kept = set(sel[r].tolist())
+            for p, q in itertools.product(range(sc.shape[1]), repeat=2):
+                if p in kept and q not in kept:
+                    assert sc[r, p] > sc[r, q] or (sc[r, p] == sc[r, q] and p < q)
+
+
+def test_heavy_ties_keep_the_lowest_positions():
+    E, D = 30, 64
+    vals = np.ones((E, 2, D), dtype=np.float32)
+    pool, bt = _pool_from_values(bf16_bits_from_f32(vals), P=4)
+    q = np.ones((4, D), dtype=np.float32)
+    for mode in (T.UNION, T.PER_HEAD):
+        sc = T.tri_scores(q, pool, bt[None], np.array([E]), 2, 3, mode)[0]
+        sel = T.tri_select(sc, 7)
+        assert np.all(sel == np.arange(7))
+
+
+def test_hand_worked_compaction_across_pages():
+    """L = 13, prefix 2, tail 3, budget 3, page 4, pages permuted: the evictable
+    region is tokens 2..9; keeping region positions {1, 4, 6} (tokens 3, 6, 8)
+    leaves tokens [0, 1, 3, 6, 8, 10, 11, 12] at positions 0..7; positions 8..12
+    keep their old rows. Per-head: head 1 keeps positions {0, 1, 2} (tokens
+    2, 3, 4) by its own selection."""
+    L, P, G, D = 13, 4, 2, 8
+    vals = np.zeros((L, G, D), dtype=np.float32)
+    for t in range(L):
+        for g in range(G):
+            vals[t, g, :] = 100 * g + t
+    K = bf16_bits_from_f32(vals)
+    V = bf16_bits_from_f32(-vals)
+    kp, bt = _pool_from_values(K, P, perm=[2, 0, 3, 1])
+    vp, _ = _pool_from_values(V, P, perm=[2, 0, 3, 1])
+
+    def token_at(pool, pos, g):
+        x = pool[bt[pos // P], pos % P, g, 0]
+        return float((np.uint32(x) << 16).view(np.float32))
+
+    sel_u = [np.array([[1, 4, 6]])]
+    k2, v2, nl = T.tri_compact(kp, vp, bt[None], np.array([L]), sel_u, 2, 3, 3, T.UNION)
+    assert nl.tolist() == [8]
+    expect = [0, 1, 3, 6, 8, 10, 11, 12, 8, 9, 10, 11, 12]
+    for pos, t in enumerate(expect):
+        for g in range(G):
+            assert token_at(k2, pos, g) == 100 * g + t
+            assert token_at(v2, pos, g) == -(100 * g + t)
+
+    sel_h = [np.array([[1, 4, 6], [0, 1, 2]])]
+    k3, _, nl = T.tri_compact(kp, None, bt[None], np.array([L]), sel_h, 2, 3, 3, T.PER_HEAD)
+    expect1 = [0, 1, 2, 3, 4, 10, 11, 12, 8, 9, 10, 11, 12]
+    for pos in range(L):
+        assert token_at(k3, pos, 0) == expect[pos]
+        assert token_at(k3, pos, 1) == 100 + expect1[pos]
+
+
+@pytest.mark.parametrize("L", [0, 3, 5, 10, 13])
+def test_nothing_moves_when_the_region_fits_the_budget(L):
+    """E = max(0, L - 5) <= budget 8: pools and lengths unchanged."""
+    rng = np.random.default_rng(L)
+    P, G, D = 4, 1, 64
+    n = max(1, (L + P - 1) // P)
+    kp = bf16_bits_from_f32(rng.standard_normal((n, P, G, D), dtype=np.float32))
+    bt = np.arange(n, dtype=np.int32)[None]
+    q = rng.standard_normal((2, D), dtype=np.float32)
+    k2, v2, nl, sel = T.tri_evict(q, kp, None, bt, np.array([L]), 2, 3, 8, T.UNION)
+    assert nl.tolist() == [L]
+    assert np.array_equal(k2, kp) and v2 is None
+    assert sel[0].shape == (1, 0)
+
+
+def test_compaction_brute_force_tiny():
+    """Every 3-subset of a 6-token region: the compacted request reads back as
+    prefix + subset + tail, and bytes past the new length are untouched."""
+    L, n_sink, n_recent, budget, P = 10, 1, 3, 3, 4
+    vals = np.arange(L, dtype=np.float32)[:, None, None] * np.ones((1, 1, 64), np.float32)
+    kp, bt = _pool_from_values(bf16_bits_from_f32(vals), P, perm=[1, 2, 0])
+    for sub in itertools.combinations(range(6), 3):
+        k2, _, nl = T.tri_compact(kp, None, bt[None], np.array([L]), [np.array([sub])], n_sink, n_recent,
+                                  budget, T.UNION)
+        assert nl[0] == 7
+        got = [float((np.uint32(k2[bt[i // P], i % P, 0, 0]) << 16).view(np.float32)) for i in range(L)]
+        assert got[:7] == [0] + [1 + s for s in sub] + [7, 8, 9]
+        assert got[7:] == [7, 8, 9]

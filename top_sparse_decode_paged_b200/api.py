@@ -24,7 +24,7 @@ SD_DEVERR_INDEX = 0x4
 EXPORTED = ("sd_workspace_size", "sd_indexer_topk", "sd_indexer_topk_noalloc", "sd_sparse_attn",
             "sd_attn_layers_workspace_size", "sd_sparse_attn_layers", "sd_csr_workspace_size",
             "sd_sparse_attn_csr", "sd_indexer_topk_hinted", "sd_decode_step_hinted", "sd_decode_step",
-            "sd_set_stage_events", "sd_get_device_errors", "sd_status_str", "sd_last_cuda_error",
+            "sd_tri_workspace_size", "sd_tri_compact", "sd_set_stage_events", "sd_get_device_errors", "sd_status_str", "sd_last_cuda_error",
             "sd_last_launch_count", "sd_version")
 
 
@@ -81,6 +81,10 @@ def load_library(path: str = LIB_PATH):
     lib.sd_decode_step.restype = i32
     lib.sd_decode_step.argtypes = [p, p, p, p, p, p, p, p, PagedDesc, i32, i32, i32, i32, i32, i32,
                                    i32, i32, ctypes.c_float, p, p, p, p, p, sz, p]
+    lib.sd_tri_workspace_size.restype = sz
+    lib.sd_tri_workspace_size.argtypes = [i32] * 10
+    lib.sd_tri_compact.restype = i32
+    lib.sd_tri_compact.argtypes = [p, p, p, p, p, PagedDesc, i32, i32, i32, i32, i32, i32, i32, i32, p, p, sz, p]
     lib.sd_set_stage_events.restype = i32
     lib.sd_set_stage_events.argtypes = [ctypes.POINTER(ctypes.c_void_p), i32]
     lib.sd_get_device_errors.restype = i32
@@ -310,6 +314,35 @@ def sd_decode_step(qi, w, ki_pages, q, k_pages, v_pages, block_table, seqlens, k
                               H, Dk, Dv, max_seqlen, k, float(scale), _ptr(indices), _ptr(scores),
                               _ptr(out), _ptr(lse), _ptr(workspace), workspace.numel(), _stream(stream)))
     return indices, out
+
+
+TRI_UNION = 0
+TRI_PER_HEAD = 1
+
+
+def sd_tri_compact(q_cal, k_pages, v_pages, block_table, seqlens, max_seqlen: int, n_sink: int, n_recent: int,
+                   budget: int, mode: int = TRI_UNION, new_seqlens=None, workspace=None, stream=None):
+    """TriAttention-style eviction of one layer: scores the evictable region of
+    every request with ``q_cal`` (fp32 [H, D]), keeps ``budget`` tokens and
+    compacts ``k_pages`` (and ``v_pages``; bf16 [num_pages, P, G, D]) in place.
+    Returns ``new_seqlens`` [B] int32."""
+    lib = load_library()
+    k_pages = _bits(k_pages)
+    v_pages = _bits(v_pages) if v_pages is not None else None
+    H, D = q_cal.shape
+    G = k_pages.shape[2]
+    B = seqlens.shape[0]
+    if new_seqlens is None:
+        new_seqlens = torch.empty((B,), dtype=torch.int32, device=k_pages.device)
+    if workspace is None:
+        nbytes = int(lib.sd_tri_workspace_size(B, G, H, D, max_seqlen, n_sink, n_recent, budget, mode,
+                                               1 if v_pages is not None else 0))
+        workspace = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=k_pages.device)
+    _check(lib.sd_tri_compact(_ptr(q_cal), _ptr(k_pages), _ptr(v_pages), _ptr(block_table), _ptr(seqlens),
+                              _desc(k_pages, block_table), B, H, D, int(max_seqlen), int(n_sink), int(n_recent),
+                              int(budget), int(mode), _ptr(new_seqlens), _ptr(workspace), workspace.numel(),
+                              _stream(stream)))
+    return new_seqlens
 
 
 def device_errors(clear: bool = True) -> int:

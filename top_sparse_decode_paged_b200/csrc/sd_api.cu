@@ -19,6 +19,7 @@
 #include "sparse_index.cuh"
 #include "topk_cluster.cuh"
 #include "topk_radix.cuh"
+#include "triattention.cuh"
 
 namespace {
 
@@ -552,6 +553,143 @@ sd_status sd_sparse_attn_csr(const uint16_t* q, const uint16_t* k_pages, const u
                   attn_ws, cap, st);
   t_launches += launches;
   return s;
+}
+
+}  // extern "C"
+
+namespace {
+struct TriPlan {
+  int rows_per_req, e_max, moved, part, n_tiles, chunk, n_chunks;
+  size_t off_tmax, off_keys, off_evict, off_sel, off_flags, total;
+};
+TriPlan tri_plan(int B, int G, int H, int D, int max_seqlen, int n_sink, int n_recent, int budget, int mode,
+                 bool has_v) {
+  TriPlan p{};
+  p.rows_per_req = mode == SD_TRI_PER_HEAD ? G : 1;
+  p.e_max = std::max(0, max_seqlen - n_sink - n_recent);
+  p.moved = budget + n_recent;
+  p.part = (mode == SD_TRI_PER_HEAD ? 1 : G) * D * 2;
+  p.n_tiles = (p.e_max + sd::kTriThreads - 1) / sd::kTriThreads;
+  p.chunk = std::max(1, std::min(sd::kTriMaxChunkTokens, sd::kTriChunkBytes / (p.part * (has_v ? 2 : 1))));
+  p.n_chunks = (p.moved + p.chunk - 1) / p.chunk;
+  const size_t rows = (size_t)B * p.rows_per_req;
+  p.off_tmax = align_up((size_t)B * H * p.e_max * sizeof(float));
+  p.off_keys = p.off_tmax + align_up((size_t)B * H * p.n_tiles * sizeof(float));
+  p.off_evict = p.off_keys + align_up(rows * p.e_max * sizeof(int32_t));
+  p.off_sel = p.off_evict + align_up((size_t)B * sizeof(int32_t));
+  p.off_flags = p.off_sel + align_up(rows * budget * sizeof(int32_t));
+  p.total = p.off_flags + align_up(rows * p.n_chunks * sizeof(int32_t));
+  return p;
+}
+bool tri_args_ok(int B, int G, int H, int D, int max_seqlen, int n_sink, int n_recent, int budget, int mode) {
+  return B >= 0 && G > 0 && H > 0 && H % G == 0 && max_seqlen >= 0 && n_sink >= 0 && n_recent >= 0 && budget >= 1 &&
+         (mode == SD_TRI_UNION || mode == SD_TRI_PER_HEAD);
+}
+// Co-resident CTAs of the compaction kernel on this device (its units wait on
+// one another, so every CTA of its grid must be resident at once).
+int tri_compact_grid() {
+  static int grid = 0;
+  if (grid == 0) {
+    int dev = 0, sms = 0, per_sm = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, sd::tri_compact_kernel, sd::kTriCompactThreads, 0) !=
+            cudaSuccess)
+      return 0;
+    grid = sms * per_sm;
+  }
+  return grid;
+}
+template <int D, int QPK>
+sd_status launch_tri_score(const float* q_cal, const uint16_t* kp, const int32_t* bt, const int32_t* seqlens,
+                           const sd_paged_desc& pd, int B, int H, int cap, int n_sink, int n_recent, int e_max, float* z,
+                           float* tmax, cudaStream_t st) {
+  auto kern = sd::tri_score_kernel<D, QPK>;
+  const int smem = static_cast<int>(sizeof(sd::TriScoreSmem<D, QPK>));
+  static int grid_cap = 0;  // co-resident CTAs (the kernel is persistent)
+  if (grid_cap == 0) {
+    int dev = 0, sms = 0, per_sm = 0;
+    sd_status s = cuda_check(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+    if (s != SD_OK) return s;
+    if ((s = cuda_check(cudaGetDevice(&dev))) != SD_OK) return s;
+    if ((s = cuda_check(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev))) != SD_OK) return s;
+    if ((s = cuda_check(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, sd::kTriThreads, smem))) !=
+        SD_OK)
+      return s;
+    grid_cap = std::max(1, sms * per_sm);
+  }
+  const long long tiles = (long long)B * pd.kv_heads * ((e_max + sd::kTriThreads - 1) / sd::kTriThreads);
+  const dim3 grid((unsigned)std::max(1LL, std::min<long long>(grid_cap, tiles)));
+  return launch_k(kern, grid, dim3(sd::kTriThreads), (size_t)smem, st, q_cal,
+                  reinterpret_cast<const __nv_bfloat16*>(kp), bt, seqlens, B, H, pd.kv_heads, pd.page_size,
+                  pd.max_pages_per_req, pd.num_pages, cap, n_sink, n_recent, e_max, z, tmax);
+}
+}  // namespace
+
+extern "C" {
+
+size_t sd_tri_workspace_size(int32_t B, int32_t G, int32_t H, int32_t D, int32_t max_seqlen, int32_t n_sink,
+                             int32_t n_recent, int32_t budget, int32_t mode, int32_t has_v) {
+  if (!tri_args_ok(B, G, H, D, max_seqlen, n_sink, n_recent, budget, mode)) return 0;
+  return tri_plan(B, G, H, D, max_seqlen, n_sink, n_recent, budget, mode, has_v != 0).total;
+}
+
+sd_status sd_tri_compact(const float* q_cal, uint16_t* k_pages, uint16_t* v_pages, const int32_t* block_table,
+                         const int32_t* seqlens, sd_paged_desc pd, int32_t B, int32_t H, int32_t D, int32_t max_seqlen,
+                         int32_t n_sink, int32_t n_recent, int32_t budget, int32_t mode, int32_t* new_seqlens,
+                         void* workspace, size_t workspace_bytes, void* stream) {
+  t_launches = 0;
+  if (!q_cal || !k_pages || !geom_ok(pd) || (B > 0 && (!block_table || !seqlens || !new_seqlens)))
+    return SD_ERR_INVALID_ARG;
+  const int G = pd.kv_heads;
+  if (!tri_args_ok(B, G, H, D, max_seqlen, n_sink, n_recent, budget, mode)) return SD_ERR_INVALID_ARG;
+  const int qpk = H / G;
+  if ((D != 64 && D != 128) || (qpk != 1 && qpk != 2 && qpk != 4 && qpk != 8) || budget > kMaxK)
+    return SD_ERR_UNSUPPORTED;
+  if ((long long)B * G > 65535 || H > sd::kTriMaxHeads) return SD_ERR_UNSUPPORTED;  // grid y; reduce heads
+  const bool has_v = v_pages != nullptr;
+  if ((mode == SD_TRI_PER_HEAD ? 1 : G) * D * 2 * (has_v ? 2 : 1) > sd::kTriChunkBytes) return SD_ERR_UNSUPPORTED;
+  const TriPlan p = tri_plan(B, G, H, D, max_seqlen, n_sink, n_recent, budget, mode, has_v);
+  if (!ws_ok(workspace, workspace_bytes, p.total)) return SD_ERR_WORKSPACE;
+  if (B == 0) return SD_OK;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  char* ws = static_cast<char*>(workspace);
+  float* z = reinterpret_cast<float*>(ws);
+  float* tmax = reinterpret_cast<float*>(ws + p.off_tmax);
+  int32_t* keys = reinterpret_cast<int32_t*>(ws + p.off_keys);
+  int32_t* evict = reinterpret_cast<int32_t*>(ws + p.off_evict);
+  int32_t* sel = reinterpret_cast<int32_t*>(ws + p.off_sel);
+  int32_t* flags = reinterpret_cast<int32_t*>(ws + p.off_flags);
+  const int cap = std::min(max_seqlen, pd.max_pages_per_req * pd.page_size);
+  const int rows = B * p.rows_per_req;
+  sd_status s = SD_OK;
+  if (p.e_max > 0) {
+#define SD_TRI(D_, Q_) \
+  s = launch_tri_score<D_, Q_>(q_cal, k_pages, block_table, seqlens, pd, B, H, cap, n_sink, n_recent, p.e_max, z, tmax, st)
+    if (D == 64) {
+      if (qpk == 1) SD_TRI(64, 1); else if (qpk == 2) SD_TRI(64, 2); else if (qpk == 4) SD_TRI(64, 4); else SD_TRI(64, 8);
+    } else {
+      if (qpk == 1) SD_TRI(128, 1); else if (qpk == 2) SD_TRI(128, 2); else if (qpk == 4) SD_TRI(128, 4); else SD_TRI(128, 8);
+    }
+#undef SD_TRI
+    if (s != SD_OK) return s;
+    const dim3 rgrid((unsigned)((p.e_max + sd::kTriReduceThreads - 1) / sd::kTriReduceThreads), (unsigned)rows);
+    if ((s = launch_k(sd::tri_reduce_kernel, rgrid, dim3(sd::kTriReduceThreads), 0, st, static_cast<const float*>(z),
+                      static_cast<const float*>(tmax), seqlens, H, G, p.rows_per_req, cap, n_sink, n_recent, p.e_max,
+                      keys, evict, flags, p.n_chunks)) != SD_OK)
+      return s;
+    if ((s = launch_topk(keys, evict, sel, B, p.rows_per_req, p.e_max, p.e_max, budget, sd::RowMap{}, nullptr, st)) !=
+        SD_OK)
+      return s;
+  }
+  const int grid = tri_compact_grid();
+  if (grid <= 0) return cuda_check(cudaGetLastError());
+  const long long units = (long long)rows * p.n_chunks;
+  return launch_k(sd::tri_compact_kernel, dim3((unsigned)std::max(1LL, std::min<long long>(grid, units))),
+                  dim3(sd::kTriCompactThreads), 0, st, reinterpret_cast<uint8_t*>(k_pages),
+                  reinterpret_cast<uint8_t*>(v_pages), block_table, seqlens, static_cast<const int32_t*>(sel),
+                  p.rows_per_req, pd.page_size, pd.max_pages_per_req, pd.num_pages, cap, n_sink, n_recent, budget,
+                  p.part, G * D * 2, p.chunk, p.n_chunks, rows, flags, new_seqlens);
 }
 
 sd_status sd_decode_step_hinted(const int8_t* qi, const int32_t* w, const int8_t* ki_pages, const uint16_t* q,

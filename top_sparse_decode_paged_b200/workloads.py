@@ -228,6 +228,123 @@ def make(s: Spec) -> Workload:
                     cluster_tokens=cluster_tokens)
 
 
+@dataclasses.dataclass
+class TriSpec:
+    """Shape and seed of one layer's eviction batch (calibrated queries plus a
+    paged K/V cache). Lengths: ``n_sink`` protected prefix tokens (the prompt)
+    + ``region`` evictable decode tokens + ``n_recent`` protected tail tokens,
+    or explicit ``seqlens``."""
+
+    name: str
+    B: int
+    page_size: int
+    G: int
+    H: int
+    D: int
+    n_sink: int
+    n_recent: int
+    budget: int
+    seed: int
+    region: int = 0
+    seqlens: Optional[tuple] = None
+    ragged: Optional[tuple] = None   # (lo, hi) evictable region, uniform integers
+    with_v: bool = True
+    spare_pages: int = 2
+
+
+def _tri_spec_table():
+    # Qwen3-8B attention shape (32 query heads over 8 KV heads, head dim 128),
+    # budget 2048, compaction every 2048 decode tokens: the region holds
+    # budget + 2048 tokens when an eviction runs.
+    q3 = dict(G=8, H=32, D=128, page_size=32, n_sink=1024, n_recent=16, budget=2048)
+    return {
+        "tri_tiny": TriSpec("tri_tiny", B=3, page_size=16, G=2, H=4, D=64, n_sink=4, n_recent=8, budget=24,
+                            seqlens=(100, 20, 37), seed=10),
+        "tri_b32_qwen3_8b": TriSpec("tri_b32_qwen3_8b", B=32, region=4096, seed=11, **q3),
+        # the same kernels on a quarter of the batch (pools still larger than L2), for detailed profiles
+        "tri_b8_qwen3_8b": TriSpec("tri_b8_qwen3_8b", B=8, region=4096, seed=13, **q3),
+        "tri_ragged_b16": TriSpec("tri_ragged_b16", B=16, ragged=(0, 8192), seed=12, **q3),
+    }
+
+
+TRI_SPECS = _tri_spec_table()
+
+
+def tri_spec(name: str, **overrides) -> TriSpec:
+    base = TRI_SPECS[name]
+    return dataclasses.replace(base, **overrides) if overrides else base
+
+
+@dataclasses.dataclass
+class TriWorkload:
+    """One eviction batch in host memory; bf16 arrays hold raw uint16 bits."""
+
+    spec: TriSpec
+    seqlens: np.ndarray       # int32 [B]
+    block_table: np.ndarray   # int32 [B, max_pages_per_req]
+    q_cal: np.ndarray         # fp32 [H, D]
+    k_pages: np.ndarray       # bf16 bits [num_pages, P, G, D]
+    v_pages: Optional[np.ndarray]
+
+    @property
+    def max_seqlen(self) -> int:
+        return int(self.seqlens.max()) if self.seqlens.size else 0
+
+
+def make_tri(s: TriSpec) -> TriWorkload:
+    """Draw order: seqlens, page permutation, q_cal, K pool, V pool; then poison
+    (bf16 NaN) in the slack of each last page and in the spare pages."""
+    rng = np.random.default_rng(s.seed)
+    P = s.page_size
+    if s.seqlens is not None:
+        seqlens = np.asarray(s.seqlens, dtype=np.int32)
+    elif s.ragged is not None:
+        region = rng.integers(s.ragged[0], s.ragged[1] + 1, size=s.B)
+        seqlens = (s.n_sink + region + s.n_recent).astype(np.int32)
+    else:
+        seqlens = np.full(s.B, s.n_sink + s.region + s.n_recent, dtype=np.int32)
+    B = int(seqlens.shape[0])
+    pages_per_req = [(int(L) + P - 1) // P for L in seqlens]
+    num_pages = int(sum(pages_per_req)) + s.spare_pages
+    max_pages = max(1, max(pages_per_req) if pages_per_req else 1)
+    perm = rng.permutation(num_pages).astype(np.int32)
+    block_table = np.full((B, max_pages), -1, dtype=np.int32)
+    cursor = 0
+    for b, n in enumerate(pages_per_req):
+        block_table[b, :n] = perm[cursor:cursor + n]
+        cursor += n
+    spare = perm[cursor:]
+    q_cal = rng.standard_normal((s.H, s.D), dtype=np.float32)
+    k_pages = _normal_bf16(rng, (num_pages, P, s.G, s.D))
+    v_pages = _normal_bf16(rng, (num_pages, P, s.G, s.D)) if s.with_v else None
+    for b in range(B):
+        L, n = int(seqlens[b]), pages_per_req[b]
+        if n and L % P:
+            for pool in (k_pages, v_pages):
+                if pool is not None:
+                    pool[block_table[b, n - 1], L % P:] = BF16_NAN
+    for phys in spare:
+        for pool in (k_pages, v_pages):
+            if pool is not None:
+                pool[phys] = BF16_NAN
+    return TriWorkload(spec=s, seqlens=seqlens, block_table=block_table, q_cal=q_cal, k_pages=k_pages,
+                       v_pages=v_pages)
+
+
+def tri_algorithmic_bytes(s: TriSpec, seqlens: np.ndarray, mode: int = 0) -> int:
+    """Bytes one eviction must move at minimum: every evictable token's K row
+    read once for scoring, plus, for each request that evicts, every moved
+    row (K and V) read once and written once."""
+    row = s.G * s.D * 2
+    total = 0
+    for L in np.asarray(seqlens):
+        E = max(0, int(L) - s.n_sink - s.n_recent)
+        total += E * row
+        if E > s.budget:
+            total += (s.budget + s.n_recent) * row * (2 if s.with_v else 1) * 2
+    return total
+
+
 def algorithmic_bytes(s: Spec, seqlens: np.ndarray) -> int:
     """Bytes a decode step must move at minimum: every cached token's indexer key
     (G*Di int8) plus each selected row (K, and V when it is a separate row)."""

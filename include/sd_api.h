@@ -132,22 +132,24 @@ sd_status sd_sparse_attn(const uint16_t* q, const uint16_t* k_pages, const uint1
  * evictable region [n_sink, L_b - n_recent) of every request with calibrated
  * per-head queries, keep the `budget` best tokens, and compact the kept K/V
  * rows in place to the front of the request's pages.
- *   q_cal       fp32 [H, D]: one calibrated query per query head (head h reads
- *               KV head h * G / H)
+ *   q_cal       bf16 [H, D]: one calibrated query per query head (head h reads
+ *               KV head h * G / H), in the cache's precision
  *   k_pages     bf16 [num_pages, P, G, D], compacted in place
  *   v_pages     bf16 [num_pages, P, G, D] compacted the same way, or NULL
  *   mode        SD_TRI_UNION: one selection per request (all KV heads move
  *               together); SD_TRI_PER_HEAD: one per (request, KV head)
  *   new_seqlens int32 [B] out: n_sink + budget + n_recent, or L_b when the
  *               evictable region holds at most `budget` tokens (nothing moves)
- * Score of evictable position p under query head h: z = q_cal[h] . K (fp32,
- * in index order, no fused multiply-add), shifted by the head's maximum over
+ * Score of evictable position p under query head h: z = q_cal[h] . K, one
+ * fp32 fused multiply-add per d in index order (the bf16 x bf16 product is
+ * exact, so the result is reproducible), shifted by the head's maximum over
  * the region; a KV head's score is the maximum over its query heads, the
  * union score the maximum over KV heads. The `budget` largest are kept (ties
  * to the lower position), followed by the recent tail. Pages past the new
  * lengths are free for the caller to release; the block table is unchanged.
- * Limits: D in {64, 128}; H / G in {1, 2, 4, 8}; 1 <= budget <= 2048;
- * B * G <= 65535. block_table, seqlens and new_seqlens may be NULL when B = 0.
+ * Limits: D in {64, 128}; H / G in {1, 2, 4, 8}; H <= 256;
+ * 1 <= budget <= 2048; B * G <= 65535; the bytes one token moves (union:
+ * G * D * 2, per-head: D * 2; twice that with V) at most 32768. block_table, seqlens and new_seqlens may be NULL when B = 0.
  * Workspace: sd_tri_workspace_size(); the caller owns every buffer. Errors:
  * SD_ERR_INVALID_ARG / SD_ERR_UNSUPPORTED / SD_ERR_WORKSPACE before any
  * launch; a block-table entry outside the pool inside a request sets
@@ -157,7 +159,7 @@ sd_status sd_sparse_attn(const uint16_t* q, const uint16_t* k_pages, const uint1
 #define SD_TRI_PER_HEAD 1
 size_t sd_tri_workspace_size(int32_t B, int32_t G, int32_t H, int32_t D, int32_t max_seqlen, int32_t n_sink,
                              int32_t n_recent, int32_t budget, int32_t mode, int32_t has_v);
-sd_status sd_tri_compact(const float* q_cal, uint16_t* k_pages, uint16_t* v_pages, const int32_t* block_table,
+sd_status sd_tri_compact(const uint16_t* q_cal, uint16_t* k_pages, uint16_t* v_pages, const int32_t* block_table,
                          const int32_t* seqlens, sd_paged_desc pd, int32_t B, int32_t H, int32_t D, int32_t max_seqlen,
                          int32_t n_sink, int32_t n_recent, int32_t budget, int32_t mode, int32_t* new_seqlens,
                          void* workspace, size_t workspace_bytes, void* stream);

@@ -12,7 +12,7 @@ per-head modes; deterministic tie settlement):
 
 1. ``tri_scores``   for request b with length L, evictable positions
    p < E = max(0, L - n_sink - n_recent) (token n_sink + p):
-     z[h, p]  = q_cal[h] . K[n_sink + p, g(h)]
+     z[h, p]  = q_cal[h] . K[n_sink + p, g(h)]      (q_cal and K bf16)
      s[g, p]  = max over the query heads h of KV head g of (z[h, p] - max_p' z[h, p'])
      union:     s[p] = max_g s[g, p]
 2. ``tri_select``   the ``budget`` largest scores, ties to the lower position,
@@ -23,11 +23,14 @@ per-head modes; deterministic tie settlement):
    moves whole rows, per-head mode each KV head's part by its own selection.
 
 Precision: the scores only decide an integer selection, so they are taken in
-the same precision as the library: fp32, every product and every partial sum
-rounded to fp32, summed over d in index order, with no fused multiply-add;
-z - max is one fp32 subtraction. (A score is never -0.0: the sums start at
-+0.0 and x - x rounds to +0.0, so the comparison of fp32 values below is the
-same order as any total order on them.)
+the same precision as the library: fp32, summed over d in index order, each
+step one fused multiply-add acc <- fl32(acc + q k). It is written out exactly:
+the bf16 x bf16 product is exact in fp64, and the fp64 sum of it and the fp32
+accumulator either is exact (operands within 2^29 of each other) or lies so far
+from an fp32 rounding boundary that rounding it to fp32 equals rounding the
+exact sum. z - max is one fp32 subtraction. (A score is never -0.0: the sums
+start at +0.0 and x - x rounds to +0.0, so the comparison of fp32 values below
+is the same order as any total order on them.)
 
 Readings where the pages are silent (they name the steps, not the formulas):
 the score is the plain dot product with the calibrated query; each head is
@@ -54,29 +57,31 @@ def _evictable(L: int, n_sink: int, n_recent: int) -> int:
 
 
 def tri_logits(q_cal: np.ndarray, K: np.ndarray, G: int) -> np.ndarray:
-    """z[h, p] = q_cal[h] . K[p, h * G // H] in fp32, summed over d in index
-    order with each product and partial sum rounded (no fused multiply-add).
+    """z[h, p] = q_cal[h] . K[p, h * G // H]: over d in index order, each step
+    one fp32 fused multiply-add (exact product, one rounding).
 
-    q_cal: fp32 [H, D]; K: fp32 [E, G, D] (bf16 values). Returns fp32 [H, E]."""
-    q_cal = np.asarray(q_cal, dtype=np.float32)
-    H, D = q_cal.shape
+    q_cal: [H, D] and K: [E, G, D], bf16 values in any float type.
+    Returns fp32 [H, E]."""
+    q = np.asarray(q_cal, dtype=np.float64)
+    H, D = q.shape
     E = K.shape[0]
     z = np.zeros((H, E), dtype=np.float32)
     for h in range(H):
         g = h * G // H
-        Kg = K[:, g, :].astype(np.float32)
+        Kg = np.asarray(K[:, g, :], dtype=np.float64)
         acc = np.zeros(E, dtype=np.float32)
         for d in range(D):
-            prod = (Kg[:, d] * q_cal[h, d]).astype(np.float32)
-            acc = (acc + prod).astype(np.float32)
+            acc = (acc.astype(np.float64) + Kg[:, d] * q[h, d]).astype(np.float32)
         z[h] = acc
     return z
 
 
 def tri_scores(q_cal, k_pages, block_table, seqlens, n_sink: int, n_recent: int, mode: int):
     """Per request, its selection rows' scores: fp32 [rows, E_b] with rows = 1
-    (union) or G (per-head). k_pages: uint16 bf16 bits [num_pages, P, G, D]."""
+    (union) or G (per-head). q_cal: bf16 bits [H, D]; k_pages: bf16 bits
+    [num_pages, P, G, D]."""
     G = k_pages.shape[2]
+    q_cal = bf16_bits_to_f64(q_cal)
     H = q_cal.shape[0]
     qpk = H // G
     out = []

@@ -27,22 +27,40 @@ def _pool_from_values(vals: np.ndarray, P: int, perm=None):
     return pool, perm.astype(np.int32)
 
 
+def _bf(x):
+    return (bf16_bits_from_f32(np.asarray(x, np.float32)).astype(np.uint32) << 16).view(np.float32)
+
+
 def test_logits_within_fp32_bound_of_fp64_dot():
     """z agrees with the exact fp64 dot product (head h reads KV head h // (H/G))
-    within the recursive-summation bound (D + 1) u sum|q k|; a transposed
-    operand, a wrong head map or a dropped term breaks the bound."""
+    within the recursive-summation bound D u sum|q k|; a transposed operand, a
+    wrong head map or a dropped term breaks the bound."""
     rng = np.random.default_rng(0)
     H, G, D, E = 6, 3, 64, 40
-    q = rng.standard_normal((H, D), dtype=np.float32)
-    K = bf16_bits_from_f32(rng.standard_normal((E, G, D), dtype=np.float32))
-    Kf = (K.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
-    z = T.tri_logits(q, Kf.astype(np.float32), G)
+    q = _bf(rng.standard_normal((H, D), dtype=np.float32)).astype(np.float64)
+    Kf = _bf(rng.standard_normal((E, G, D), dtype=np.float32)).astype(np.float64)
+    z = T.tri_logits(q, Kf, G)
     u = 2.0 ** -24
     for h in range(H):
         g = h // (H // G)
-        exact = Kf[:, g, :] @ q[h].astype(np.float64)
-        bound = (D + 1) * u * (np.abs(Kf[:, g, :]) @ np.abs(q[h].astype(np.float64)))
+        exact = Kf[:, g, :] @ q[h]
+        bound = D * u * (np.abs(Kf[:, g, :]) @ np.abs(q[h]))
         assert np.all(np.abs(z[h] - exact) <= bound)
+
+
+def test_each_step_rounds_to_fp32_in_index_order():
+    """Products 1, 2^-24, 2^-24 (q = k = 1, 2^-12, 2^-12): rounding after every
+    step in index order keeps 1 (each 1 + 2^-24 is a tie, to even); one
+    rounding of the exact sum, or the reverse order, gives 1 + 2^-23. A tiny
+    product under a large accumulator leaves it unchanged."""
+    v = np.array([1.0, 2.0 ** -12, 2.0 ** -12])
+    z = T.tri_logits(v[None, :], v.reshape(1, 1, 3), 1)
+    assert z[0, 0] == np.float32(1.0)
+    z = T.tri_logits(v[None, ::-1].copy(), v[::-1].reshape(1, 1, 3).copy(), 1)
+    assert z[0, 0] == np.float32(1.0 + 2.0 ** -23)
+    q = np.array([[2.0 ** 40, 2.0 ** -60]])
+    K = np.array([[[1.0, 1.0]]]).reshape(1, 1, 2)
+    assert T.tri_logits(q, K, 1)[0, 0] == np.float32(2.0 ** 40)
 
 
 def test_one_hot_queries_closed_form_and_independent_sort():
@@ -57,7 +75,7 @@ def test_one_hot_queries_closed_form_and_independent_sort():
     z = T.tri_logits(q, vals, 1)
     assert np.array_equal(z[0], 2.0 * vals[:, 0, 5])
     pool, bt = _pool_from_values(K, P=8, perm=[3, 0, 6, 1, 5, 2, 4])
-    s = T.tri_scores(q, pool, bt[None], np.array([E]), 0, 0, T.UNION)[0]
+    s = T.tri_scores(bf16_bits_from_f32(q), pool, bt[None], np.array([E]), 0, 0, T.UNION)[0]
     sel = T.tri_select(s, budget)[0]
     expect = sorted(sorted(range(E), key=lambda p: (-vals[p, 0, 5], p))[:budget])
     assert sel.tolist() == expect
@@ -79,8 +97,10 @@ def test_each_head_normalised_by_its_own_maximum():
     q_shift[1, 63] = 16.0  # head 1 logits + 128 everywhere
     pool, bt = _pool_from_values(bf16_bits_from_f32(vals), P=8)
     budget = 6
-    sel = T.tri_select(T.tri_scores(q, pool, bt[None], np.array([E]), 0, 0, T.UNION)[0], budget)[0]
-    sel2 = T.tri_select(T.tri_scores(q_shift, pool, bt[None], np.array([E]), 0, 0, T.UNION)[0], budget)[0]
+    sel = T.tri_select(T.tri_scores(bf16_bits_from_f32(q), pool, bt[None], np.array([E]), 0, 0, T.UNION)[0],
+                       budget)[0]
+    sel2 = T.tri_select(T.tri_scores(bf16_bits_from_f32(q_shift), pool, bt[None], np.array([E]), 0, 0,
+                                     T.UNION)[0], budget)[0]
     assert sel.tolist() == sel2.tolist()
     for h, d in ((0, 3), (1, 7)):
         best = min(range(E), key=lambda p: (-vals[p, 0, d], p))
@@ -111,7 +131,7 @@ def test_heavy_ties_keep_the_lowest_positions():
     E, D = 30, 64
     vals = np.ones((E, 2, D), dtype=np.float32)
     pool, bt = _pool_from_values(bf16_bits_from_f32(vals), P=4)
-    q = np.ones((4, D), dtype=np.float32)
+    q = bf16_bits_from_f32(np.ones((4, D), dtype=np.float32))
     for mode in (T.UNION, T.PER_HEAD):
         sc = T.tri_scores(q, pool, bt[None], np.array([E]), 2, 3, mode)[0]
         sel = T.tri_select(sc, 7)
@@ -163,7 +183,7 @@ def test_nothing_moves_when_the_region_fits_the_budget(L):
     n = max(1, (L + P - 1) // P)
     kp = bf16_bits_from_f32(rng.standard_normal((n, P, G, D), dtype=np.float32))
     bt = np.arange(n, dtype=np.int32)[None]
-    q = rng.standard_normal((2, D), dtype=np.float32)
+    q = bf16_bits_from_f32(rng.standard_normal((2, D), dtype=np.float32))
     k2, v2, nl, sel = T.tri_evict(q, kp, None, bt, np.array([L]), 2, 3, 8, T.UNION)
     assert nl.tolist() == [L]
     assert np.array_equal(k2, kp) and v2 is None

@@ -323,11 +323,11 @@ TRI_PER_HEAD = 1
 def sd_tri_compact(q_cal, k_pages, v_pages, block_table, seqlens, max_seqlen: int, n_sink: int, n_recent: int,
                    budget: int, mode: int = TRI_UNION, new_seqlens=None, workspace=None, stream=None):
     """TriAttention-style eviction of one layer: scores the evictable region of
-    every request with ``q_cal`` (fp32 [H, D]), keeps ``budget`` tokens and
+    every request with ``q_cal``, keeps ``budget`` tokens and
     compacts ``k_pages`` (and ``v_pages``; bf16 [num_pages, P, G, D]) in place.
-    Returns ``new_seqlens`` [B] int32."""
+    ``q_cal`` is bf16 [H, D]. Returns ``new_seqlens`` [B] int32."""
     lib = load_library()
-    k_pages = _bits(k_pages)
+    q_cal, k_pages = _bits(q_cal), _bits(k_pages)
     v_pages = _bits(v_pages) if v_pages is not None else None
     H, D = q_cal.shape
     G = k_pages.shape[2]

@@ -569,7 +569,7 @@ TriPlan tri_plan(int B, int G, int H, int D, int max_seqlen, int n_sink, int n_r
   p.e_max = std::max(0, max_seqlen - n_sink - n_recent);
   p.moved = budget + n_recent;
   p.part = (mode == SD_TRI_PER_HEAD ? 1 : G) * D * 2;
-  p.n_tiles = (p.e_max + sd::kTriThreads - 1) / sd::kTriThreads;
+  p.n_tiles = (p.e_max + sd::kTriTileTok - 1) / sd::kTriTileTok;
   p.chunk = std::max(1, std::min(sd::kTriMaxChunkTokens, sd::kTriChunkBytes / (p.part * (has_v ? 2 : 1))));
   p.n_chunks = (p.moved + p.chunk - 1) / p.chunk;
   const size_t rows = (size_t)B * p.rows_per_req;
@@ -601,28 +601,14 @@ int tri_compact_grid() {
   return grid;
 }
 template <int D, int QPK>
-sd_status launch_tri_score(const float* q_cal, const uint16_t* kp, const int32_t* bt, const int32_t* seqlens,
+sd_status launch_tri_score(const uint16_t* q_cal, const uint16_t* kp, const int32_t* bt, const int32_t* seqlens,
                            const sd_paged_desc& pd, int B, int H, int cap, int n_sink, int n_recent, int e_max, float* z,
                            float* tmax, cudaStream_t st) {
-  auto kern = sd::tri_score_kernel<D, QPK>;
-  const int smem = static_cast<int>(sizeof(sd::TriScoreSmem<D, QPK>));
-  static int grid_cap = 0;  // co-resident CTAs (the kernel is persistent)
-  if (grid_cap == 0) {
-    int dev = 0, sms = 0, per_sm = 0;
-    sd_status s = cuda_check(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
-    if (s != SD_OK) return s;
-    if ((s = cuda_check(cudaGetDevice(&dev))) != SD_OK) return s;
-    if ((s = cuda_check(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev))) != SD_OK) return s;
-    if ((s = cuda_check(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, sd::kTriThreads, smem))) !=
-        SD_OK)
-      return s;
-    grid_cap = std::max(1, sms * per_sm);
-  }
-  const long long tiles = (long long)B * pd.kv_heads * ((e_max + sd::kTriThreads - 1) / sd::kTriThreads);
-  const dim3 grid((unsigned)std::max(1LL, std::min<long long>(grid_cap, tiles)));
-  return launch_k(kern, grid, dim3(sd::kTriThreads), (size_t)smem, st, q_cal,
-                  reinterpret_cast<const __nv_bfloat16*>(kp), bt, seqlens, B, H, pd.kv_heads, pd.page_size,
-                  pd.max_pages_per_req, pd.num_pages, cap, n_sink, n_recent, e_max, z, tmax);
+  const dim3 grid((unsigned)((e_max + sd::kTriTileTok - 1) / sd::kTriTileTok), (unsigned)(B * pd.kv_heads));
+  return launch_k(sd::tri_score_kernel<D, QPK>, grid, dim3(sd::kTriThreads), 0, st,
+                  reinterpret_cast<const __nv_bfloat16*>(q_cal), reinterpret_cast<const __nv_bfloat16*>(kp), bt,
+                  seqlens, H, pd.kv_heads, pd.page_size, pd.max_pages_per_req, pd.num_pages, cap, n_sink, n_recent,
+                  e_max, z, tmax);
 }
 }  // namespace
 
@@ -634,7 +620,7 @@ size_t sd_tri_workspace_size(int32_t B, int32_t G, int32_t H, int32_t D, int32_t
   return tri_plan(B, G, H, D, max_seqlen, n_sink, n_recent, budget, mode, has_v != 0).total;
 }
 
-sd_status sd_tri_compact(const float* q_cal, uint16_t* k_pages, uint16_t* v_pages, const int32_t* block_table,
+sd_status sd_tri_compact(const uint16_t* q_cal, uint16_t* k_pages, uint16_t* v_pages, const int32_t* block_table,
                          const int32_t* seqlens, sd_paged_desc pd, int32_t B, int32_t H, int32_t D, int32_t max_seqlen,
                          int32_t n_sink, int32_t n_recent, int32_t budget, int32_t mode, int32_t* new_seqlens,
                          void* workspace, size_t workspace_bytes, void* stream) {
@@ -646,7 +632,8 @@ sd_status sd_tri_compact(const float* q_cal, uint16_t* k_pages, uint16_t* v_page
   const int qpk = H / G;
   if ((D != 64 && D != 128) || (qpk != 1 && qpk != 2 && qpk != 4 && qpk != 8) || budget > kMaxK)
     return SD_ERR_UNSUPPORTED;
-  if ((long long)B * G > 65535 || H > sd::kTriMaxHeads) return SD_ERR_UNSUPPORTED;  // grid y; reduce heads
+  // grid y of the score and reduce passes; heads of the reduce
+  if ((long long)B * G > 65535 || H > sd::kTriMaxHeads) return SD_ERR_UNSUPPORTED;
   const bool has_v = v_pages != nullptr;
   if ((mode == SD_TRI_PER_HEAD ? 1 : G) * D * 2 * (has_v ? 2 : 1) > sd::kTriChunkBytes) return SD_ERR_UNSUPPORTED;
   const TriPlan p = tri_plan(B, G, H, D, max_seqlen, n_sink, n_recent, budget, mode, has_v);

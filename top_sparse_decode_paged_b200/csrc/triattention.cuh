@@ -8,8 +8,9 @@
 // Scoring (a reading; the pages do not write the formula). For request b,
 // query head h (KV head g = h * G / H) and evictable position p (token
 // t = n_sink + p, p < E_b = L_b - n_sink - n_recent):
-//   z[b,h,p] = q_cal[h] . K[t, g]     fp32, products and sums in index order,
-//                                     no fused multiply-add (reproducible)
+//   z[b,h,p] = q_cal[h] . K[t, g]     q_cal and K bf16; one fp32 fused
+//                                     multiply-add per d, in index order
+//                                     (reproducible: the product is exact)
 //   m[b,h]   = max_p z[b,h,p]
 //   s[b,g,p] = max over the heads h of KV head g of (z[b,h,p] - m[b,h])
 //   union:     s[b,p] = max_g s[b,g,p]
@@ -42,180 +43,130 @@ __device__ __forceinline__ int tri_evictable(int L, int n_sink, int n_recent) {
   return max(0, L - n_sink - n_recent);
 }
 
-// Packed fp32 pair arithmetic: two independent IEEE round-to-nearest
-// operations per instruction (no fusion, no flush to zero).
-__device__ __forceinline__ unsigned long long tri_pack(float lo, float hi) {
-  unsigned long long r;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
-  return r;
-}
-__device__ __forceinline__ void tri_unpack(unsigned long long v, float& lo, float& hi) {
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
-}
-__device__ __forceinline__ unsigned long long tri_mul2(unsigned long long a, unsigned long long b) {
-  unsigned long long r;
-  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-  return r;
-}
-__device__ __forceinline__ unsigned long long tri_add2(unsigned long long a, unsigned long long b) {
-  unsigned long long r;
-  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-  return r;
-}
+constexpr int kTriTileTok = kTriThreads;  // evictable positions per score tile
 
-constexpr int kTriStages = 3;
-
-template <int D, int QPK>
-struct TriScoreSmem {
-  static constexpr int kStride = D * 2 + 16;  // padded row: per-thread row reads do not share banks
-  uint8_t k[kTriStages][kTriThreads * kStride];
-  float q[kTriStages][D * QPK];
-  float wmax[kTriThreads / 32][QPK];
-};
-
-// z[b][h][p] and the per-tile maxima tmax[b][h][tile], one tile = 128
-// consecutive evictable positions of one (request, KV head). Persistent: a
-// CTA walks tiles blockIdx.x, + gridDim.x, ... through a 3-stage cp.async ring,
-// so the rows of the next two tiles are in flight while a tile is summed.
-// Thread r copies and sums row r of each tile (the row's page id is fetched
-// one tile ahead into a register); a stage also holds the tile's q_cal slice,
-// interleaved by head ([d][j]), so one broadcast load feeds every head at a
-// given d. Each row is summed over d in index order, two heads per packed
-// instruction.
+// z[b][h][p] and the per-tile maxima tmax[b][h][tile] for one tile of 128
+// consecutive evictable positions of one (request, KV head) per CTA. The
+// tile's K rows (one D-wide bf16 segment per token) are staged in shared
+// memory by coalesced 16-byte cp.async (kChunks lanes per row; rows padded by
+// 16 bytes so that the per-thread row reads do not share banks); the KV
+// head's q_cal slice sits there as fp32 in [d][j] order, so one broadcast
+// load feeds four heads at a given d. Each row's source offset is computed
+// once (no division per copied piece).
+// Thread r sums row r over d in index order, one fused multiply-add per
+// (d, head). Small CTAs (about 37 KB) let six share an SM, so copies of some
+// overlap the arithmetic of others.
 template <int D, int QPK>
 __global__ void __launch_bounds__(kTriThreads) tri_score_kernel(
-    const float* __restrict__ q_cal, const __nv_bfloat16* __restrict__ k_pages, const int32_t* __restrict__ block_table,
-    const int32_t* __restrict__ seqlens, int B, int H, int G, int page_size, int max_pages, int num_pages,
-    int seqlen_cap, int n_sink, int n_recent, int e_max, float* __restrict__ z, float* __restrict__ tmax) {
-  using Smem = TriScoreSmem<D, QPK>;
-  constexpr int kChunks = D / 8, kStride = Smem::kStride;
-  extern __shared__ __align__(16) uint8_t smem_raw[];
-  Smem& sm = *reinterpret_cast<Smem*>(smem_raw);
+    const __nv_bfloat16* __restrict__ q_cal, const __nv_bfloat16* __restrict__ k_pages,
+    const int32_t* __restrict__ block_table, const int32_t* __restrict__ seqlens, int H, int G, int page_size,
+    int max_pages, int num_pages, int seqlen_cap, int n_sink, int n_recent, int e_max, float* __restrict__ z,
+    float* __restrict__ tmax) {
+  constexpr int kRowBytes = D * 2, kStride = kRowBytes + 16, kChunks = kRowBytes / 16;
+  __shared__ __align__(16) uint8_t ks[kTriThreads * kStride];
+  __shared__ __align__(16) float qs[D * QPK];
+  __shared__ long long roff[kTriThreads];
+  __shared__ float wmax[kTriThreads / 32][QPK];
+  const int b = blockIdx.y / G, g = blockIdx.y % G;
   pdl_wait();  // every input may come from earlier work in the stream
   pdl_trigger();
-  const int n_tiles = (e_max + kTriThreads - 1) / kTriThreads;
-  const long long total = (long long)B * G * n_tiles;
   const int r = threadIdx.x;
-  // tile k of this CTA: index blockIdx.x + k * gridDim.x
-  auto tile_of = [&](int k, int& b, int& g, int& p0, int& E) -> bool {
-    const long long T = blockIdx.x + (long long)k * gridDim.x;
-    if (T >= total) return false;
-    const int bg = static_cast<int>(T / n_tiles);
-    b = bg / G;
-    g = bg % G;
-    p0 = static_cast<int>(T % n_tiles) * kTriThreads;
-    E = tri_evictable(checked_seqlen(seqlens, b, seqlen_cap), n_sink, n_recent);
-    return p0 < E;
-  };
-  auto page_of = [&](int k) -> int {  // row r's page in tile k (-1: no row)
-    int b, g, p0, E;
-    if (!tile_of(k, b, g, p0, E) || p0 + r >= E) return -1;
-    const int t = n_sink + p0 + r;
-    return block_table[(size_t)b * max_pages + t / page_size];
-  };
-  auto issue = [&](int k, int page) {  // tile k into stage k % kTriStages
-    int b, g, p0, E;
-    if (tile_of(k, b, g, p0, E)) {
-      const int st = k % kTriStages;
-      for (int i = r; i < D * QPK; i += kTriThreads) {  // q slice in [d][j] order
-        const int d = i / QPK, j = i % QPK;
-        cp_async_4(&sm.q[st][i], q_cal + (size_t)(g * QPK + j) * D + d);
-      }
-      const bool ok = p0 + r < E && page >= 0 && page < num_pages;
-      const int t = n_sink + p0 + r;
-      const uint8_t* src = reinterpret_cast<const uint8_t*>(
-          k_pages + (((size_t)(ok ? page : 0) * page_size + t % page_size) * G + g) * D);
+  const int p0 = blockIdx.x * kTriTileTok;
+  // independent loads first: the length, row r's block-table entry (read
+  // whether or not the row exists, inside the request's table row) and this
+  // thread's share of q_cal
+  const int t = n_sink + p0 + r;
+  const int pi = t / page_size;
+  const int page_raw = pi < max_pages ? block_table[(size_t)b * max_pages + pi] : -1;
+  float qv[(D * QPK + kTriThreads - 1) / kTriThreads];
 #pragma unroll
-      for (int c = 0; c < kChunks; ++c) cp_async_16(&sm.k[st][r * kStride + c * 16], src + c * 16, ok ? 16 : 0);
-    }
-    cp_async_commit();  // one group per tile, empty or not
-  };
-  int pg_next = page_of(kTriStages - 1);
-  for (int k = 0; k < kTriStages - 1; ++k) issue(k, page_of(k));
-  for (int k = 0;; ++k) {
-    int b, g, p0, E;
-    const long long T = blockIdx.x + (long long)k * gridDim.x;
-    if (T >= total) break;
-    cp_async_wait<kTriStages - 2>();  // tile k has landed
-    __syncthreads();                  // ... for every thread; stage (k - 1) % kTriStages is free
-    issue(k + kTriStages - 1, pg_next);
-    pg_next = page_of(k + kTriStages);
-    if (!tile_of(k, b, g, p0, E)) continue;
-    const int st = k % kTriStages;
-    const bool in = p0 + r < E;
-    int page = -1;
-    if (in) page = block_table[(size_t)b * max_pages + (n_sink + p0 + r) / page_size];
-    const bool live = in && page >= 0 && page < num_pages;
-    if (in && !live) raise_error(SD_DEVERR_PAGE);
-    const uint8_t* krow = &sm.k[st][r * kStride];
-    const float* qs = sm.q[st];
-    float zv[QPK];
-    if constexpr (QPK == 1) {
-      float acc = 0.f;
+  for (int m = 0; m < (D * QPK + kTriThreads - 1) / kTriThreads; ++m) {
+    const int i = r + m * kTriThreads;
+    qv[m] = i < D * QPK ? __bfloat162float(q_cal[(size_t)(g * QPK + i % QPK) * D + i / QPK]) : 0.f;
+  }
+  const int L = checked_seqlen(seqlens, b, seqlen_cap);
+  const int E = tri_evictable(L, n_sink, n_recent);
+  if (p0 >= E) return;
+  const int nrows = min(kTriTileTok, E - p0);
+  const bool in = r < nrows;
+  // row r's source offset, once, for every copy of the row (-1: no row)
+  long long off = -1;
+  if (in) {
+    if (page_raw >= 0 && page_raw < num_pages)
+      off = (((long long)page_raw * page_size + t % page_size) * G + g) * kRowBytes;
+    else
+      raise_error(SD_DEVERR_PAGE);
+  }
+  const bool live = off >= 0;
+  roff[r] = off;
+#pragma unroll
+  for (int m = 0; m < (D * QPK + kTriThreads - 1) / kTriThreads; ++m) {  // [d][j] <- q_cal[g * QPK + j][d]
+    const int i = r + m * kTriThreads;
+    if (i < D * QPK) qs[i] = qv[m];
+  }
+  __syncthreads();
+  const uint8_t* kbase = reinterpret_cast<const uint8_t*>(k_pages);
 #pragma unroll 4
-      for (int c = 0; c < kChunks; ++c) {
-        const uint4 raw = *reinterpret_cast<const uint4*>(krow + c * 16);
-        const __nv_bfloat16* kv = reinterpret_cast<const __nv_bfloat16*>(&raw);
+  for (int i = threadIdx.x; i < nrows * kChunks; i += kTriThreads) {
+    const int rr = i / kChunks, c = i % kChunks;  // kChunks is a power of two
+    const long long o = roff[rr];
+    cp_async_16(ks + rr * kStride + c * 16, kbase + (o >= 0 ? o : 0) + c * 16, o >= 0 ? 16 : 0);
+  }
+  cp_async_commit();
+  cp_async_wait<0>();
+  __syncthreads();
+  const uint8_t* krow = ks + r * kStride;
+  float zv[QPK];
 #pragma unroll
-        for (int dd = 0; dd < 8; ++dd) acc = __fadd_rn(acc, __fmul_rn(qs[c * 8 + dd], __bfloat162float(kv[dd])));
-      }
-      zv[0] = acc;
-    } else {
-      constexpr int kPairs = QPK / 2;
-      unsigned long long acc[kPairs];
-#pragma unroll
-      for (int j = 0; j < kPairs; ++j) acc[j] = 0ull;  // (+0.0f, +0.0f)
+  for (int j = 0; j < QPK; ++j) zv[j] = 0.f;
 #pragma unroll 2
-      for (int c = 0; c < kChunks; ++c) {
-        const uint4 raw = *reinterpret_cast<const uint4*>(krow + c * 16);
-        const __nv_bfloat16* kv = reinterpret_cast<const __nv_bfloat16*>(&raw);
+  for (int c = 0; c < kChunks; ++c) {
+    const uint4 raw = *reinterpret_cast<const uint4*>(krow + c * 16);
+    const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
 #pragma unroll
-        for (int dd = 0; dd < 8; ++dd) {
-          const float kf = __bfloat162float(kv[dd]);
-          const unsigned long long kk = tri_pack(kf, kf);
-          unsigned long long qp[kPairs];
-          if constexpr (QPK == 2) {
-            qp[0] = *reinterpret_cast<const unsigned long long*>(qs + (c * 8 + dd) * QPK);
-          } else {
+    for (int dd = 0; dd < 8; ++dd) {
+      // bf16 -> fp32: the 16 bits become the high half
+      const float kf = __uint_as_float(dd & 1 ? (w[dd >> 1] & 0xffff0000u) : (w[dd >> 1] << 16));
+      const float* qd = qs + (c * 8 + dd) * QPK;
+      if constexpr (QPK % 4 == 0) {
 #pragma unroll
-            for (int v = 0; v < QPK / 4; ++v) {
-              const ulonglong2 q4 = *reinterpret_cast<const ulonglong2*>(qs + (c * 8 + dd) * QPK + 4 * v);
-              qp[2 * v] = q4.x;
-              qp[2 * v + 1] = q4.y;
-            }
-          }
-#pragma unroll
-          for (int j = 0; j < kPairs; ++j) acc[j] = tri_add2(acc[j], tri_mul2(qp[j], kk));
+        for (int v = 0; v < QPK / 4; ++v) {
+          const float4 q4 = *reinterpret_cast<const float4*>(qd + 4 * v);
+          zv[4 * v + 0] = __fmaf_rn(q4.x, kf, zv[4 * v + 0]);
+          zv[4 * v + 1] = __fmaf_rn(q4.y, kf, zv[4 * v + 1]);
+          zv[4 * v + 2] = __fmaf_rn(q4.z, kf, zv[4 * v + 2]);
+          zv[4 * v + 3] = __fmaf_rn(q4.w, kf, zv[4 * v + 3]);
         }
+      } else {
+#pragma unroll
+        for (int j = 0; j < QPK; ++j) zv[j] = __fmaf_rn(qd[j], kf, zv[j]);
       }
-#pragma unroll
-      for (int j = 0; j < kPairs; ++j) tri_unpack(acc[j], zv[2 * j], zv[2 * j + 1]);
-    }
-    // positions past the region and rows on a bad page count as -inf
-#pragma unroll
-    for (int j = 0; j < QPK; ++j) zv[j] = live ? zv[j] : -INFINITY;
-    if (in) {
-      float* zb = z + ((size_t)b * H + g * QPK) * e_max + p0 + r;
-#pragma unroll
-      for (int j = 0; j < QPK; ++j) zb[(size_t)j * e_max] = zv[j];
-    }
-    // this tile's maximum per query head, for the per-head shift
-#pragma unroll
-    for (int j = 0; j < QPK; ++j) {
-      float m = zv[j];
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-      if ((r & 31) == 0) sm.wmax[r >> 5][j] = m;
-    }
-    __syncthreads();
-    if (r < QPK) {
-      float m = sm.wmax[0][r];
-#pragma unroll
-      for (int w = 1; w < kTriThreads / 32; ++w) m = fmaxf(m, sm.wmax[w][r]);
-      tmax[((size_t)b * H + g * QPK + r) * n_tiles + p0 / kTriThreads] = m;
     }
   }
-  cp_async_wait<0>();  // no copy may outlive the CTA
+  // positions past the region and rows on a bad page count as -inf
+#pragma unroll
+  for (int j = 0; j < QPK; ++j) zv[j] = live ? zv[j] : -INFINITY;
+  if (in) {
+    float* zb = z + ((size_t)b * H + g * QPK) * e_max + p0 + r;
+#pragma unroll
+    for (int j = 0; j < QPK; ++j) zb[(size_t)j * e_max] = zv[j];
+  }
+  // this tile's maximum per query head, for the per-head shift
+#pragma unroll
+  for (int j = 0; j < QPK; ++j) {
+    float m = zv[j];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if ((r & 31) == 0) wmax[r >> 5][j] = m;
+  }
+  __syncthreads();
+  if (r < QPK) {
+    float m = wmax[0][r];
+#pragma unroll
+    for (int w = 1; w < kTriThreads / 32; ++w) m = fmaxf(m, wmax[w][r]);
+    const int n_tiles = (e_max + kTriTileTok - 1) / kTriTileTok;
+    tmax[((size_t)b * H + g * QPK + r) * n_tiles + blockIdx.x] = m;
+  }
 }
 
 constexpr int kTriReduceThreads = 256;
@@ -244,8 +195,8 @@ __global__ void __launch_bounds__(kTriReduceThreads) tri_reduce_kernel(
   if (blockIdx.x == 0 && threadIdx.x == 0 && (r % rows_per_req) == 0) evictable[b] = E;
   const int p0 = blockIdx.x * kTriReduceThreads;
   if (p0 >= E) return;
-  const int n_tiles = (e_max + kTriThreads - 1) / kTriThreads;
-  const int live_tiles = (E + kTriThreads - 1) / kTriThreads;
+  const int n_tiles = (e_max + kTriTileTok - 1) / kTriTileTok;
+  const int live_tiles = (E + kTriTileTok - 1) / kTriTileTok;
   const float* tb = tmax + ((size_t)b * H + h0) * n_tiles;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   for (int h = warp; h < nh; h += kTriReduceThreads / 32) {
@@ -309,7 +260,7 @@ __device__ __forceinline__ int tri_warp_search(int x, int n, int n_sink, int bud
 }
 
 constexpr int kTriCompactThreads = 256;
-constexpr int kTriChunkBytes = 32768;                 // K + V bytes of one unit
+constexpr int kTriChunkBytes = 32768;  // K + V bytes of one unit
 constexpr int kTriMaxChunkTokens = kTriChunkBytes / 128;
 constexpr uint32_t kTriWaitLimit = 1u << 22;
 
@@ -342,6 +293,7 @@ __global__ void __launch_bounds__(kTriCompactThreads) tri_compact_kernel(
   const int moved = budget + n_recent;
   const int pieces_per_part = part / 16;
   const int pieces_per_token = pieces_per_part * (v_pages ? 2 : 1);
+  const int step_i = kTriCompactThreads / pieces_per_token, step_w = kTriCompactThreads % pieces_per_token;
   const long long n_units = (long long)n_rows * n_chunks;
   for (long long u = blockIdx.x; u < n_units; u += gridDim.x) {
     const int r = static_cast<int>(u / n_chunks), c = static_cast<int>(u % n_chunks);
@@ -369,13 +321,23 @@ __global__ void __launch_bounds__(kTriCompactThreads) tri_compact_kernel(
       dst_off[i] = dof;
     }
     __syncthreads();
-    // 1. sources into shared memory
-    for (int pc = threadIdx.x; pc < nj * pieces_per_token; pc += kTriCompactThreads) {
-      const int i = pc / pieces_per_token, w = pc % pieces_per_token;
-      const long long so = src_off[i];
-      if (so < 0) continue;
-      const uint8_t* base = w < pieces_per_part ? k_pages : v_pages;
-      cp_async_16(buf + pc * 16, base + so + (w % pieces_per_part) * 16, 16);
+    // 1. sources into shared memory (piece pc = token i, piece w of the token;
+    // indices advance by carries, not by division)
+    {
+      int i = threadIdx.x / pieces_per_token, w = threadIdx.x % pieces_per_token;
+      for (int pc = threadIdx.x; pc < nj * pieces_per_token; pc += kTriCompactThreads) {
+        const long long so = src_off[i];
+        if (so >= 0) {
+          const bool kpart = w < pieces_per_part;
+          cp_async_16(buf + pc * 16, (kpart ? k_pages : v_pages) + so + (kpart ? w : w - pieces_per_part) * 16, 16);
+        }
+        w += step_w;
+        i += step_i;
+        if (w >= pieces_per_token) {
+          w -= pieces_per_token;
+          ++i;
+        }
+      }
     }
     cp_async_commit();
     // while the copies fly: the kept tokens whose sources lie in
@@ -417,13 +379,20 @@ __global__ void __launch_bounds__(kTriCompactThreads) tri_compact_kernel(
     __syncthreads();
     // 3. destinations
     if (wait_ok) {
+      int i = threadIdx.x / pieces_per_token, w = threadIdx.x % pieces_per_token;
       for (int pc = threadIdx.x; pc < nj * pieces_per_token; pc += kTriCompactThreads) {
-        const int i = pc / pieces_per_token, w = pc % pieces_per_token;
         const long long dof = dst_off[i];
-        if (dof < 0) continue;
-        uint8_t* base = w < pieces_per_part ? k_pages : v_pages;
-        *reinterpret_cast<uint4*>(base + dof + (w % pieces_per_part) * 16) =
-            *reinterpret_cast<const uint4*>(buf + pc * 16);
+        if (dof >= 0) {
+          const bool kpart = w < pieces_per_part;
+          *reinterpret_cast<uint4*>((kpart ? k_pages : v_pages) + dof + (kpart ? w : w - pieces_per_part) * 16) =
+              *reinterpret_cast<const uint4*>(buf + pc * 16);
+        }
+        w += step_w;
+        i += step_i;
+        if (w >= pieces_per_token) {
+          w -= pieces_per_token;
+          ++i;
+        }
       }
     }
     __syncthreads();  // buf and the offsets are reused by the next unit

@@ -282,7 +282,7 @@ class TriWorkload:
     spec: TriSpec
     seqlens: np.ndarray       # int32 [B]
     block_table: np.ndarray   # int32 [B, max_pages_per_req]
-    q_cal: np.ndarray         # fp32 [H, D]
+    q_cal: np.ndarray         # bf16 bits [H, D]
     k_pages: np.ndarray       # bf16 bits [num_pages, P, G, D]
     v_pages: Optional[np.ndarray]
 
@@ -314,7 +314,7 @@ def make_tri(s: TriSpec) -> TriWorkload:
         block_table[b, :n] = perm[cursor:cursor + n]
         cursor += n
     spare = perm[cursor:]
-    q_cal = rng.standard_normal((s.H, s.D), dtype=np.float32)
+    q_cal = bf16_bits_from_f32(rng.standard_normal((s.H, s.D), dtype=np.float32))
     k_pages = _normal_bf16(rng, (num_pages, P, s.G, s.D))
     v_pages = _normal_bf16(rng, (num_pages, P, s.G, s.D)) if s.with_v else None
     for b in range(B):

@@ -723,31 +723,41 @@ def bench_tri(args, rank, world, local):
     torch.cuda.set_device(local)
     base = W.tri_spec(args.tri)
     s = W.tri_spec(args.tri, seed=base.seed + 1000 * rank) if rank else base
-    w = W.make_tri(s)
-    mode = sd.TRI_PER_HEAD if args.tri_per_head else sd.TRI_UNION
+    n_layers = max(args.tri_layers, 1)
+    wls = W.make_tri_layers(s, n_layers)
+    w = wls[0]
+    mode = {"union": sd.TRI_UNION, "per_head": sd.TRI_PER_HEAD,
+            "per_layer_per_head": sd.TRI_PER_LAYER_PER_HEAD}[args.tri_mode]
     dev = "cuda"
     t = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(dev)  # noqa: E731
-    kp0 = t(w.k_pages.view(np.int16)).view(torch.bfloat16)
-    vp0 = t(w.v_pages.view(np.int16)).view(torch.bfloat16)
-    kp, vp = kp0.clone(), vp0.clone()
-    q_cal, bt, sl = t(w.q_cal), t(w.block_table), t(w.seqlens)
+    bf = lambda a: t(a.view(np.int16)).view(torch.bfloat16)  # noqa: E731
+    kp0 = [bf(x.k_pages) for x in wls]
+    vp0 = [bf(x.v_pages) for x in wls]
+    kp, vp = [x.clone() for x in kp0], [x.clone() for x in vp0]
+    q_cals = [bf(x.q_cal) for x in wls]
+    bt, sl = t(w.block_table), t(w.seqlens)
     B = int(w.seqlens.shape[0])
     lib = sd.load_library()
-    ws = torch.empty(int(lib.sd_tri_workspace_size(B, s.G, s.H, s.D, w.max_seqlen, s.n_sink, s.n_recent, s.budget,
-                                                     mode, 1)), dtype=torch.uint8, device=dev)
+    ws = torch.empty(int(lib.sd_tri_layers_workspace_size(n_layers, B, s.G, s.H, s.D, w.max_seqlen, s.n_sink,
+                                                            s.n_recent, s.budget, mode, 1)),
+                     dtype=torch.uint8, device=dev)
     nl = torch.empty((B,), dtype=torch.int32, device=dev)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     clean = torch.zeros(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
 
     def prepare():
-        kp.copy_(kp0)
-        vp.copy_(vp0)
+        for a, b in zip(kp + vp, kp0 + vp0):
+            a.copy_(b)
         flush.zero_()
         clean.max()
 
     def call():
-        sd.sd_tri_compact(q_cal, kp, vp, bt, sl, w.max_seqlen, s.n_sink, s.n_recent, s.budget, mode,
-                          new_seqlens=nl, workspace=ws)
+        if n_layers == 1:
+            sd.sd_tri_compact(q_cals[0], kp[0], vp[0], bt, sl, w.max_seqlen, s.n_sink, s.n_recent, s.budget, mode,
+                              new_seqlens=nl, workspace=ws)
+        else:
+            sd.sd_tri_compact_layers(q_cals, kp, vp, bt, sl, w.max_seqlen, s.n_sink, s.n_recent, s.budget, mode,
+                                     new_seqlens=nl, workspace=ws)
 
     side = torch.cuda.Stream()
     side.wait_stream(torch.cuda.current_stream())
@@ -775,17 +785,17 @@ def bench_tri(args, rank, world, local):
             tot += a.elapsed_time(b)
     del g
     ms = max_over_ranks(tot / args.steps, world)
-    nbytes = W.tri_algorithmic_bytes(s, w.seqlens, mode)
+    nbytes = n_layers * W.tri_algorithmic_bytes(s, w.seqlens, mode)
     peak, peak_kind = _peaks()
     achieved = nbytes / (ms * 1e-3) / 1e9
     line = {
-        "metric": "KV-cache eviction (score, select, compact one layer) requests/s, 1 B200",
+        "metric": "KV-cache eviction (score, select, compact every layer) requests/s, 1 B200",
         "value": world * B / (ms * 1e-3), "unit": "requests/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f32 scores, bf16 rows", "data": "synthetic",
         "config": {"workload": s.name, "B": B, "H": s.H, "kv_heads": s.G, "D": s.D, "page_size": s.page_size,
                    "n_sink": s.n_sink, "n_recent": s.n_recent, "budget": s.budget,
-                   "mode": "per_head" if mode else "union", "max_seqlen": w.max_seqlen,
+                   "mode": args.tri_mode, "layers": n_layers, "max_seqlen": w.max_seqlen,
                    "l2": "pools restored, then flushed (256 MiB write, 256 MiB read) before every step, "
                          "outside the timed events"},
         "gpu_launches": launches,
@@ -801,8 +811,12 @@ def bench_tri(args, rank, world, local):
         t0 = time.perf_counter()
         n = 0
         while n < B and (n == 0 or time.perf_counter() - t0 < 15.0):
-            T.tri_evict(w.q_cal, w.k_pages, w.v_pages, w.block_table[n:n + 1], w.seqlens[n:n + 1], s.n_sink,
-                        s.n_recent, s.budget, mode, inplace=True)
+            if n_layers == 1:
+                T.tri_evict(w.q_cal, w.k_pages, w.v_pages, w.block_table[n:n + 1], w.seqlens[n:n + 1], s.n_sink,
+                            s.n_recent, s.budget, mode, inplace=True)
+            else:
+                T.tri_evict_layers([x.q_cal for x in wls], [x.k_pages for x in wls], [x.v_pages for x in wls],
+                                   w.block_table[n:n + 1], w.seqlens[n:n + 1], s.n_sink, s.n_recent, s.budget, mode)
             n += 1
         el = time.perf_counter() - t0
         line["cpu_baseline"] = {"value": n / el, "unit": "requests/s", "cores": 1, "kind": "oracle",
@@ -828,7 +842,9 @@ def main():
                     help="time attention-only decode over this many layers sharing one selection instead")
     ap.add_argument("--tri", default="", choices=[""] + list(W.TRI_SPECS),
                     help="time one layer's KV-cache eviction (score, select, compact) on this workload instead")
-    ap.add_argument("--tri-per-head", action="store_true", help="with --tri: one selection per KV head")
+    ap.add_argument("--tri-mode", default="union", choices=["union", "per_head", "per_layer_per_head"],
+                    help="with --tri: one selection per request, per KV head, or per (layer, KV head)")
+    ap.add_argument("--tri-layers", type=int, default=1, help="with --tri: layers sharing the block table")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     rank, world, local = _dist_env()

@@ -137,7 +137,8 @@ sd_status sd_sparse_attn(const uint16_t* q, const uint16_t* k_pages, const uint1
  *   k_pages     bf16 [num_pages, P, G, D], compacted in place
  *   v_pages     bf16 [num_pages, P, G, D] compacted the same way, or NULL
  *   mode        SD_TRI_UNION: one selection per request (all KV heads move
- *               together); SD_TRI_PER_HEAD: one per (request, KV head)
+ *               together); SD_TRI_PER_HEAD (or SD_TRI_PER_LAYER_PER_HEAD):
+ *               one per (request, KV head)
  *   new_seqlens int32 [B] out: n_sink + budget + n_recent, or L_b when the
  *               evictable region holds at most `budget` tokens (nothing moves)
  * Score of evictable position p under query head h: z = q_cal[h] . K, one
@@ -157,12 +158,34 @@ sd_status sd_sparse_attn(const uint16_t* q, const uint16_t* k_pages, const uint1
  * unspecified, the pools outside its pages untouched). */
 #define SD_TRI_UNION 0
 #define SD_TRI_PER_HEAD 1
+#define SD_TRI_PER_LAYER_PER_HEAD 2 /* with one layer, the same as SD_TRI_PER_HEAD */
 size_t sd_tri_workspace_size(int32_t B, int32_t G, int32_t H, int32_t D, int32_t max_seqlen, int32_t n_sink,
                              int32_t n_recent, int32_t budget, int32_t mode, int32_t has_v);
 sd_status sd_tri_compact(const uint16_t* q_cal, uint16_t* k_pages, uint16_t* v_pages, const int32_t* block_table,
                          const int32_t* seqlens, sd_paged_desc pd, int32_t B, int32_t H, int32_t D, int32_t max_seqlen,
                          int32_t n_sink, int32_t n_recent, int32_t budget, int32_t mode, int32_t* new_seqlens,
                          void* workspace, size_t workspace_bytes, void* stream);
+
+/* The same over n_layers layers that share the block table and lengths
+ * ("Add TriAttention KV-cache compression method", Summary: union, per_head
+ * and per_layer_perhead eviction modes). q_cal, k_pages and v_pages are HOST
+ * arrays of n_layers device pointers (v_pages may be NULL: no V pools).
+ *   SD_TRI_UNION              one selection per request for every layer and
+ *                             head: score = max over layers and heads
+ *   SD_TRI_PER_HEAD           one selection per (request, KV head) for every
+ *                             layer: score = max over layers and that KV
+ *                             head's query heads
+ *   SD_TRI_PER_LAYER_PER_HEAD an independent per-head selection in each layer
+ * (each head's logits shifted by that layer's and head's maximum, as above).
+ * Every layer is compacted; new_seqlens holds the common new lengths.
+ * Workspace: sd_tri_layers_workspace_size(). Limits and errors as above. */
+size_t sd_tri_layers_workspace_size(int32_t n_layers, int32_t B, int32_t G, int32_t H, int32_t D, int32_t max_seqlen,
+                                    int32_t n_sink, int32_t n_recent, int32_t budget, int32_t mode, int32_t has_v);
+sd_status sd_tri_compact_layers(const uint16_t* const* q_cal, uint16_t* const* k_pages, uint16_t* const* v_pages,
+                                int32_t n_layers, const int32_t* block_table, const int32_t* seqlens, sd_paged_desc pd,
+                                int32_t B, int32_t H, int32_t D, int32_t max_seqlen, int32_t n_sink, int32_t n_recent,
+                                int32_t budget, int32_t mode, int32_t* new_seqlens, void* workspace,
+                                size_t workspace_bytes, void* stream);
 
 /* Steps 1 + 2, and the whole decode step, with the previous step's selection
  * as a hint: the "heuristic_prev_topk" feedback of "Overlap DSA heuristic

@@ -18,4 +18,5 @@ from .sd_oracle import (  # noqa: F401
 )
 from .tri_oracle import PER_HEAD as TRI_PER_HEAD  # noqa: F401
 from .tri_oracle import UNION as TRI_UNION  # noqa: F401
-from .tri_oracle import tri_compact, tri_evict, tri_logits, tri_scores, tri_select  # noqa: F401
+from .tri_oracle import PER_LAYER_PER_HEAD as TRI_PER_LAYER_PER_HEAD  # noqa: F401
+from .tri_oracle import tri_compact, tri_evict, tri_evict_layers, tri_logits, tri_scores, tri_select  # noqa: F401

@@ -50,6 +50,7 @@ from .sd_oracle import bf16_bits_to_f64, gather_token_rows
 
 UNION = 0
 PER_HEAD = 1
+PER_LAYER_PER_HEAD = 2
 
 
 def _evictable(L: int, n_sink: int, n_recent: int) -> int:
@@ -160,3 +161,33 @@ def tri_evict(q_cal, k_pages, v_pages, block_table, seqlens, n_sink: int, n_rece
     k, v, new_len = tri_compact(k_pages, v_pages, block_table, seqlens, selections, n_sink, n_recent, budget, mode,
                                 inplace)
     return k, v, new_len, selections
+
+
+def tri_evict_layers(q_cals, k_pools, v_pools, block_table, seqlens, n_sink: int, n_recent: int, budget: int,
+                     mode: int):
+    """Several layers sharing the block table ("Add TriAttention KV-cache
+    compression method", Summary: union, per_head and per_layer_perhead modes).
+    UNION / PER_HEAD: one selection for every layer, from the maximum over
+    layers of each layer's scores in that mode; PER_LAYER_PER_HEAD: each layer
+    evicted on its own, per head. Returns (k_pools, v_pools, new_seqlens,
+    selections); v_pools is None without V."""
+    n = len(k_pools)
+    if mode == PER_LAYER_PER_HEAD:
+        ks, vs, sels = [], [], []
+        for l in range(n):
+            k, v, nl, sel = tri_evict(q_cals[l], k_pools[l], None if v_pools is None else v_pools[l], block_table,
+                                      seqlens, n_sink, n_recent, budget, PER_HEAD)
+            ks.append(k)
+            vs.append(v)
+            sels.append(sel)
+        return ks, (None if v_pools is None else vs), nl, sels
+    per_layer = [tri_scores(q_cals[l], k_pools[l], block_table, seqlens, n_sink, n_recent, mode) for l in range(n)]
+    scores = [np.maximum.reduce([per_layer[l][b] for l in range(n)]) for b in range(len(seqlens))]
+    selections = [tri_select(sc, budget) for sc in scores]
+    ks, vs = [], []
+    for l in range(n):
+        k, v, nl = tri_compact(k_pools[l], None if v_pools is None else v_pools[l], block_table, seqlens, selections,
+                               n_sink, n_recent, budget, mode)
+        ks.append(k)
+        vs.append(v)
+    return ks, (None if v_pools is None else vs), nl, selections

@@ -112,7 +112,7 @@ def test_tri_compact_argument_errors(lib):
                                                               8, budget, mode, 256, 256 if nws else None, nws, None)
     assert f(*args(H=5)) == 1            # H not a multiple of G
     assert f(*args(budget=0)) == 1       # empty budget
-    assert f(*args(mode=2)) == 1         # unknown mode
+    assert f(*args(mode=3)) == 1         # unknown mode
     assert f(*args(D=96)) == 2           # head width
     assert f(*args(H=32)) == 2           # 16 query heads per KV head
     assert f(*args(budget=4096)) == 2    # above the top-k limit
@@ -122,4 +122,23 @@ def test_tri_compact_argument_errors(lib):
     a = ws(2, 2, 4, 64, 100, 4, 8, 24, 0, 0)
     assert ws(2, 2, 4, 64, 100, 4, 8, 24, 0, 1) >= a > 0
     assert ws(2, 2, 4, 64, 100, 4, 8, 48, 0, 0) > a
+    assert lib.sd_last_launch_count() == 0
+
+
+def test_tri_layers_argument_errors(lib):
+    desc = api.PagedDesc(64, 16, 8, 2)
+    f = lib.sd_tri_compact_layers
+    ptrs = (ctypes.c_void_p * 2)(256, 256)
+    holes = (ctypes.c_void_p * 2)(256, None)
+    arr = lambda a: ctypes.cast(a, ctypes.c_void_p)  # noqa: E731
+    args = lambda q, k, n, mode=0: (arr(q), arr(k), None, n, 256, 256, desc, 2, 4, 64, 100, 4, 8, 24, mode,  # noqa: E731
+                                    256, None, 0, None)
+    assert f(*args(ptrs, ptrs, 0)) == 1          # no layers
+    assert f(*args(ptrs, holes, 2)) == 1         # a NULL pool
+    assert f(*args(ptrs, ptrs, 2, mode=3)) == 1  # unknown mode
+    assert f(*args(ptrs, ptrs, 2)) == 3          # no workspace
+    one = lib.sd_tri_layers_workspace_size(1, 2, 2, 4, 64, 100, 4, 8, 24, 0, 1)
+    assert one == lib.sd_tri_workspace_size(2, 2, 4, 64, 100, 4, 8, 24, 0, 1)
+    assert lib.sd_tri_layers_workspace_size(4, 64, 2, 4, 64, 5000, 4, 8, 2048, 0, 1) > \
+        lib.sd_tri_layers_workspace_size(1, 64, 2, 4, 64, 5000, 4, 8, 2048, 0, 1)  # a flag set per layer
     assert lib.sd_last_launch_count() == 0

@@ -142,3 +142,45 @@ def test_full_size_sampled_requests():
         assert nl_ref[0] == nl[b]
         assert np.array_equal(k[pages], k_ref[pages])
         assert np.array_equal(v[pages], v_ref[pages])
+
+
+@pytest.mark.parametrize("mode", [T.UNION, T.PER_HEAD, T.PER_LAYER_PER_HEAD])
+@pytest.mark.parametrize("with_v", [True, False])
+def test_layers_every_mode(mode, with_v):
+    """Three layers sharing the block table ("Add TriAttention KV-cache
+    compression method", Summary: union / per_head / per_layer_perhead): one
+    selection across layers, or one per layer, every layer compacted."""
+    import torch
+    import top_sparse_decode_paged_b200 as sd
+    from top_sparse_decode_paged_b200.workloads import make_tri_layers
+    s = tri_spec("tri_ragged_b16", B=4, page_size=16, n_sink=24, n_recent=7, budget=150, ragged=(0, 600),
+                 with_v=with_v, seed=41 + mode)
+    ws = make_tri_layers(s, 3)
+    k_ref, v_ref, nl_ref, _ = T.tri_evict_layers([w.q_cal for w in ws], [w.k_pages for w in ws],
+                                                 None if not with_v else [w.v_pages for w in ws], ws[0].block_table,
+                                                 ws[0].seqlens, s.n_sink, s.n_recent, s.budget, mode)
+    kps = [_bf16(w.k_pages) for w in ws]
+    vps = None if not with_v else [_bf16(w.v_pages) for w in ws]
+    nl = sd.sd_tri_compact_layers([_bf16(w.q_cal) for w in ws], kps, vps, _dev(ws[0].block_table),
+                                  _dev(ws[0].seqlens), ws[0].max_seqlen, s.n_sink, s.n_recent, s.budget, mode)
+    torch.cuda.synchronize()
+    assert sd.device_errors() == 0
+    assert np.array_equal(nl.cpu().numpy(), nl_ref)
+    for l in range(3):
+        assert np.array_equal(_bits(kps[l]), k_ref[l])
+        if with_v:
+            assert np.array_equal(_bits(vps[l]), v_ref[l])
+
+
+def test_layers_one_layer_matches_single_call():
+    import torch
+    import top_sparse_decode_paged_b200 as sd
+    w = make_tri(tri_spec("tri_tiny"))
+    s = w.spec
+    a, b = _bf16(w.k_pages), _bf16(w.k_pages)
+    sd.sd_tri_compact(_dev(w.q_cal), a, None, _dev(w.block_table), _dev(w.seqlens), w.max_seqlen, s.n_sink,
+                      s.n_recent, s.budget, T.PER_HEAD)
+    sd.sd_tri_compact_layers([_dev(w.q_cal)], [b], None, _dev(w.block_table), _dev(w.seqlens), w.max_seqlen,
+                             s.n_sink, s.n_recent, s.budget, T.PER_LAYER_PER_HEAD)
+    torch.cuda.synchronize()
+    assert torch.equal(a.view(torch.int16), b.view(torch.int16))

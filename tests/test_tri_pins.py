@@ -203,3 +203,39 @@ def test_compaction_brute_force_tiny():
         got = [float((np.uint32(k2[bt[i // P], i % P, 0, 0]) << 16).view(np.float32)) for i in range(L)]
         assert got[:7] == [0] + [1 + s for s in sub] + [7, 8, 9]
         assert got[7:] == [7, 8, 9]
+
+
+def test_layers_identical_layers_select_as_one():
+    """Two copies of one layer: the union and per-head selections across
+    layers equal the single layer's (the maximum of equal scores)."""
+    w = make_tri(tri_spec("tri_tiny"))
+    s = w.spec
+    for mode in (T.UNION, T.PER_HEAD):
+        _, _, nl1, sel1 = T.tri_evict(w.q_cal, w.k_pages, w.v_pages, w.block_table, w.seqlens, s.n_sink,
+                                      s.n_recent, s.budget, mode)
+        _, _, nl2, sel2 = T.tri_evict_layers([w.q_cal] * 2, [w.k_pages] * 2, [w.v_pages] * 2, w.block_table,
+                                             w.seqlens, s.n_sink, s.n_recent, s.budget, mode)
+        assert np.array_equal(nl1, nl2)
+        for a, b in zip(sel1, sel2):
+            assert np.array_equal(a, b)
+
+
+def test_layers_union_keeps_each_layers_favourite():
+    """Layer 0's query picks one key column, layer 1's another; with a budget
+    of 2 the cross-layer union keeps each layer's best position (score 0, the
+    maximum), and per-layer-per-head keeps each layer's own top 2."""
+    E, D = 12, 64
+    vals = np.zeros((E, 1, D), dtype=np.float32)
+    vals[:, 0, 0] = [1, 9, 2, 3, 1, 2, 0, 1, 2, 1, 0, 8]   # layer 0 prefers 1, then 11
+    vals[:, 0, 1] = [0, 1, 2, 3, 4, 7, 2, 11, 1, 1, 6, 1]  # layer 1 prefers 7, then 5
+    pool, bt = _pool_from_values(bf16_bits_from_f32(vals), P=4)
+    q0 = np.zeros((1, D), np.float32)
+    q0[0, 0] = 1.0
+    q1 = np.zeros((1, D), np.float32)
+    q1[0, 1] = 1.0
+    qs = [bf16_bits_from_f32(q0), bf16_bits_from_f32(q1)]
+    _, _, _, sel = T.tri_evict_layers(qs, [pool, pool], None, bt[None], np.array([E]), 0, 0, 2, T.UNION)
+    assert sel[0].tolist() == [[1, 7]]
+    _, _, _, sels = T.tri_evict_layers(qs, [pool, pool], None, bt[None], np.array([E]), 0, 0, 2,
+                                       T.PER_LAYER_PER_HEAD)
+    assert sels[0][0].tolist() == [[1, 11]] and sels[1][0].tolist() == [[5, 7]]

@@ -12,6 +12,7 @@ from .api import (  # noqa: F401
     SD_DEVERR_SEQLEN,
     SdError,
     TRI_PER_HEAD,
+    TRI_PER_LAYER_PER_HEAD,
     TRI_UNION,
     StageTimer,
     alloc_workspace,
@@ -27,11 +28,13 @@ from .api import (  # noqa: F401
     sd_sparse_attn_csr,
     sd_sparse_attn_layers,
     sd_tri_compact,
+    sd_tri_compact_layers,
     workspace_size,
 )
 
 __all__ = [
     "sd_indexer_topk", "sd_indexer_topk_hinted", "sd_indexer_topk_noalloc", "sd_decode_step_hinted", "sd_sparse_attn", "sd_sparse_attn_layers", "sd_sparse_attn_csr",
-    "sd_decode_step", "sd_tri_compact", "TRI_UNION", "TRI_PER_HEAD",
+    "sd_decode_step", "sd_tri_compact", "sd_tri_compact_layers", "TRI_UNION", "TRI_PER_HEAD",
+    "TRI_PER_LAYER_PER_HEAD",
     "workspace_size", "alloc_workspace", "device_errors", "load_library", "SdError", "StageTimer",
 ]

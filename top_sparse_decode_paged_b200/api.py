@@ -24,7 +24,8 @@ SD_DEVERR_INDEX = 0x4
 EXPORTED = ("sd_workspace_size", "sd_indexer_topk", "sd_indexer_topk_noalloc", "sd_sparse_attn",
             "sd_attn_layers_workspace_size", "sd_sparse_attn_layers", "sd_csr_workspace_size",
             "sd_sparse_attn_csr", "sd_indexer_topk_hinted", "sd_decode_step_hinted", "sd_decode_step",
-            "sd_tri_workspace_size", "sd_tri_compact", "sd_set_stage_events", "sd_get_device_errors", "sd_status_str", "sd_last_cuda_error",
+            "sd_tri_workspace_size", "sd_tri_compact", "sd_tri_layers_workspace_size", "sd_tri_compact_layers",
+            "sd_set_stage_events", "sd_get_device_errors", "sd_status_str", "sd_last_cuda_error",
             "sd_last_launch_count", "sd_version")
 
 
@@ -85,6 +86,11 @@ def load_library(path: str = LIB_PATH):
     lib.sd_tri_workspace_size.argtypes = [i32] * 10
     lib.sd_tri_compact.restype = i32
     lib.sd_tri_compact.argtypes = [p, p, p, p, p, PagedDesc, i32, i32, i32, i32, i32, i32, i32, i32, p, p, sz, p]
+    lib.sd_tri_layers_workspace_size.restype = sz
+    lib.sd_tri_layers_workspace_size.argtypes = [i32] * 11
+    lib.sd_tri_compact_layers.restype = i32
+    lib.sd_tri_compact_layers.argtypes = [p, p, p, i32, p, p, PagedDesc, i32, i32, i32, i32, i32, i32, i32, i32, p, p,
+                                          sz, p]
     lib.sd_set_stage_events.restype = i32
     lib.sd_set_stage_events.argtypes = [ctypes.POINTER(ctypes.c_void_p), i32]
     lib.sd_get_device_errors.restype = i32
@@ -318,6 +324,7 @@ def sd_decode_step(qi, w, ki_pages, q, k_pages, v_pages, block_table, seqlens, k
 
 TRI_UNION = 0
 TRI_PER_HEAD = 1
+TRI_PER_LAYER_PER_HEAD = 2
 
 
 def sd_tri_compact(q_cal, k_pages, v_pages, block_table, seqlens, max_seqlen: int, n_sink: int, n_recent: int,
@@ -342,6 +349,40 @@ def sd_tri_compact(q_cal, k_pages, v_pages, block_table, seqlens, max_seqlen: in
                               _desc(k_pages, block_table), B, H, D, int(max_seqlen), int(n_sink), int(n_recent),
                               int(budget), int(mode), _ptr(new_seqlens), _ptr(workspace), workspace.numel(),
                               _stream(stream)))
+    return new_seqlens
+
+
+def sd_tri_compact_layers(q_cals, k_pools, v_pools, block_table, seqlens, max_seqlen: int, n_sink: int,
+                          n_recent: int, budget: int, mode: int = TRI_UNION, new_seqlens=None, workspace=None,
+                          stream=None):
+    """Eviction over several layers sharing the block table: ``q_cals``,
+    ``k_pools`` (and ``v_pools``) are per-layer lists; ``mode`` is TRI_UNION,
+    TRI_PER_HEAD (one selection for all layers) or TRI_PER_LAYER_PER_HEAD.
+    Compacts every layer in place; returns ``new_seqlens`` [B] int32."""
+    lib = load_library()
+    qs = [_bits(q) for q in q_cals]
+    ks = [_bits(k) for k in k_pools]
+    vs = None if v_pools is None else [_bits(v) for v in v_pools]
+    L = len(ks)
+    if len(qs) != L or (vs is not None and len(vs) != L):
+        raise ValueError("q_cals, k_pools and v_pools need one entry per layer")
+    H, D = qs[0].shape
+    G = ks[0].shape[2]
+    B = seqlens.shape[0]
+    if new_seqlens is None:
+        new_seqlens = torch.empty((B,), dtype=torch.int32, device=ks[0].device)
+    if workspace is None:
+        nbytes = int(lib.sd_tri_layers_workspace_size(L, B, G, H, D, max_seqlen, n_sink, n_recent, budget, mode,
+                                                      1 if vs is not None else 0))
+        workspace = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=ks[0].device)
+    qarr = (ctypes.c_void_p * L)(*[_ptr(t) for t in qs])
+    karr = (ctypes.c_void_p * L)(*[_ptr(t) for t in ks])
+    varr = None if vs is None else (ctypes.c_void_p * L)(*[_ptr(t) for t in vs])
+    _check(lib.sd_tri_compact_layers(ctypes.cast(qarr, ctypes.c_void_p), ctypes.cast(karr, ctypes.c_void_p),
+                                     None if varr is None else ctypes.cast(varr, ctypes.c_void_p), L,
+                                     _ptr(block_table), _ptr(seqlens), _desc(ks[0], block_table), B, H, D,
+                                     int(max_seqlen), int(n_sink), int(n_recent), int(budget), int(mode),
+                                     _ptr(new_seqlens), _ptr(workspace), workspace.numel(), _stream(stream)))
     return new_seqlens
 
 

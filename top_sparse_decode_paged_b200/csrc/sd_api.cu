@@ -560,30 +560,33 @@ sd_status sd_sparse_attn_csr(const uint16_t* q, const uint16_t* k_pages, const u
 namespace {
 struct TriPlan {
   int rows_per_req, e_max, moved, part, n_tiles, chunk, n_chunks;
-  size_t off_tmax, off_keys, off_evict, off_sel, off_flags, total;
+  size_t off_tmax, off_keys, off_evict, off_sel, off_flags, flags_per_layer, total;
 };
-TriPlan tri_plan(int B, int G, int H, int D, int max_seqlen, int n_sink, int n_recent, int budget, int mode,
-                 bool has_v) {
+TriPlan tri_plan(int n_layers, int B, int G, int H, int D, int max_seqlen, int n_sink, int n_recent, int budget,
+                 int mode, bool has_v) {
   TriPlan p{};
-  p.rows_per_req = mode == SD_TRI_PER_HEAD ? G : 1;
+  p.rows_per_req = mode == SD_TRI_UNION ? 1 : G;
   p.e_max = std::max(0, max_seqlen - n_sink - n_recent);
   p.moved = budget + n_recent;
-  p.part = (mode == SD_TRI_PER_HEAD ? 1 : G) * D * 2;
+  p.part = (mode == SD_TRI_UNION ? G : 1) * D * 2;
   p.n_tiles = (p.e_max + sd::kTriTileTok - 1) / sd::kTriTileTok;
   p.chunk = std::max(1, std::min(sd::kTriMaxChunkTokens, sd::kTriChunkBytes / (p.part * (has_v ? 2 : 1))));
   p.n_chunks = (p.moved + p.chunk - 1) / p.chunk;
   const size_t rows = (size_t)B * p.rows_per_req;
+  p.flags_per_layer = rows * p.n_chunks;
   p.off_tmax = align_up((size_t)B * H * p.e_max * sizeof(float));
   p.off_keys = p.off_tmax + align_up((size_t)B * H * p.n_tiles * sizeof(float));
   p.off_evict = p.off_keys + align_up(rows * p.e_max * sizeof(int32_t));
   p.off_sel = p.off_evict + align_up((size_t)B * sizeof(int32_t));
   p.off_flags = p.off_sel + align_up(rows * budget * sizeof(int32_t));
-  p.total = p.off_flags + align_up(rows * p.n_chunks * sizeof(int32_t));
+  p.total = p.off_flags + align_up((size_t)n_layers * p.flags_per_layer * sizeof(int32_t));
   return p;
 }
-bool tri_args_ok(int B, int G, int H, int D, int max_seqlen, int n_sink, int n_recent, int budget, int mode) {
-  return B >= 0 && G > 0 && H > 0 && H % G == 0 && max_seqlen >= 0 && n_sink >= 0 && n_recent >= 0 && budget >= 1 &&
-         (mode == SD_TRI_UNION || mode == SD_TRI_PER_HEAD);
+bool tri_args_ok(int n_layers, int B, int G, int H, int D, int max_seqlen, int n_sink, int n_recent, int budget,
+                 int mode) {
+  return n_layers >= 1 && B >= 0 && G > 0 && H > 0 && H % G == 0 && max_seqlen >= 0 && n_sink >= 0 &&
+         n_recent >= 0 && budget >= 1 &&
+         (mode == SD_TRI_UNION || mode == SD_TRI_PER_HEAD || mode == SD_TRI_PER_LAYER_PER_HEAD);
 }
 // Co-resident CTAs of the compaction kernel on this device (its units wait on
 // one another, so every CTA of its grid must be resident at once).
@@ -610,61 +613,41 @@ sd_status launch_tri_score(const uint16_t* q_cal, const uint16_t* kp, const int3
                   seqlens, H, pd.kv_heads, pd.page_size, pd.max_pages_per_req, pd.num_pages, cap, n_sink, n_recent,
                   e_max, z, tmax);
 }
-}  // namespace
 
-extern "C" {
-
-size_t sd_tri_workspace_size(int32_t B, int32_t G, int32_t H, int32_t D, int32_t max_seqlen, int32_t n_sink,
-                             int32_t n_recent, int32_t budget, int32_t mode, int32_t has_v) {
-  if (!tri_args_ok(B, G, H, D, max_seqlen, n_sink, n_recent, budget, mode)) return 0;
-  return tri_plan(B, G, H, D, max_seqlen, n_sink, n_recent, budget, mode, has_v != 0).total;
-}
-
-sd_status sd_tri_compact(const uint16_t* q_cal, uint16_t* k_pages, uint16_t* v_pages, const int32_t* block_table,
-                         const int32_t* seqlens, sd_paged_desc pd, int32_t B, int32_t H, int32_t D, int32_t max_seqlen,
-                         int32_t n_sink, int32_t n_recent, int32_t budget, int32_t mode, int32_t* new_seqlens,
-                         void* workspace, size_t workspace_bytes, void* stream) {
-  t_launches = 0;
-  if (!q_cal || !k_pages || !geom_ok(pd) || (B > 0 && (!block_table || !seqlens || !new_seqlens)))
-    return SD_ERR_INVALID_ARG;
-  const int G = pd.kv_heads;
-  if (!tri_args_ok(B, G, H, D, max_seqlen, n_sink, n_recent, budget, mode)) return SD_ERR_INVALID_ARG;
-  const int qpk = H / G;
-  if ((D != 64 && D != 128) || (qpk != 1 && qpk != 2 && qpk != 4 && qpk != 8) || budget > kMaxK)
-    return SD_ERR_UNSUPPORTED;
-  // grid y of the score and reduce passes; heads of the reduce
-  if ((long long)B * G > 65535 || H > sd::kTriMaxHeads) return SD_ERR_UNSUPPORTED;
-  const bool has_v = v_pages != nullptr;
-  if ((mode == SD_TRI_PER_HEAD ? 1 : G) * D * 2 * (has_v ? 2 : 1) > sd::kTriChunkBytes) return SD_ERR_UNSUPPORTED;
-  const TriPlan p = tri_plan(B, G, H, D, max_seqlen, n_sink, n_recent, budget, mode, has_v);
-  if (!ws_ok(workspace, workspace_bytes, p.total)) return SD_ERR_WORKSPACE;
-  if (B == 0) return SD_OK;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  char* ws = static_cast<char*>(workspace);
+// One selection from the scores of layers [l0, l0 + nl) (folded by maximum),
+// then every one of those layers compacted with it.
+sd_status tri_select_compact(const uint16_t* const* q_cal, uint16_t* const* k_pages, uint16_t* const* v_pages, int l0,
+                             int nl, const int32_t* block_table, const int32_t* seqlens, const sd_paged_desc& pd, int B,
+                             int H, int D, int cap, int n_sink, int n_recent, int budget, int mode, const TriPlan& p,
+                             int32_t* new_seqlens, char* ws, cudaStream_t st) {
+  const int G = pd.kv_heads, qpk = H / G;
   float* z = reinterpret_cast<float*>(ws);
   float* tmax = reinterpret_cast<float*>(ws + p.off_tmax);
   int32_t* keys = reinterpret_cast<int32_t*>(ws + p.off_keys);
   int32_t* evict = reinterpret_cast<int32_t*>(ws + p.off_evict);
   int32_t* sel = reinterpret_cast<int32_t*>(ws + p.off_sel);
   int32_t* flags = reinterpret_cast<int32_t*>(ws + p.off_flags);
-  const int cap = std::min(max_seqlen, pd.max_pages_per_req * pd.page_size);
   const int rows = B * p.rows_per_req;
   sd_status s = SD_OK;
   if (p.e_max > 0) {
-#define SD_TRI(D_, Q_) \
-  s = launch_tri_score<D_, Q_>(q_cal, k_pages, block_table, seqlens, pd, B, H, cap, n_sink, n_recent, p.e_max, z, tmax, st)
-    if (D == 64) {
-      if (qpk == 1) SD_TRI(64, 1); else if (qpk == 2) SD_TRI(64, 2); else if (qpk == 4) SD_TRI(64, 4); else SD_TRI(64, 8);
-    } else {
-      if (qpk == 1) SD_TRI(128, 1); else if (qpk == 2) SD_TRI(128, 2); else if (qpk == 4) SD_TRI(128, 4); else SD_TRI(128, 8);
-    }
+    for (int l = l0; l < l0 + nl; ++l) {
+#define SD_TRI(D_, Q_)                                                                                            \
+  s = launch_tri_score<D_, Q_>(q_cal[l], k_pages[l], block_table, seqlens, pd, B, H, cap, n_sink, n_recent, p.e_max, z, \
+                               tmax, st)
+      if (D == 64) {
+        if (qpk == 1) SD_TRI(64, 1); else if (qpk == 2) SD_TRI(64, 2); else if (qpk == 4) SD_TRI(64, 4); else SD_TRI(64, 8);
+      } else {
+        if (qpk == 1) SD_TRI(128, 1); else if (qpk == 2) SD_TRI(128, 2); else if (qpk == 4) SD_TRI(128, 4); else SD_TRI(128, 8);
+      }
 #undef SD_TRI
-    if (s != SD_OK) return s;
-    const dim3 rgrid((unsigned)((p.e_max + sd::kTriReduceThreads - 1) / sd::kTriReduceThreads), (unsigned)rows);
-    if ((s = launch_k(sd::tri_reduce_kernel, rgrid, dim3(sd::kTriReduceThreads), 0, st, static_cast<const float*>(z),
-                      static_cast<const float*>(tmax), seqlens, H, G, p.rows_per_req, cap, n_sink, n_recent, p.e_max,
-                      keys, evict, flags, p.n_chunks)) != SD_OK)
-      return s;
+      if (s != SD_OK) return s;
+      const dim3 rgrid((unsigned)((p.e_max + sd::kTriReduceThreads - 1) / sd::kTriReduceThreads), (unsigned)rows);
+      if ((s = launch_k(sd::tri_reduce_kernel, rgrid, dim3(sd::kTriReduceThreads), 0, st, static_cast<const float*>(z),
+                        static_cast<const float*>(tmax), seqlens, H, G, p.rows_per_req, cap, n_sink, n_recent,
+                        p.e_max, keys, evict, flags + (size_t)l * p.flags_per_layer, p.n_chunks, l > l0 ? 1 : 0)) !=
+          SD_OK)
+        return s;
+    }
     if ((s = launch_topk(keys, evict, sel, B, p.rows_per_req, p.e_max, p.e_max, budget, sd::RowMap{}, nullptr, st)) !=
         SD_OK)
       return s;
@@ -672,11 +655,78 @@ sd_status sd_tri_compact(const uint16_t* q_cal, uint16_t* k_pages, uint16_t* v_p
   const int grid = tri_compact_grid();
   if (grid <= 0) return cuda_check(cudaGetLastError());
   const long long units = (long long)rows * p.n_chunks;
-  return launch_k(sd::tri_compact_kernel, dim3((unsigned)std::max(1LL, std::min<long long>(grid, units))),
-                  dim3(sd::kTriCompactThreads), 0, st, reinterpret_cast<uint8_t*>(k_pages),
-                  reinterpret_cast<uint8_t*>(v_pages), block_table, seqlens, static_cast<const int32_t*>(sel),
-                  p.rows_per_req, pd.page_size, pd.max_pages_per_req, pd.num_pages, cap, n_sink, n_recent, budget,
-                  p.part, G * D * 2, p.chunk, p.n_chunks, rows, flags, new_seqlens);
+  for (int l = l0; l < l0 + nl; ++l) {
+    if ((s = launch_k(sd::tri_compact_kernel, dim3((unsigned)std::max(1LL, std::min<long long>(grid, units))),
+                      dim3(sd::kTriCompactThreads), 0, st, reinterpret_cast<uint8_t*>(k_pages[l]),
+                      reinterpret_cast<uint8_t*>(v_pages ? v_pages[l] : nullptr), block_table, seqlens,
+                      static_cast<const int32_t*>(sel), p.rows_per_req, pd.page_size, pd.max_pages_per_req,
+                      pd.num_pages, cap, n_sink, n_recent, budget, p.part, G * D * 2, p.chunk, p.n_chunks, rows,
+                      flags + (size_t)l * p.flags_per_layer, new_seqlens)) != SD_OK)
+      return s;
+  }
+  return SD_OK;
+}
+}  // namespace
+
+extern "C" {
+
+size_t sd_tri_layers_workspace_size(int32_t n_layers, int32_t B, int32_t G, int32_t H, int32_t D, int32_t max_seqlen,
+                                    int32_t n_sink, int32_t n_recent, int32_t budget, int32_t mode, int32_t has_v) {
+  if (!tri_args_ok(n_layers, B, G, H, D, max_seqlen, n_sink, n_recent, budget, mode)) return 0;
+  return tri_plan(n_layers, B, G, H, D, max_seqlen, n_sink, n_recent, budget, mode, has_v != 0).total;
+}
+
+size_t sd_tri_workspace_size(int32_t B, int32_t G, int32_t H, int32_t D, int32_t max_seqlen, int32_t n_sink,
+                             int32_t n_recent, int32_t budget, int32_t mode, int32_t has_v) {
+  return sd_tri_layers_workspace_size(1, B, G, H, D, max_seqlen, n_sink, n_recent, budget, mode, has_v);
+}
+
+sd_status sd_tri_compact_layers(const uint16_t* const* q_cal, uint16_t* const* k_pages, uint16_t* const* v_pages,
+                                int32_t n_layers, const int32_t* block_table, const int32_t* seqlens, sd_paged_desc pd,
+                                int32_t B, int32_t H, int32_t D, int32_t max_seqlen, int32_t n_sink, int32_t n_recent,
+                                int32_t budget, int32_t mode, int32_t* new_seqlens, void* workspace,
+                                size_t workspace_bytes, void* stream) {
+  t_launches = 0;
+  if (n_layers < 1 || !q_cal || !k_pages || !geom_ok(pd) || (B > 0 && (!block_table || !seqlens || !new_seqlens)))
+    return SD_ERR_INVALID_ARG;
+  for (int l = 0; l < n_layers; ++l)
+    if (!q_cal[l] || !k_pages[l] || (v_pages && !v_pages[l])) return SD_ERR_INVALID_ARG;
+  const int G = pd.kv_heads;
+  if (!tri_args_ok(n_layers, B, G, H, D, max_seqlen, n_sink, n_recent, budget, mode)) return SD_ERR_INVALID_ARG;
+  const int qpk = H / G;
+  if ((D != 64 && D != 128) || (qpk != 1 && qpk != 2 && qpk != 4 && qpk != 8) || budget > kMaxK)
+    return SD_ERR_UNSUPPORTED;
+  // grid y of the score and reduce passes; heads of the reduce
+  if ((long long)B * G > 65535 || H > sd::kTriMaxHeads) return SD_ERR_UNSUPPORTED;
+  const bool has_v = v_pages != nullptr;
+  if ((mode == SD_TRI_UNION ? G : 1) * D * 2 * (has_v ? 2 : 1) > sd::kTriChunkBytes) return SD_ERR_UNSUPPORTED;
+  const TriPlan p = tri_plan(n_layers, B, G, H, D, max_seqlen, n_sink, n_recent, budget, mode, has_v);
+  if (!ws_ok(workspace, workspace_bytes, p.total)) return SD_ERR_WORKSPACE;
+  if (B == 0) return SD_OK;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  char* ws = static_cast<char*>(workspace);
+  const int cap = std::min(max_seqlen, pd.max_pages_per_req * pd.page_size);
+  if (mode == SD_TRI_PER_LAYER_PER_HEAD) {  // an independent per-head selection in every layer
+    for (int l = 0; l < n_layers; ++l) {
+      const sd_status s = tri_select_compact(q_cal, k_pages, v_pages, l, 1, block_table, seqlens, pd, B, H, D, cap,
+                                             n_sink, n_recent, budget, mode, p, new_seqlens, ws, st);
+      if (s != SD_OK) return s;
+    }
+    return SD_OK;
+  }
+  return tri_select_compact(q_cal, k_pages, v_pages, 0, n_layers, block_table, seqlens, pd, B, H, D, cap, n_sink,
+                            n_recent, budget, mode, p, new_seqlens, ws, st);
+}
+
+sd_status sd_tri_compact(const uint16_t* q_cal, uint16_t* k_pages, uint16_t* v_pages, const int32_t* block_table,
+                         const int32_t* seqlens, sd_paged_desc pd, int32_t B, int32_t H, int32_t D, int32_t max_seqlen,
+                         int32_t n_sink, int32_t n_recent, int32_t budget, int32_t mode, int32_t* new_seqlens,
+                         void* workspace, size_t workspace_bytes, void* stream) {
+  const uint16_t* q1[1] = {q_cal};
+  uint16_t* k1[1] = {k_pages};
+  uint16_t* v1[1] = {v_pages};
+  return sd_tri_compact_layers(q1, k1, v_pages ? v1 : nullptr, 1, block_table, seqlens, pd, B, H, D, max_seqlen,
+                               n_sink, n_recent, budget, mode, new_seqlens, workspace, workspace_bytes, stream);
 }
 
 sd_status sd_decode_step_hinted(const int8_t* qi, const int32_t* w, const int8_t* ki_pages, const uint16_t* q,

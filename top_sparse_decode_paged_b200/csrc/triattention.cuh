@@ -174,12 +174,13 @@ constexpr int kTriMaxHeads = 256;
 
 // Selection keys: one block per (256 positions, selection row). The per-head
 // maxima come from the score tiles' maxima (one warp per head); a row's score
-// at p is the maximum over its heads of z - m. Also zeroes the row's
-// compaction flags.
+// at p is the maximum over its heads of z - m, or, with `accumulate` (a later
+// layer of a cross-layer selection), the maximum of that and the key already
+// there. Also zeroes the row's compaction flags.
 __global__ void __launch_bounds__(kTriReduceThreads) tri_reduce_kernel(
     const float* __restrict__ z, const float* __restrict__ tmax, const int32_t* __restrict__ seqlens, int H, int G,
     int rows_per_req, int seqlen_cap, int n_sink, int n_recent, int e_max, int32_t* __restrict__ keys,
-    int32_t* __restrict__ evictable, int32_t* __restrict__ flags, int n_chunks) {
+    int32_t* __restrict__ evictable, int32_t* __restrict__ flags, int n_chunks, int accumulate) {
   pdl_wait();
   pdl_trigger();
   __shared__ float m_s[kTriMaxHeads];
@@ -222,7 +223,9 @@ __global__ void __launch_bounds__(kTriReduceThreads) tri_reduce_kernel(
   }
   for (; h < nh; ++h)
     if (m_s[h] != -INFINITY) s = fmaxf(s, __fsub_rn(zb[(size_t)h * e_max], m_s[h]));
-  keys[(size_t)r * e_max + p] = tri_key(s);
+  int32_t* kp = keys + (size_t)r * e_max + p;
+  const int32_t key = tri_key(s);
+  *kp = accumulate ? max(*kp, key) : key;  // the key order is the score order
 }
 
 // Source of kept token j (0-based after the prefix) of a request.

@@ -331,6 +331,28 @@ def make_tri(s: TriSpec) -> TriWorkload:
                        v_pages=v_pages)
 
 
+def make_tri_layers(s: TriSpec, n_layers: int):
+    """n_layers layers of one eviction batch: layer 0 is make_tri(s); each later
+    layer draws its own q_cal, K pool and V pool (in that order, from one
+    generator seeded seed + 7919) with the same lengths, block table and
+    poison."""
+    base = make_tri(s)
+    out = [base]
+    rng = np.random.default_rng(s.seed + 7919)
+    shape = base.k_pages.shape
+    for _ in range(1, n_layers):
+        q_cal = bf16_bits_from_f32(rng.standard_normal((s.H, s.D), dtype=np.float32))
+        k = _normal_bf16(rng, shape)
+        v = _normal_bf16(rng, shape) if s.with_v else None
+        nan = base.k_pages == BF16_NAN  # the base layer's poisoned slots
+        k[nan] = BF16_NAN
+        if v is not None:
+            v[nan] = BF16_NAN
+        out.append(TriWorkload(spec=s, seqlens=base.seqlens, block_table=base.block_table, q_cal=q_cal, k_pages=k,
+                               v_pages=v))
+    return out
+
+
 def tri_algorithmic_bytes(s: TriSpec, seqlens: np.ndarray, mode: int = 0) -> int:
     """Bytes one eviction must move at minimum: every evictable token's K row
     read once for scoring, plus, for each request that evicts, every moved

@@ -154,7 +154,12 @@ sd_status launch_indexer_t(const int8_t* qi, const int32_t* w, const int8_t* ki,
                            const int32_t* seqlens, int32_t* scores, const sd_paged_desc& pd, int B,
                            int Hi, int max_seqlen, cudaStream_t st) {
   const size_t smem = sd::indexer_dp4a_smem(pd.kv_heads, Hi, DI);
-  dim3 grid(sd::ceil_div(max_seqlen, sd::kIdxTokensPerCta), B);
+  if (smem > 48 * 1024) {
+    const sd_status s = cuda_check(cudaFuncSetAttribute(sd::indexer_dp4a_kernel<DI>,
+                                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+    if (s != SD_OK) return s;
+  }
+  dim3 grid(sd::ceil_div(max_seqlen, sd::indexer_dp4a_tokens(pd.kv_heads, DI)), B);
   stage_mark(kStageIndexer, 0, st);
   const sd_status s = launch_k(sd::indexer_dp4a_kernel<DI>, grid, dim3(sd::kIdxThreads), smem, st, qi, w, ki, bt,
                                seqlens, scores, pd.num_pages, pd.page_size, pd.max_pages_per_req, pd.kv_heads, Hi,

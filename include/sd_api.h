@@ -97,7 +97,8 @@ size_t sd_workspace_size(int32_t B, int32_t G, int32_t max_seqlen, int32_t k,
 /* Steps 1 + 2: indexer scores and per-(request, KV head) top-k.
  *   qi          int8  [B, G, Hi, Di]  indexer queries
  *   w           int32 [B, G, Hi]      indexer head weights
- *   ki_pages    int8  [num_pages, page_size, G, Di]  indexer key pool
+ *   ki_pages    int8  [num_pages, page_size, G, Di]  indexer key pool, 16-byte
+ *               aligned (SD_ERR_INVALID_ARG otherwise)
  *   block_table int32 [B, max_pages_per_req]  physical page per logical page
  *   seqlens     int32 [B]             cached tokens per request (incl. current)
  *   max_seqlen  host upper bound of seqlens (sizes grids and scores)

@@ -142,3 +142,9 @@ def test_tri_layers_argument_errors(lib):
     assert lib.sd_tri_layers_workspace_size(4, 64, 2, 4, 64, 5000, 4, 8, 2048, 0, 1) > \
         lib.sd_tri_layers_workspace_size(1, 64, 2, 4, 64, 5000, 4, 8, 2048, 0, 1)  # a flag set per layer
     assert lib.sd_last_launch_count() == 0
+
+
+def test_indexer_rejects_a_misaligned_key_pool(lib):
+    desc = api.PagedDesc(4, 16, 4, 1)
+    # qi, w, ki_pages, block_table, seqlens, pd, B, Hi, Di, max_seqlen, k, indices, scores, ws, ws_bytes, stream
+    assert lib.sd_indexer_topk(256, 256, 264, 256, 256, desc, 1, 4, 32, 64, 8, 256, None, None, 0, None) == 1

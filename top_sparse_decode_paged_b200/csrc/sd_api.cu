@@ -131,6 +131,8 @@ sd_status check_indexer_args(const int8_t* qi, const int32_t* w, const int8_t* k
     return SD_ERR_INVALID_ARG;
   if (Di != 32 && Di != 64 && Di != 128) return SD_ERR_UNSUPPORTED;
   if (Hi > 64 || pd.kv_heads * Di > 1024) return SD_ERR_UNSUPPORTED;
+  // key rows are copied in 16-byte units (bulk copies, TMA)
+  if ((reinterpret_cast<uintptr_t>(ki_pages) & 15u) != 0) return SD_ERR_INVALID_ARG;
   if (k > kMaxK || max_seqlen > kMaxSeqlen) return SD_ERR_UNSUPPORTED;
   return SD_OK;
 }

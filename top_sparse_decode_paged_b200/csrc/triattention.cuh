@@ -24,7 +24,9 @@
 // Compaction moves kept token i from logical position t_i to position i in
 // one pass over the pools (see tri_compact_kernel). Union mode moves whole
 // rows (all KV heads); per-head mode moves each KV head's part by its own
-// selection.
+// selection. Selections shared across layers are composed on the host: the
+// key pass folds each layer's scores in by maximum, then every layer is
+// compacted with the one selection.
 #pragma once
 
 #include "sd_common.cuh"
@@ -54,7 +56,7 @@ constexpr int kTriTileTok = kTriThreads;  // evictable positions per score tile
 // load feeds four heads at a given d. Each row's source offset is computed
 // once (no division per copied piece).
 // Thread r sums row r over d in index order, one fused multiply-add per
-// (d, head). Small CTAs (about 37 KB) let six share an SM, so copies of some
+// (d, head). Small CTAs (about 40 KB) let five share an SM, so copies of some
 // overlap the arithmetic of others.
 template <int D, int QPK>
 __global__ void __launch_bounds__(kTriThreads) tri_score_kernel(

@@ -68,7 +68,7 @@ def test_tiny_ragged(mode, with_v):
     assert nl.tolist() == [4 + 24 + 8, 20, 4 + 24 + 8]
 
 
-@pytest.mark.parametrize("H,G,D", [(32, 8, 128), (8, 8, 64), (16, 8, 64), (16, 2, 128)])
+@pytest.mark.parametrize("H,G,D", [(32, 8, 128), (8, 8, 64), (16, 8, 64), (16, 2, 128), (4, 1, 64)])
 @pytest.mark.parametrize("mode", [T.UNION, T.PER_HEAD])
 def test_shapes_span_tiles(H, G, D, mode):
     """Regions of several 128-position score tiles with ragged tails, every
@@ -76,6 +76,29 @@ def test_shapes_span_tiles(H, G, D, mode):
     s = tri_spec("tri_ragged_b16", B=5, H=H, G=G, D=D, page_size=16, n_sink=40, n_recent=9, budget=200,
                  ragged=(0, 700), seed=20 + H + G + D)
     _check(make_tri(s), mode)
+
+
+def test_misaligned_queries():
+    """A q_cal that is not 16-byte aligned (the score pass reads it element by
+    element) gives the same result bit for bit."""
+    import torch
+    import top_sparse_decode_paged_b200 as sd
+    w = make_tri(tri_spec("tri_ragged_b16", B=3, page_size=16, n_sink=40, n_recent=9, budget=200, ragged=(0, 700),
+                          seed=35))
+    s = w.spec
+    k_ref, v_ref, nl_ref, _ = T.tri_evict(w.q_cal, w.k_pages, w.v_pages, w.block_table, w.seqlens, s.n_sink,
+                                          s.n_recent, s.budget, T.UNION)
+    flat = torch.zeros(s.H * s.D + 1, dtype=torch.int16, device="cuda")
+    flat[1:] = torch.from_numpy(w.q_cal.view(np.int16).reshape(-1)).cuda()
+    q = flat[1:].view(s.H, s.D).view(torch.bfloat16)
+    assert q.data_ptr() % 16 != 0
+    kp, vp = _bf16(w.k_pages), _bf16(w.v_pages)
+    nl = sd.sd_tri_compact(q, kp, vp, _dev(w.block_table), _dev(w.seqlens), w.max_seqlen, s.n_sink, s.n_recent,
+                           s.budget, T.UNION)
+    torch.cuda.synchronize()
+    assert sd.device_errors() == 0
+    assert np.array_equal(nl.cpu().numpy(), nl_ref)
+    assert np.array_equal(_bits(kp), k_ref) and np.array_equal(_bits(vp), v_ref)
 
 
 def test_heavy_ties_on_gpu():

@@ -135,8 +135,9 @@ sd_status sd_sparse_attn(const uint16_t* q, const uint16_t* k_pages, const uint1
  * rows in place to the front of the request's pages.
  *   q_cal       bf16 [H, D]: one calibrated query per query head (head h reads
  *               KV head h * G / H), in the cache's precision
- *   k_pages     bf16 [num_pages, P, G, D], compacted in place
- *   v_pages     bf16 [num_pages, P, G, D] compacted the same way, or NULL
+ *   k_pages     bf16 [num_pages, P, G, D], compacted in place; 16-byte aligned
+ *   v_pages     bf16 [num_pages, P, G, D] compacted the same way, or NULL;
+ *               16-byte aligned
  *   mode        SD_TRI_UNION: one selection per request (all KV heads move
  *               together); SD_TRI_PER_HEAD (or SD_TRI_PER_LAYER_PER_HEAD):
  *               one per (request, KV head)

@@ -148,3 +148,13 @@ def test_indexer_rejects_a_misaligned_key_pool(lib):
     desc = api.PagedDesc(4, 16, 4, 1)
     # qi, w, ki_pages, block_table, seqlens, pd, B, Hi, Di, max_seqlen, k, indices, scores, ws, ws_bytes, stream
     assert lib.sd_indexer_topk(256, 256, 264, 256, 256, desc, 1, 4, 32, 64, 8, 256, None, None, 0, None) == 1
+
+
+def test_tri_rejects_misaligned_pools(lib):
+    desc = api.PagedDesc(64, 16, 8, 2)
+    f = lib.sd_tri_compact
+    # q_cal, k_pages, v_pages, block_table, seqlens, pd, B, H, D, max_seqlen, n_sink, n_recent, budget, mode,
+    # new_seqlens, workspace, workspace_bytes, stream
+    assert f(256, 264, None, 256, 256, desc, 2, 4, 64, 100, 4, 8, 24, 0, 256, None, 0, None) == 1
+    assert f(256, 256, 264, 256, 256, desc, 2, 4, 64, 100, 4, 8, 24, 0, 256, None, 0, None) == 1
+    assert f(256, 256, 256, 256, 256, desc, 2, 4, 64, 100, 4, 8, 24, 0, 256, None, 0, None) == 3  # aligned: workspace

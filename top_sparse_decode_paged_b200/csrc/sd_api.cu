@@ -696,8 +696,13 @@ sd_status sd_tri_compact_layers(const uint16_t* const* q_cal, uint16_t* const* k
   t_launches = 0;
   if (n_layers < 1 || !q_cal || !k_pages || !geom_ok(pd) || (B > 0 && (!block_table || !seqlens || !new_seqlens)))
     return SD_ERR_INVALID_ARG;
-  for (int l = 0; l < n_layers; ++l)
+  for (int l = 0; l < n_layers; ++l) {
     if (!q_cal[l] || !k_pages[l] || (v_pages && !v_pages[l])) return SD_ERR_INVALID_ARG;
+    // pool rows are copied in 16-byte units
+    if ((reinterpret_cast<uintptr_t>(k_pages[l]) & 15u) != 0 ||
+        (v_pages && (reinterpret_cast<uintptr_t>(v_pages[l]) & 15u) != 0))
+      return SD_ERR_INVALID_ARG;
+  }
   const int G = pd.kv_heads;
   if (!tri_args_ok(n_layers, B, G, H, D, max_seqlen, n_sink, n_recent, budget, mode)) return SD_ERR_INVALID_ARG;
   const int qpk = H / G;

@@ -150,14 +150,19 @@ sd_status sd_sparse_attn(const uint16_t* q, const uint16_t* k_pages, const uint1
  * union score the maximum over KV heads. The `budget` largest are kept (ties
  * to the lower position), followed by the recent tail. Pages past the new
  * lengths are free for the caller to release; the block table is unchanged.
+ * max_seqlen is a host upper bound of seqlens (it sizes the workspace);
+ * larger lengths are clamped and flag SD_DEVERR_SEQLEN.
  * Limits: D in {64, 128}; H / G in {1, 2, 4, 8}; H <= 256;
  * 1 <= budget <= 2048; B * G <= 65535; the bytes one token moves (union:
- * G * D * 2, per-head: D * 2; twice that with V) at most 32768. block_table, seqlens and new_seqlens may be NULL when B = 0.
- * Workspace: sd_tri_workspace_size(); the caller owns every buffer. Errors:
- * SD_ERR_INVALID_ARG / SD_ERR_UNSUPPORTED / SD_ERR_WORKSPACE before any
- * launch; a block-table entry outside the pool inside a request sets
+ * G * D * 2, per-head: D * 2; twice that with V) at most 32768.
+ * block_table, seqlens and new_seqlens may be NULL when B = 0.
+ * Workspace: sd_tri_workspace_size(); the caller owns every buffer.
+ * Errors: SD_ERR_INVALID_ARG / SD_ERR_UNSUPPORTED / SD_ERR_WORKSPACE before
+ * any launch. A block-table entry outside the pool inside a request sets
  * SD_DEVERR_PAGE and that row is skipped (the request's result is then
- * unspecified, the pools outside its pages untouched). */
+ * unspecified, the pools outside its pages untouched). The compaction's
+ * units wait on one another with bounded waits; one that runs out sets
+ * SD_DEVERR_TIMEOUT and skips its writes. */
 #define SD_TRI_UNION 0
 #define SD_TRI_PER_HEAD 1
 #define SD_TRI_PER_LAYER_PER_HEAD 2 /* with one layer, the same as SD_TRI_PER_HEAD */

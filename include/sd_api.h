@@ -143,12 +143,13 @@ sd_status sd_sparse_attn(const uint16_t* q, const uint16_t* k_pages, const uint1
  *               one per (request, KV head)
  *   new_seqlens int32 [B] out: n_sink + budget + n_recent, or L_b when the
  *               evictable region holds at most `budget` tokens (nothing moves)
- * Score of evictable position p under query head h: z = q_cal[h] . K, one
- * fp32 fused multiply-add per d in index order (the bf16 x bf16 product is
- * exact, so the result is reproducible), shifted by the head's maximum over
- * the region; a KV head's score is the maximum over its query heads, the
- * union score the maximum over KV heads. The `budget` largest are kept (ties
- * to the lower position), followed by the recent tail. Pages past the new
+ * Score of evictable position p under query head h: z = q_cal[h] . K, summed
+ * in fp32 (each bf16 x bf16 product exact; one fused multiply-add per d, so
+ * equal inputs give equal scores), shifted by the head's maximum over the
+ * region; a KV head's score is the maximum over its query heads, the union
+ * score the maximum over KV heads. The `budget` largest are kept (ties to the
+ * lower position), followed by the recent tail. The kept set is a top-budget
+ * set of the exact scores up to the fp32 rounding of the sums. Pages past the new
  * lengths are free for the caller to release; the block table is unchanged.
  * max_seqlen is a host upper bound of seqlens (it sizes the workspace);
  * larger lengths are clamped and flag SD_DEVERR_SEQLEN.

@@ -22,24 +22,23 @@ per-head modes; deterministic tie settlement):
    [L - n_recent, L); the new length is n_sink + budget + n_recent. Union mode
    moves whole rows, per-head mode each KV head's part by its own selection.
 
-Precision: the scores only decide an integer selection, so they are taken in
-the same precision as the library: fp32, summed over d in index order, each
-step one fused multiply-add acc <- fl32(acc + q k). It is written out exactly:
-the bf16 x bf16 product is exact in fp64, and the fp64 sum of it and the fp32
-accumulator either is exact (operands within 2^29 of each other) or lies so far
-from an fp32 rounding boundary that rounding it to fp32 equals rounding the
-exact sum. z - max is one fp32 subtraction. (A score is never -0.0: the sums
-start at +0.0 and x - x rounds to +0.0, so the comparison of fp32 values below
-is the same order as any total order on them.)
+Precision: the scores are the plain definition, computed in fp64. The
+factors are bf16 values, so every product q k is exact in fp64; the sum of D
+of them is rounded at most D times at 2^-53, far below anything a selection
+can depend on, and the shift and the maxima are exact fp64 operations on it.
+No summation order is assumed: a kernel that sums in fp32, in any order, is
+checked against these scores with the fp32 error bound of its arithmetic
+(the tests derive that bound), not against a restatement of its rounding.
 
 Readings where the pages are silent (they name the steps, not the formulas):
 the score is the plain dot product with the calibrated query; each head is
 shifted by its own maximum before the maximum over heads; the protected prefix
 and tail are uniform sizes. The design notes list them.
 
-Parity pins: ``tests/test_tri_pins.py`` (one-hot queries against a closed form
-and an independent sort, an fp64 error bound, shift invariance of the per-head
-normalisation, a hand-worked compaction across pages, the degenerate cases).
+Parity pins: ``tests/test_tri_pins.py`` (the logits against an exact rational
+dot product, one-hot queries against a closed form and an independent sort,
+shift invariance of the per-head normalisation, a hand-worked compaction
+across pages, brute force over small subsets, the degenerate cases).
 """
 
 from __future__ import annotations
@@ -58,27 +57,23 @@ def _evictable(L: int, n_sink: int, n_recent: int) -> int:
 
 
 def tri_logits(q_cal: np.ndarray, K: np.ndarray, G: int) -> np.ndarray:
-    """z[h, p] = q_cal[h] . K[p, h * G // H]: over d in index order, each step
-    one fp32 fused multiply-add (exact product, one rounding).
+    """z[h, p] = q_cal[h] . K[p, h * G // H], the plain dot product in fp64
+    (each bf16 x bf16 product exact; the sum rounded in fp64).
 
     q_cal: [H, D] and K: [E, G, D], bf16 values in any float type.
-    Returns fp32 [H, E]."""
+    Returns fp64 [H, E]."""
     q = np.asarray(q_cal, dtype=np.float64)
     H, D = q.shape
     E = K.shape[0]
-    z = np.zeros((H, E), dtype=np.float32)
+    z = np.zeros((H, E), dtype=np.float64)
     for h in range(H):
         g = h * G // H
-        Kg = np.asarray(K[:, g, :], dtype=np.float64)
-        acc = np.zeros(E, dtype=np.float32)
-        for d in range(D):
-            acc = (acc.astype(np.float64) + Kg[:, d] * q[h, d]).astype(np.float32)
-        z[h] = acc
+        z[h] = np.asarray(K[:, g, :], dtype=np.float64) @ q[h]
     return z
 
 
 def tri_scores(q_cal, k_pages, block_table, seqlens, n_sink: int, n_recent: int, mode: int):
-    """Per request, its selection rows' scores: fp32 [rows, E_b] with rows = 1
+    """Per request, its selection rows' scores: fp64 [rows, E_b] with rows = 1
     (union) or G (per-head). q_cal: bf16 bits [H, D]; k_pages: bf16 bits
     [num_pages, P, G, D]."""
     G = k_pages.shape[2]
@@ -89,13 +84,10 @@ def tri_scores(q_cal, k_pages, block_table, seqlens, n_sink: int, n_recent: int,
     for b, L in enumerate(np.asarray(seqlens)):
         E = _evictable(int(L), n_sink, n_recent)
         tokens = np.arange(n_sink, n_sink + E)
-        K = bf16_bits_to_f64(gather_token_rows(k_pages, block_table[b], tokens)).astype(np.float32)
+        K = bf16_bits_to_f64(gather_token_rows(k_pages, block_table[b], tokens))
         z = tri_logits(q_cal, K, G)
-        if E > 0:
-            zs = (z - z.max(axis=1, keepdims=True)).astype(np.float32)
-        else:
-            zs = z
-        per_g = np.stack([zs[g * qpk:(g + 1) * qpk].max(axis=0) if E > 0 else np.zeros(0, np.float32)
+        zs = z - z.max(axis=1, keepdims=True) if E > 0 else z
+        per_g = np.stack([zs[g * qpk:(g + 1) * qpk].max(axis=0) if E > 0 else np.zeros(0, np.float64)
                           for g in range(G)])
         out.append(per_g if mode == PER_HEAD else per_g.max(axis=0, keepdims=True))
     return out
@@ -110,7 +102,7 @@ def tri_select(scores_b: np.ndarray, budget: int) -> np.ndarray:
     out = np.zeros((rows, budget), dtype=np.int64)
     for r in range(rows):
         # full sort by (score descending, position ascending); lexsort keys go last-first
-        order = np.lexsort((np.arange(E), -scores_b[r].astype(np.float64)))
+        order = np.lexsort((np.arange(E), -np.asarray(scores_b[r], dtype=np.float64)))
         out[r] = np.sort(order[:budget])
     return out
 

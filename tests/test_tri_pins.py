@@ -31,36 +31,74 @@ def _bf(x):
     return (bf16_bits_from_f32(np.asarray(x, np.float32)).astype(np.uint32) << 16).view(np.float32)
 
 
-def test_logits_within_fp32_bound_of_fp64_dot():
-    """z agrees with the exact fp64 dot product (head h reads KV head h // (H/G))
-    within the recursive-summation bound D u sum|q k|; a transposed operand, a
-    wrong head map or a dropped term breaks the bound."""
+def test_logits_equal_the_exact_rational_dot_product():
+    """z[h, p] equals q_cal[h] . K[p, h // (H/G)] summed exactly in rationals
+    (bf16 values are dyadic), up to the fp64 rounding of the sum; a transposed
+    operand, a wrong head map or a dropped term is off by far more."""
+    from fractions import Fraction
     rng = np.random.default_rng(0)
-    H, G, D, E = 6, 3, 64, 40
+    H, G, D, E = 6, 3, 64, 12
     q = _bf(rng.standard_normal((H, D), dtype=np.float32)).astype(np.float64)
     Kf = _bf(rng.standard_normal((E, G, D), dtype=np.float32)).astype(np.float64)
     z = T.tri_logits(q, Kf, G)
-    u = 2.0 ** -24
+    assert z.dtype == np.float64
     for h in range(H):
         g = h // (H // G)
-        exact = Kf[:, g, :] @ q[h]
-        bound = D * u * (np.abs(Kf[:, g, :]) @ np.abs(q[h]))
-        assert np.all(np.abs(z[h] - exact) <= bound)
+        for p in range(E):
+            exact = sum(Fraction(float(q[h, d])) * Fraction(float(Kf[p, g, d])) for d in range(D))
+            scale = float(np.abs(q[h]) @ np.abs(Kf[p, g]))
+            assert abs(Fraction(float(z[h, p])) - exact) <= Fraction(D * 2.0 ** -53 * scale)
 
 
-def test_each_step_rounds_to_fp32_in_index_order():
-    """Products 1, 2^-24, 2^-24 (q = k = 1, 2^-12, 2^-12): rounding after every
-    step in index order keeps 1 (each 1 + 2^-24 is a tie, to even); one
-    rounding of the exact sum, or the reverse order, gives 1 + 2^-23. A tiny
-    product under a large accumulator leaves it unchanged."""
-    v = np.array([1.0, 2.0 ** -12, 2.0 ** -12])
-    z = T.tri_logits(v[None, :], v.reshape(1, 1, 3), 1)
-    assert z[0, 0] == np.float32(1.0)
-    z = T.tri_logits(v[None, ::-1].copy(), v[::-1].reshape(1, 1, 3).copy(), 1)
-    assert z[0, 0] == np.float32(1.0 + 2.0 ** -23)
-    q = np.array([[2.0 ** 40, 2.0 ** -60]])
-    K = np.array([[[1.0, 1.0]]]).reshape(1, 1, 2)
-    assert T.tri_logits(q, K, 1)[0, 0] == np.float32(2.0 ** 40)
+def _fp32_scores_reverse_order(w, mode):
+    """Scores as an fp32 kernel could take them: products summed in fp32 in
+    reverse index order (one rounding per step), shift and maxima in fp32. A
+    different evaluation from the oracle's, inside the bound the GPU check
+    allows."""
+    s = w.spec
+    from oracle.sd_oracle import bf16_bits_to_f64, gather_token_rows
+    q = bf16_bits_to_f64(w.q_cal)
+    H, D = q.shape
+    qpk = H // s.G
+    out = []
+    for b, L in enumerate(w.seqlens):
+        E = max(0, int(L) - s.n_sink - s.n_recent)
+        K = bf16_bits_to_f64(gather_token_rows(w.k_pages, w.block_table[b], np.arange(s.n_sink, s.n_sink + E)))
+        z = np.zeros((H, E), dtype=np.float32)
+        for h in range(H):
+            acc = np.zeros(E, dtype=np.float32)
+            for d in range(D - 1, -1, -1):
+                acc = (acc.astype(np.float64) + K[:, h // qpk, d] * q[h, d]).astype(np.float32)
+            z[h] = acc
+        zs = (z - z.max(axis=1, keepdims=True)).astype(np.float32) if E else z
+        per_g = np.stack([zs[g * qpk:(g + 1) * qpk].max(axis=0) for g in range(s.G)])
+        out.append(per_g if mode == T.PER_HEAD else per_g.max(axis=0, keepdims=True))
+    return out
+
+
+@pytest.mark.parametrize("mode", [T.UNION, T.PER_HEAD])
+def test_gpu_check_accepts_an_fp32_evaluation_and_rejects_planted_mistakes(mode):
+    """The validity check the GPU tests use (tests/tri_check.py): a selection
+    from an fp32 evaluation in another order passes; swapping one kept
+    position for the worst dropped one fails; the bound is far below the
+    spread of the scores, so it does not accept everything."""
+    from tri_check import score_bounds, valid_selection
+    s = tri_spec("tri_ragged_b16", B=3, H=8, G=4, D=128, page_size=16, n_sink=8, n_recent=4, budget=100,
+                 ragged=(200, 400), seed=5)
+    w = make_tri(s)
+    bounds = score_bounds(w.q_cal, w.k_pages, w.block_table, w.seqlens, s.n_sink, s.n_recent, mode)
+    f32 = _fp32_scores_reverse_order(w, mode)
+    for (sc, slack), sc32 in zip(bounds, f32):
+        assert np.median(slack) < 1e-3 * np.std(sc)
+        assert np.all(np.abs(sc32.astype(np.float64) - sc) <= slack)
+        sel32 = T.tri_select(sc32, s.budget)
+        for r in range(sc.shape[0]):
+            assert valid_selection(sc[r], slack[r], sel32[r], s.budget)
+            bad = sel32[r].copy()
+            dropped = np.setdiff1d(np.arange(sc.shape[1]), bad)
+            bad[np.argmax(sc[r][bad])] = dropped[np.argmin(sc[r][dropped])]
+            assert not valid_selection(sc[r], slack[r], np.sort(bad), s.budget)
+            assert not valid_selection(sc[r], slack[r], sel32[r][:-1], s.budget)
 
 
 def test_one_hot_queries_closed_form_and_independent_sort():
@@ -239,3 +277,32 @@ def test_layers_union_keeps_each_layers_favourite():
     _, _, _, sels = T.tri_evict_layers(qs, [pool, pool], None, bt[None], np.array([E]), 0, 0, 2,
                                        T.PER_LAYER_PER_HEAD)
     assert sels[0][0].tolist() == [[1, 11]] and sels[1][0].tolist() == [[5, 7]]
+
+
+def test_gpu_check_reads_the_kept_set_back_and_compares_every_byte():
+    """check_eviction on the oracle's own eviction (standing in for the GPU's
+    pools) passes and reads back the oracle's kept sets; a wrong V row in one
+    kept slot, or a changed byte in a page no request owns, fails."""
+    from tri_check import check_eviction
+    w = make_tri(tri_spec("tri_tiny"))
+    s = w.spec
+    for mode in (T.UNION, T.PER_HEAD):
+        k2, v2, nl, sel = T.tri_evict(w.q_cal, w.k_pages, w.v_pages, w.block_table, w.seqlens, s.n_sink,
+                                      s.n_recent, s.budget, mode)
+        kept = check_eviction([w.q_cal], [w.k_pages], [w.v_pages], w.block_table, w.seqlens, s.n_sink, s.n_recent,
+                              s.budget, mode, [k2], [v2], nl)
+        for b in range(len(w.seqlens)):
+            assert np.array_equal(kept[0][b], sel[b])
+        P = s.page_size
+        t = s.n_sink + 3  # a kept slot of request 0 (it evicts)
+        bad_v = v2.copy()
+        bad_v[w.block_table[0, t // P], t % P, 0, 0] ^= 1
+        with pytest.raises(AssertionError):
+            check_eviction([w.q_cal], [w.k_pages], [w.v_pages], w.block_table, w.seqlens, s.n_sink, s.n_recent,
+                           s.budget, mode, [k2], [bad_v], nl)
+        spare = w.k_pages.shape[0] - 1  # the workload's spare pages belong to no request
+        bad_k = k2.copy()
+        bad_k[spare, 0, 0, 0] ^= 1
+        with pytest.raises(AssertionError):
+            check_eviction([w.q_cal], [w.k_pages], [w.v_pages], w.block_table, w.seqlens, s.n_sink, s.n_recent,
+                           s.budget, mode, [bad_k], [v2], nl)

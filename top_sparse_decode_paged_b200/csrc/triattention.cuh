@@ -8,9 +8,9 @@
 // Scoring (a reading; the pages do not write the formula). For request b,
 // query head h (KV head g = h * G / H) and evictable position p (token
 // t = n_sink + p, p < E_b = L_b - n_sink - n_recent):
-//   z[b,h,p] = q_cal[h] . K[t, g]     q_cal and K bf16; one fp32 fused
-//                                     multiply-add per d, in index order
-//                                     (reproducible: the product is exact)
+//   z[b,h,p] = q_cal[h] . K[t, g]     q_cal and K bf16, summed in fp32: one
+//                                     fused multiply-add per d (the product is
+//                                     exact; equal inputs give equal scores)
 //   m[b,h]   = max_p z[b,h,p]
 //   s[b,g,p] = max over the heads h of KV head g of (z[b,h,p] - m[b,h])
 //   union:     s[b,p] = max_g s[b,g,p]

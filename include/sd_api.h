@@ -283,15 +283,21 @@ sd_status sd_decode_step(const int8_t* qi, const int32_t* w, const int8_t* ki_pa
  * allocate device memory: a plugin that runs inside a host application which
  * owns every device allocation, or a serving loop that must not allocate once
  * it has started. Such callers cannot provide a scores workspace. Here the
- * scores live in a scratch array that the library itself holds on each device
- * it is used on, from first use until process exit:
- * SD_NOALLOC_MAX_SCORES int32 values (16 MiB).
+ * scores live in a scratch array inside the library's device image:
+ * SD_NOALLOC_MAX_SCORES int32 values (16 MiB). It is resident on every device
+ * where the library's device code is loaded, whichever entry point loaded
+ * it, from then until the context is destroyed.
  *   Arguments, outputs and errors are as for sd_indexer_topk. There is no
  *   scores output. The call returns SD_ERR_WORKSPACE, with nothing enqueued,
  *   when B * G * max_seqlen > SD_NOALLOC_MAX_SCORES.
- *   The first call on a device looks up that device's scratch address (a
- *   runtime query, not an allocation). Make that first call before any stream
- *   capture on that device.
+ *   A call that is not being captured looks up the device's scratch address
+ *   (a runtime query, not an allocation) and remembers it; a call under
+ *   stream capture uses the remembered address. So make one call on a device
+ *   before capturing any, and again after a device reset or anything else
+ *   that destroys the primary context (that reloads the library's device
+ *   image at another address): a captured graph keeps the address it was
+ *   captured with and must be captured anew after such a reset. A first call
+ *   on a device made under capture returns SD_ERR_INVALID_ARG.
  *   Every call on a device shares the one scratch array. Calls whose work
  *   overlaps on the GPU (other streams, other threads) race on it and give
  *   undefined results: serialise them. The array keeps the last call's scores,
@@ -311,6 +317,19 @@ sd_status sd_indexer_topk_noalloc(const int8_t* qi, const int32_t* w, const int8
  * a call does not run records nothing). n = 0 or events = NULL switches it
  * off. The handles must outlive their use; the library does not own them. */
 sd_status sd_set_stage_events(void* const* events, int32_t n);
+
+/* Test hook for the failure path of bounded waits (no counterpart on the
+ * pages). The eviction compaction's units wait on one another through flags
+ * in global memory (sd_tri_compact); each wait gives up after a bounded number
+ * of polls, sets SD_DEVERR_TIMEOUT and skips that unit's writes, so a wait
+ * that never ends cannot hang the GPU. This sets that number for compactions
+ * launched afterwards by any thread of the process (it is a launch argument,
+ * so a captured graph keeps the value it was captured with): polls < 0
+ * restores the default of 2^22, 0 makes every such wait give up at once (the
+ * compaction then leaves the pools in an unspecified state and flags the
+ * timeout). Values above 2^22 return SD_ERR_INVALID_ARG. No other wait of
+ * the library is affected. Nothing is enqueued; no CUDA call is made. */
+sd_status sd_set_wait_limit(int32_t polls);
 
 /* Reads (and with clear != 0 resets) the sticky device error word of the
  * current device. Synchronises the device: for tests and debugging only. */

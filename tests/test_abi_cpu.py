@@ -158,3 +158,27 @@ def test_tri_rejects_misaligned_pools(lib):
     assert f(256, 264, None, 256, 256, desc, 2, 4, 64, 100, 4, 8, 24, 0, 256, None, 0, None) == 1
     assert f(256, 256, 264, 256, 256, desc, 2, 4, 64, 100, 4, 8, 24, 0, 256, None, 0, None) == 1
     assert f(256, 256, 256, 256, 256, desc, 2, 4, 64, 100, 4, 8, 24, 0, 256, None, 0, None) == 3  # aligned: workspace
+
+
+def test_wait_limit_hook_checks_its_argument_without_cuda(lib):
+    """sd_set_wait_limit makes no CUDA call: it accepts 0 .. 2^22 and < 0
+    (the default) and rejects a limit above the default."""
+    assert lib.sd_set_wait_limit(0) == 0
+    assert lib.sd_set_wait_limit(1 << 22) == 0
+    assert lib.sd_set_wait_limit((1 << 22) + 1) == 1
+    assert lib.sd_set_wait_limit(-1) == 0
+
+
+def test_noalloc_argument_errors_return_before_any_cuda_call(lib):
+    """sd_indexer_topk_noalloc rejects bad arguments before it looks up its
+    scratch array or launches anything."""
+    desc = api.PagedDesc(4, 16, 4, 1)
+
+    def call(qi=256, idx=256, Di=32, B=1, L=64):
+        return lib.sd_indexer_topk_noalloc(qi, 256, 256, 256, 256, desc, B, 4, Di, L, 8, idx, None)
+
+    assert call(qi=None) == 1                                   # SD_ERR_INVALID_ARG
+    assert call(idx=None) == 1
+    assert call(Di=48) == 2                                     # SD_ERR_UNSUPPORTED
+    assert call(B=8, L=(api.NOALLOC_MAX_SCORES // 8) + 1) == 3  # SD_ERR_WORKSPACE
+    assert lib.sd_last_launch_count() == 0

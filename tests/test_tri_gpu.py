@@ -239,3 +239,30 @@ def test_layers_one_layer_matches_single_call():
                              s.n_sink, s.n_recent, s.budget, T.PER_LAYER_PER_HEAD)
     torch.cuda.synchronize()
     assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+
+
+def test_compaction_wait_runs_out_and_the_device_stays_usable():
+    """Failure path of the bounded cross-CTA waits, made to happen from the
+    host: with the wait limit at 0 polls every unit that waits on an earlier
+    one gives up at once. The call returns, SD_DEVERR_TIMEOUT is set, and the
+    next call with the default limit evicts a fresh copy correctly. No unit
+    has a copy in flight when it gives up, and nothing waits without bound."""
+    import torch
+    import top_sparse_decode_paged_b200 as sd
+    s = tri_spec("tri_ragged_b16", B=4, H=32, G=8, D=128, page_size=16, n_sink=40, n_recent=9, budget=200,
+                 ragged=(300, 700), seed=51)
+    w = make_tri(s)
+    # 2048 bytes per union token (K and V: 4096), so a 32 KB unit holds 8 kept tokens and every
+    # row has many units; later units read destinations that earlier units hold
+    assert (s.budget + s.n_recent) > 2 * (32768 // (2 * s.G * s.D * 2))
+    assert sd.device_errors() == 0
+    try:
+        sd.set_wait_limit(0)
+        kp, vp = _bf16(w.k_pages), _bf16(w.v_pages)
+        sd.sd_tri_compact(_dev(w.q_cal), kp, vp, _dev(w.block_table), _dev(w.seqlens), w.max_seqlen, s.n_sink,
+                          s.n_recent, s.budget, T.UNION)
+        torch.cuda.synchronize()
+        assert sd.device_errors() & sd.SD_DEVERR_TIMEOUT
+    finally:
+        sd.set_wait_limit(-1)
+    _check(w, T.UNION)  # default limit: fresh pools, the full check, no error bit

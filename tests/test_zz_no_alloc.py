@@ -52,7 +52,10 @@ def test_noalloc_limit_is_on_scratch_size():
     spec = W.spec("perhead_b16_gqa", seqlens=(3000,), seed=33)      # B=1, G=8
     wl = W.make(spec)
     d = to_device(wl)
-    at_limit = sd.NOALLOC_MAX_SCORES // 8                           # 524288 <= 1 << 20
+    # 8 * 524288 == NOALLOC_MAX_SCORES, and at_limit + 1 is still below the
+    # library's max_seqlen limit (1 << 20), so only the scratch check can
+    # reject the second call
+    at_limit = sd.NOALLOC_MAX_SCORES // 8
     idx = torch.empty((1, 8, spec.k), dtype=torch.int32, device="cuda")
     sd.sd_indexer_topk_noalloc(d["qi"], d["w"], d["ki_pages"], d["block_table"], d["seqlens"], spec.k,
                                at_limit, idx)
@@ -64,3 +67,27 @@ def test_noalloc_limit_is_on_scratch_size():
         sd.sd_indexer_topk_noalloc(d["qi"], d["w"], d["ki_pages"], d["block_table"], d["seqlens"], spec.k,
                                    at_limit + 1, idx)
     assert e.value.name == "SD_ERR_WORKSPACE"
+
+
+def test_noalloc_allocates_no_device_memory():
+    """The property the entry point exists for: after one warm-up call (which
+    loads every kernel it uses), a call at the scratch limit changes neither
+    the device's free memory nor torch's allocated bytes."""
+    import torch
+    import top_sparse_decode_paged_b200 as sd
+    spec = W.spec("perhead_b16_gqa", seqlens=(3000,), seed=34)      # B=1, G=8
+    wl = W.make(spec)
+    d = to_device(wl)
+    at_limit = sd.NOALLOC_MAX_SCORES // 8
+    idx = torch.empty((1, 8, spec.k), dtype=torch.int32, device="cuda")
+
+    def call():
+        sd.sd_indexer_topk_noalloc(d["qi"], d["w"], d["ki_pages"], d["block_table"], d["seqlens"], spec.k,
+                                   at_limit, idx)
+        torch.cuda.synchronize()
+
+    call()
+    free0, alloc0 = torch.cuda.mem_get_info()[0], torch.cuda.memory_allocated()
+    call()
+    assert torch.cuda.mem_get_info()[0] == free0
+    assert torch.cuda.memory_allocated() == alloc0

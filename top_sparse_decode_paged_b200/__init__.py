@@ -10,6 +10,7 @@ from .api import (  # noqa: F401
     SD_DEVERR_INDEX,
     SD_DEVERR_PAGE,
     SD_DEVERR_SEQLEN,
+    SD_DEVERR_TIMEOUT,
     SdError,
     TRI_PER_HEAD,
     TRI_PER_LAYER_PER_HEAD,
@@ -29,6 +30,7 @@ from .api import (  # noqa: F401
     sd_sparse_attn_layers,
     sd_tri_compact,
     sd_tri_compact_layers,
+    set_wait_limit,
     workspace_size,
 )
 
@@ -36,5 +38,5 @@ __all__ = [
     "sd_indexer_topk", "sd_indexer_topk_hinted", "sd_indexer_topk_noalloc", "sd_decode_step_hinted", "sd_sparse_attn", "sd_sparse_attn_layers", "sd_sparse_attn_csr",
     "sd_decode_step", "sd_tri_compact", "sd_tri_compact_layers", "TRI_UNION", "TRI_PER_HEAD",
     "TRI_PER_LAYER_PER_HEAD",
-    "workspace_size", "alloc_workspace", "device_errors", "load_library", "SdError", "StageTimer",
+    "workspace_size", "alloc_workspace", "device_errors", "set_wait_limit", "load_library", "SdError", "StageTimer",
 ]

@@ -20,12 +20,13 @@ LIB_PATH = os.path.join(_PKG, "libsd.so")
 SD_DEVERR_SEQLEN = 0x1
 SD_DEVERR_PAGE = 0x2
 SD_DEVERR_INDEX = 0x4
+SD_DEVERR_TIMEOUT = 0x8
 
 EXPORTED = ("sd_workspace_size", "sd_indexer_topk", "sd_indexer_topk_noalloc", "sd_sparse_attn",
             "sd_attn_layers_workspace_size", "sd_sparse_attn_layers", "sd_csr_workspace_size",
             "sd_sparse_attn_csr", "sd_indexer_topk_hinted", "sd_decode_step_hinted", "sd_decode_step",
             "sd_tri_workspace_size", "sd_tri_compact", "sd_tri_layers_workspace_size", "sd_tri_compact_layers",
-            "sd_set_stage_events", "sd_get_device_errors", "sd_status_str", "sd_last_cuda_error",
+            "sd_set_stage_events", "sd_set_wait_limit", "sd_get_device_errors", "sd_status_str", "sd_last_cuda_error",
             "sd_last_launch_count", "sd_version")
 
 
@@ -93,6 +94,8 @@ def load_library(path: str = LIB_PATH):
                                           sz, p]
     lib.sd_set_stage_events.restype = i32
     lib.sd_set_stage_events.argtypes = [ctypes.POINTER(ctypes.c_void_p), i32]
+    lib.sd_set_wait_limit.restype = i32
+    lib.sd_set_wait_limit.argtypes = [i32]
     lib.sd_get_device_errors.restype = i32
     lib.sd_get_device_errors.argtypes = [ctypes.POINTER(ctypes.c_uint32), i32]
     lib.sd_status_str.restype = ctypes.c_char_p
@@ -384,6 +387,12 @@ def sd_tri_compact_layers(q_cals, k_pools, v_pools, block_table, seqlens, max_se
                                      int(max_seqlen), int(n_sink), int(n_recent), int(budget), int(mode),
                                      _ptr(new_seqlens), _ptr(workspace), workspace.numel(), _stream(stream)))
     return new_seqlens
+
+
+def set_wait_limit(polls: int) -> None:
+    """Polls the eviction compaction's cross-CTA waits make before giving up
+    (a test hook; < 0 restores the default)."""
+    _check(load_library().sd_set_wait_limit(int(polls)))
 
 
 def device_errors(clear: bool = True) -> int:

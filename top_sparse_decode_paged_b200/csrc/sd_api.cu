@@ -7,6 +7,7 @@
 #include <math.h>
 
 #include <algorithm>
+#include <atomic>
 #include <mutex>
 #include <stdint.h>
 
@@ -35,6 +36,10 @@ void stage_mark(int stage, int edge, cudaStream_t st) {
   // a host can time after each graph replay
   if (stage < t_stage_count) cudaEventRecordWithFlags(t_stage_events[2 * stage + edge], st, cudaEventRecordExternal);
 }
+
+// Polls the eviction compaction's cross-CTA waits make before giving up
+// (sd_set_wait_limit; a launch argument, read on the host at launch).
+std::atomic<uint32_t> g_tri_wait_limit{sd::kTriWaitLimit};
 
 constexpr size_t kAlign = 256;
 constexpr int kMaxK = 2048;
@@ -668,7 +673,8 @@ sd_status tri_select_compact(const uint16_t* const* q_cal, uint16_t* const* k_pa
                       reinterpret_cast<uint8_t*>(v_pages ? v_pages[l] : nullptr), block_table, seqlens,
                       static_cast<const int32_t*>(sel), p.rows_per_req, pd.page_size, pd.max_pages_per_req,
                       pd.num_pages, cap, n_sink, n_recent, budget, p.part, G * D * 2, p.chunk, p.n_chunks, rows,
-                      flags + (size_t)l * p.flags_per_layer, new_seqlens)) != SD_OK)
+                      flags + (size_t)l * p.flags_per_layer, new_seqlens,
+                      g_tri_wait_limit.load(std::memory_order_relaxed))) != SD_OK)
       return s;
   }
   return SD_OK;
@@ -802,6 +808,12 @@ sd_status sd_set_stage_events(void* const* events, int32_t n) {
   return SD_OK;
 }
 
+sd_status sd_set_wait_limit(int32_t polls) {
+  if (polls > static_cast<int32_t>(sd::kTriWaitLimit)) return SD_ERR_INVALID_ARG;
+  g_tri_wait_limit.store(polls < 0 ? sd::kTriWaitLimit : static_cast<uint32_t>(polls), std::memory_order_relaxed);
+  return SD_OK;
+}
+
 sd_status sd_get_device_errors(uint32_t* bits, int32_t clear) {
   if (!bits) return SD_ERR_INVALID_ARG;
   sd_status s = cuda_check(cudaDeviceSynchronize());
@@ -843,18 +855,26 @@ constexpr int kNoallocMaxDevices = 64;
 std::mutex g_noalloc_mutex;
 int32_t* g_noalloc_addr[kNoallocMaxDevices] = {};
 
-// The current device's address of g_noalloc_scores (looked up on first use).
-sd_status noalloc_scores_for_current_device(int32_t** out) {
+// The current device's address of g_noalloc_scores. Outside stream capture it
+// is looked up again on every call (a device reset reloads the module at
+// another address, so a remembered one could be stale); under capture the
+// remembered address is used, since a lookup could load the module.
+sd_status noalloc_scores_for_current_device(cudaStream_t st, int32_t** out) {
   int dev = 0;
   sd_status s = cuda_check(cudaGetDevice(&dev));
   if (s != SD_OK) return s;
   if (dev < 0 || dev >= kNoallocMaxDevices) return SD_ERR_UNSUPPORTED;
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  s = cuda_check(cudaStreamIsCapturing(st, &cap));
+  if (s != SD_OK) return s;
   std::lock_guard<std::mutex> lock(g_noalloc_mutex);
-  if (g_noalloc_addr[dev] == nullptr) {
+  if (cap == cudaStreamCaptureStatusNone) {
     void* p = nullptr;
     s = cuda_check(cudaGetSymbolAddress(&p, g_noalloc_scores));
     if (s != SD_OK) return s;
     g_noalloc_addr[dev] = static_cast<int32_t*>(p);
+  } else if (g_noalloc_addr[dev] == nullptr) {
+    return SD_ERR_INVALID_ARG;  // first call on this device under capture
   }
   *out = g_noalloc_addr[dev];
   return SD_OK;
@@ -872,7 +892,7 @@ extern "C" sd_status sd_indexer_topk_noalloc(const int8_t* qi, const int32_t* w,
   if (s != SD_OK) return s;
   if ((size_t)B * pd.kv_heads * (size_t)max_seqlen > (size_t)SD_NOALLOC_MAX_SCORES) return SD_ERR_WORKSPACE;
   int32_t* scores = nullptr;
-  s = noalloc_scores_for_current_device(&scores);
+  s = noalloc_scores_for_current_device(static_cast<cudaStream_t>(stream), &scores);
   if (s != SD_OK) return s;
   // Scores are written for every t < seqlens[b] before top-k reads them, so
   // nothing left over from an earlier call is ever read.

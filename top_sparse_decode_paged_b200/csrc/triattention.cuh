@@ -284,13 +284,16 @@ constexpr uint32_t kTriWaitLimit = 1u << 22;
 // increasing order, so the smallest unfinished unit never waits on a unit
 // that has not started; no dependent launch is triggered early, so no later
 // kernel takes an SM slot while units wait. Tokens already in place
-// (source == destination) are skipped. A wait that runs out sets
-// SD_DEVERR_TIMEOUT and skips that unit's writes.
+// (source == destination) are skipped. A wait gives up after `wait_limit`
+// polls (kTriWaitLimit unless a test lowers it; 0 gives up at once): it sets
+// SD_DEVERR_TIMEOUT and that unit skips its writes. No copy is in flight at
+// that point (step 1 has completed), so the unit simply moves on.
 __global__ void __launch_bounds__(kTriCompactThreads) tri_compact_kernel(
     uint8_t* __restrict__ k_pages, uint8_t* __restrict__ v_pages, const int32_t* __restrict__ block_table,
     const int32_t* __restrict__ seqlens, const int32_t* __restrict__ sel, int rows_per_req, int page_size,
     int max_pages, int num_pages, int seqlen_cap, int n_sink, int n_recent, int budget, int part, int row_bytes,
-    int chunk, int n_chunks, int n_rows, int32_t* __restrict__ flags, int32_t* __restrict__ new_seqlens) {
+    int chunk, int n_chunks, int n_rows, int32_t* __restrict__ flags, int32_t* __restrict__ new_seqlens,
+    uint32_t wait_limit) {
   pdl_wait();
   __shared__ __align__(16) uint8_t buf[kTriChunkBytes];
   __shared__ long long src_off[kTriMaxChunkTokens], dst_off[kTriMaxChunkTokens];
@@ -371,7 +374,7 @@ __global__ void __launch_bounds__(kTriCompactThreads) tri_compact_kernel(
       const int32_t* f = flags + (size_t)r * n_chunks + cc;
       uint32_t it = 0;
       int v = 0;
-      for (; it < kTriWaitLimit; ++it) {
+      for (; it < wait_limit; ++it) {
         asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(f) : "memory");
         if (v) break;
         __nanosleep(64);

@@ -142,6 +142,20 @@ def _blas_threads():
         return os.cpu_count() or 1
 
 
+def _host():
+    """The host the oracle ran on: logical CPUs and the CPU model."""
+    model = "unknown"
+    try:
+        with open("/proc/cpuinfo") as f:
+            for ln in f:
+                if ln.startswith("model name"):
+                    model = ln.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return {"nproc": os.cpu_count(), "cpu_model": model}
+
+
 def cpu_baseline(name: str, budget_s: float = 15.0):
     """The oracle as it stands on a bounded sample: requests are added until the
     sample has taken about budget_s seconds of host time."""
@@ -154,10 +168,16 @@ def cpu_baseline(name: str, budget_s: float = 15.0):
         spent += time.perf_counter() - t0
         done += 1
     return {"value": done / spent, "unit": "queries/s", "cores": _blas_threads(), "kind": "oracle",
-            "sample": f"{done} of {wl.seqlens.shape[0]} requests of {name}, {spent:.1f} s host time"}
+            "sample": f"{done} of {wl.seqlens.shape[0]} requests of {name}, {spent:.1f} s host time",
+            "threads": "the int and fp64 matmuls use `cores` BLAS threads; the lexsort top-k and the attention "
+                       "loops run on one thread", **_host()}
 
 
 def bench_reference(args, rank, world):
+    """The oracle, unchanged, on the host cores. A step is the oracle's decode
+    step over a fixed sample of the batch's requests (the full batch would take
+    minutes per step); ms_per_step is the time of that sample, and the value
+    is the requests it decoded per second."""
     if rank != 0:
         return
     n_steps = args.steps
@@ -168,23 +188,28 @@ def bench_reference(args, rank, world):
         t = run_oracle_sample(wl, per_step)
         if i >= args.warmup:
             times.append(t)
-    ms = 1e3 * float(np.mean(times)) / per_step * wl.seqlens.shape[0]
+    ms = 1e3 * float(np.mean(times))
     value = per_step / float(np.mean(times))
+    sample = f"the first {per_step} of {wl.seqlens.shape[0]} requests of {args.config} per step"
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "queries/s", "n_gpus": world,
         "steps": n_steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "int64/f64", "data": "synthetic",
-        "config": _config(wl.spec, "host memory (CPU oracle)"),
+        "config": _config(wl.spec),
+        "l2": "host memory (CPU oracle)",
+        "queries_per_step": per_step,
         "cpu_baseline": {"value": value, "unit": "queries/s", "cores": _blas_threads(), "kind": "oracle",
-                         "sample": f"{per_step} requests per step of {args.config}"},
+                         "sample": sample,
+                         "threads": "the int and fp64 matmuls use `cores` BLAS threads; the lexsort top-k and the "
+                                    "attention loops run on one thread", **_host()},
         "e2e": {"value": value, "unit": "queries/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
 
 
-def _config(s: W.Spec, l2: str):
+def _config(s: W.Spec):
     cfg = {"workload": s.name, "B": s.B, "page": s.page_size, "kv_heads": s.G, "Hi": s.Hi, "Di": s.Di,
-           "k": s.k, "H": s.H, "Dk": s.Dk, "Dv": s.Dv, "l2": l2}
+           "k": s.k, "H": s.H, "Dk": s.Dk, "Dv": s.Dv}
     if s.seqlen is not None:
         cfg["seqlen"] = s.seqlen
     if s.ragged is not None:
@@ -408,7 +433,9 @@ def bench_ours(args, rank, world, local):
         "ms_per_step": step_ms,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "int8/bf16", "data": "synthetic",
-        "config": _config(s, "flushed before every step (256 MiB write, then 256 MiB read so the lines left are clean; outside the timed events)"),
+        "config": _config(s),
+        "l2": "flushed before every step (256 MiB write, then 256 MiB read so the lines left are clean; outside the "
+              "timed events)",
         "timing": ("CUDA graph of one sd_decode_step, replayed; the per-kernel split comes from a second graph with "
                    "stage events inside") if not args.no_graph else "eager sd_decode_step calls",
         "hbm_gbs_step": alg / (step_ms * 1e-3) / 1e9,
@@ -516,7 +543,8 @@ def bench_layers(args, rank, world, local):
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "layers": n,
         "ms_per_step": ms_together, "ms_per_step_separate_calls": ms_apart,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": _config(s, "flushed before every step (256 MiB write, then 256 MiB read; outside the timed events)"),
+        "config": _config(s),
+        "l2": "flushed before every step (256 MiB write, then 256 MiB read; outside the timed events)",
         "roofline": {"kernel": "attn (all layers, with combine)", "bound": "hbm", "achieved": achieved, "peak": peak,
                      "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak, "traffic": None,
                      "algorithmic_bytes_per_launch": nbytes, "ms_per_launch": ms_together},
@@ -615,7 +643,8 @@ def bench_csr(args, rank, world, local):
         "warmup": args.warmup, "block_size": bs, "selected_tokens": sel_tokens,
         "ms_per_step": ms_csr, "ms_per_step_padded_topk_selection": ms_pad,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": _config(s, "flushed before every step (256 MiB write, then 256 MiB read; outside the timed events)"),
+        "config": _config(s),
+        "l2": "flushed before every step (256 MiB write, then 256 MiB read; outside the timed events)",
         "roofline": {"kernel": "csr expansion + attn + combine", "bound": "hbm", "achieved": achieved, "peak": peak,
                      "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak, "traffic": None,
                      "algorithmic_bytes_per_launch": nbytes, "ms_per_launch": ms_csr},
@@ -705,7 +734,8 @@ def bench_hint(args, rank, world, local):
         "value": res["perturbed"]["topk"], "unit": "ms", "higher_is_better": False, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "hint_overlap_with_selection": same,
         "stage_ms": res, "data": "synthetic",
-        "config": _config(s, "flushed before every step (256 MiB write, then 256 MiB read; outside the timed events)"),
+        "config": _config(s),
+        "l2": "flushed before every step (256 MiB write, then 256 MiB read; outside the timed events)",
     }
     if rank == 0:
         print(json.dumps(line), flush=True)
@@ -825,6 +855,33 @@ def bench_tri(args, rank, world, local):
         print(json.dumps(line), flush=True)
 
 
+def _spawned_rank(rank: int, world: int, port: int, argv):
+    """One rank started by _launch_ranks (torchrun's environment, set by hand)."""
+    os.environ.update(RANK=str(rank), LOCAL_RANK=str(rank), WORLD_SIZE=str(world), MASTER_ADDR="127.0.0.1",
+                      MASTER_PORT=str(port))
+    sys.argv = [sys.argv[0]] + list(argv)
+    main()
+
+
+def _launch_ranks(n: int, argv) -> int:
+    """`--gpus N` without torchrun: starts N ranks (spawned processes, one per
+    GPU) with the same arguments and returns the first non-zero exit code."""
+    import multiprocessing as mp
+    import socket
+    with socket.socket() as so:
+        so.bind(("127.0.0.1", 0))
+        port = so.getsockname()[1]
+    ctx = mp.get_context("spawn")
+    procs = [ctx.Process(target=_spawned_rank, args=(r, n, port, argv)) for r in range(n)]
+    for p in procs:
+        p.start()
+    rc = 0
+    for p in procs:
+        p.join()
+        rc = rc or (p.exitcode or 0)
+    return rc
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -847,7 +904,11 @@ def main():
     ap.add_argument("--tri-layers", type=int, default=1, help="with --tri: layers sharing the block table")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
+    if "WORLD_SIZE" not in os.environ and args.gpus > 1:
+        sys.exit(_launch_ranks(args.gpus, sys.argv[1:]))
     rank, world, local = _dist_env()
+    if world != args.gpus:
+        sys.exit(f"bench.py: --gpus {args.gpus} but WORLD_SIZE={world}")
     if world > 1:
         import datetime
         import torch

@@ -38,3 +38,29 @@ def test_two_gloo_ranks_shard_and_take_max(tmp_path):
     assert (r0["shape"] == r1["shape"]).all()              # of the same shape
     assert not np.array_equal(r0["qi"], r1["qi"])
     assert float(r0["t"]) == float(r1["t"]) == 2.0         # MAX over ranks
+
+
+def test_gpus_flag_starts_that_many_ranks():
+    """`bench.py --gpus 2` without torchrun starts two ranks itself: the
+    reference arm (CPU, gloo) prints one line from rank 0 with n_gpus 2, and
+    the other rank exits 0 without output. A --gpus that contradicts
+    WORLD_SIZE is refused."""
+    import json
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = {k: v for k, v in os.environ.items() if k not in ("RANK", "WORLD_SIZE", "LOCAL_RANK")}
+    r = subprocess.run([sys.executable, "bench.py", "--gpus", "2", "--impl", "reference", "--config", "tiny",
+                        "--steps", "1", "--warmup", "3"], cwd=root, env=env, capture_output=True, text=True,
+                       timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1
+    line = json.loads(lines[0])
+    assert line["impl"] == "reference" and line["n_gpus"] == 2
+    assert line["ms_per_step"] * line["steps"] < 600e3
+    env2 = dict(env, WORLD_SIZE="1", RANK="0", LOCAL_RANK="0")
+    r2 = subprocess.run([sys.executable, "bench.py", "--gpus", "2", "--impl", "reference", "--config", "tiny",
+                         "--steps", "1", "--warmup", "3"], cwd=root, env=env2, capture_output=True, text=True,
+                        timeout=600)
+    assert r2.returncode != 0 and "WORLD_SIZE" in r2.stderr

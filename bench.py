@@ -62,10 +62,14 @@ def _dist_env():
     return rank, world, local
 
 
+BATCH_OVERRIDE = None  # --batch: requests per rank (profiling a reduced batch of the same workload)
+
+
 def rank_spec(name: str, rank: int) -> W.Spec:
     """Each rank draws its own batch of the same shape (weak scaling)."""
-    base = W.spec(name)
-    return W.spec(name, seed=base.seed + 1000 * rank) if rank else base
+    over = {} if BATCH_OVERRIDE is None else {"B": BATCH_OVERRIDE}
+    base = W.spec(name, **over)
+    return W.spec(name, seed=base.seed + 1000 * rank, **over) if rank else base
 
 
 def max_over_ranks(value: float, world: int) -> float:
@@ -181,7 +185,7 @@ def bench_reference(args, rank, world):
     if rank != 0:
         return
     n_steps = args.steps
-    wl = W.make(W.spec(args.config))
+    wl = W.make(rank_spec(args.config, 0))
     times = []
     per_step = max(1, min(wl.seqlens.shape[0], 2))
     for i in range(args.warmup + n_steps):
@@ -418,7 +422,8 @@ def bench_ours(args, rank, world, local):
         ms = stage_ms[stage]
         achieved = nbytes / (ms * 1e-3) / 1e9 if ms > 0 else None
         tv = NCU_TRAFFIC.get((s.name, stage))
-        traffic = tv[1] if tv and tv[0] == lib_version and rank_spec(args.config, 0).seed == s.seed else None
+        traffic = (tv[1] if tv and tv[0] == lib_version and rank_spec(args.config, 0).seed == s.seed
+                   and BATCH_OVERRIDE is None else None)
         return {"kernel": stage, "bound": "hbm", "achieved": achieved, "peak": peak, "peak_kind": peak_kind,
                 "unit": "GB/s", "frac": (achieved / peak) if achieved else None, "traffic": traffic,
                 "algorithmic_bytes_per_launch": nbytes, "ms_per_launch": ms}
@@ -902,7 +907,11 @@ def main():
     ap.add_argument("--tri-mode", default="union", choices=["union", "per_head", "per_layer_per_head"],
                     help="with --tri: one selection per request, per KV head, or per (layer, KV head)")
     ap.add_argument("--tri-layers", type=int, default=1, help="with --tri: layers sharing the block table")
+    ap.add_argument("--batch", type=int, default=0,
+                    help="requests per rank instead of the workload's (a reduced batch for profiling)")
     args = ap.parse_args()
+    global BATCH_OVERRIDE
+    BATCH_OVERRIDE = args.batch if args.batch > 0 else None
     args.warmup = max(args.warmup, 3)
     if "WORLD_SIZE" not in os.environ and args.gpus > 1:
         sys.exit(_launch_ranks(args.gpus, sys.argv[1:]))

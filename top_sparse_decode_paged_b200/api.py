@@ -47,11 +47,14 @@ class SdError(RuntimeError):
 _lib = None
 
 
-def load_library(path: str = LIB_PATH):
-    """Loads libsd.so once and declares the exported signatures."""
+def load_library(path: Optional[str] = None):
+    """Loads libsd.so once and declares the exported signatures. The path is
+    ``path``, else the ``SD_LIBRARY`` environment variable, else the in-tree
+    build."""
     global _lib
     if _lib is not None:
         return _lib
+    path = path or os.environ.get("SD_LIBRARY") or LIB_PATH
     if not os.path.exists(path):
         raise RuntimeError(f"libsd.so not built ({path}); run `python -m top_sparse_decode_paged_b200.build`")
     lib = ctypes.CDLL(path)

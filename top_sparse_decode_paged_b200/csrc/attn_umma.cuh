@@ -46,10 +46,12 @@
 // covers parts of several requests writes one partial (O, m, l) per request.
 // The combine kernel merges them.
 //
-// Roles (320 threads): warps 0-3 copy (thread 0 also loads Q by TMA), warps
+// Roles (352 threads): warps 0-3 copy (thread 0 also loads Q by TMA), warps
 // 4-7 run the softmax, rescale and write partials (warp w owns TMEM lanes
-// 32*(w%4)..+31), warp 8 issues the MMAs as their inputs become ready, warp 9
-// streams row ids. Every wait is bounded (a timeout flags SD_DEVERR_TIMEOUT).
+// 32*(w%4)..+31), warp 8 owns tensor memory and issues the S products, warp
+// 10 issues the P V products (each issuer blocks on its own inputs, in
+// order), warp 9 streams row ids and has their rows prefetched into L2.
+// Every wait is bounded (a timeout flags SD_DEVERR_TIMEOUT).
 #pragma once
 
 #include "sm100.cuh"
@@ -69,11 +71,10 @@ constexpr int kAuQChunkBytes = kAuHalfHeads * 128;        // 8 KB
 constexpr int kAuQBytes = kAuChunks * kAuQChunkBytes;     // 72 KB
 constexpr int kAuPBytes = kAuHalfHeads * 128;             // 8 KB: 64 head rows of up to 64 tokens
 constexpr int kAuBufs = 2;
-constexpr int kAuThreads = 320;
-constexpr int kAuRidSlots = 4;             // row-id lookahead (tiles)
+constexpr int kAuThreads = 352;
+constexpr int kAuRidSlots = 4;             // row-id lookahead (tiles); rows are prefetched into L2 as their ids enter the ring
 constexpr int kAuRanges = 74;              // CTA pairs: 148 CTAs, one per SM
 constexpr float kAuRescaleLog2 = 8.0f;     // lazy rescale threshold (log2 units)
-constexpr int kMaxTopK = 2048;             // largest k the library accepts
 static_assert(kAuTile % 32 == 0 && kAuTile <= 64, "tile of 32 or 64 tokens");
 
 // Row-id slots per request in the resolved-row array (whole tiles).
@@ -84,7 +85,7 @@ struct AttnUmmaLayout {
   static constexpr int kOffRing = kOffQ + kAuQBytes;
   static constexpr int kOffP = kOffRing + kAuBufs * kAuTileBytes;
   static constexpr int kOffBar = kOffP + kAuPBytes;
-  static constexpr int kNumBars = 2 * kAuBufs + 9 + 2 * kAuRidSlots;
+  static constexpr int kNumBars = 2 * kAuBufs + 10 + 2 * kAuRidSlots;
   static constexpr int kOffRid = kOffBar + 8 * kNumBars;             // [slots][tile] pool row ids (-1: skip)
   static constexpr int kOffAlpha = kOffRid + 4 * kAuTile * kAuRidSlots;  // [64] rescale factors
   static constexpr int kOffMisc = kOffAlpha + 4 * kAuHalfHeads;
@@ -203,8 +204,9 @@ __global__ void __launch_bounds__(kAuThreads, 1) attn_mla_umma_kernel(
   uint64_t* s_free = q_full + 4;                 // [2] the four softmax warps have read S
   uint64_t* p_full = q_full + 6;                 // the four epilogue warps: P written, O rescaled/read out
   uint64_t* pv_done = q_full + 7;                // MMA commit after P V
-  uint64_t* mma_fin = q_full + 8;                // MMA commit at exit
-  uint64_t* rid_full = q_full + 9;               // [slots] 32 row-id lanes (cp.async)
+  uint64_t* mma_fin = q_full + 8;                // S issuer's commit at exit
+  uint64_t* pv_fin = q_full + 9;                 // P V issuer's commit at exit
+  uint64_t* rid_full = q_full + 10;              // [slots] 32 row-id lanes (cp.async)
   uint64_t* rid_empty = rid_full + kAuRidSlots;  // [slots] 4 copy warps + the epilogue
   int32_t* rid = reinterpret_cast<int32_t*>(smem + Lay::kOffRid);
   float* alpha_s = reinterpret_cast<float*>(smem + Lay::kOffAlpha);
@@ -231,6 +233,7 @@ __global__ void __launch_bounds__(kAuThreads, 1) attn_mla_umma_kernel(
     sm100::mbar_init(p_full, 4);
     sm100::mbar_init(pv_done, 1);
     sm100::mbar_init(mma_fin, 1);
+    sm100::mbar_init(pv_fin, 1);
     for (int i = 0; i < kAuRidSlots; ++i) {
       sm100::mbar_init(&rid_full[i], 32);
       sm100::mbar_init(&rid_empty[i], 5);
@@ -256,6 +259,7 @@ __global__ void __launch_bounds__(kAuThreads, 1) attn_mla_umma_kernel(
   const long long total = attn_total_tiles(seqlens, B, seqlen_cap, k, breq);
   const long long first = total * range / n_ranges;
   const long long count = total * (range + 1) / n_ranges - first;
+  if (threadIdx.x == 0) SD_PROBE_MARK(3, 0, count);
 
   if (warp < 4) {
     // ------------------------------ copies ------------------------------
@@ -310,6 +314,7 @@ __global__ void __launch_bounds__(kAuThreads, 1) attn_mla_umma_kernel(
         for (int cc = 0; cc < kAuChunks; ++cc) cp_async_16(dst + cc * kAuChunkBytes, src + cc * 64, rw >= 0 ? 16 : 0);
       }
       sm100::cp_async_arrive_noinc(&tile_full[slot]);
+      if (pt == 0) SD_PROBE_MARK(3, 1, n);
       ++n;
       c.next(seqlens, B, seqlen_cap, k);
     }
@@ -352,10 +357,12 @@ __global__ void __launch_bounds__(kAuThreads, 1) attn_mla_umma_kernel(
       ok = sm100::named_bar_and(1, 128, ok);
       if (!ok) { *abort_flag = 1; break; }
       if (threadIdx.x == 128) sm100::mbar_arrive(&rid_empty[rs]);
+      if (threadIdx.x == 128) SD_PROBE_MARK(3, 6, j);
       sm100::tc_fence_after();
       uint32_t r[4 * kReps];
       sm100::tmem_ld_16x256b(tm_s + kAuTile * static_cast<uint32_t>(j & 1) + lane_base, r);
       sm100::tmem_ld_wait();
+      if (threadIdx.x == 128) SD_PROBE_MARK(3, 7, j);
       sm100::tc_fence_before();
       __syncwarp();
       if (lane == 0) sm100::mbar_arrive(&s_free[j & 1]);
@@ -402,6 +409,7 @@ __global__ void __launch_bounds__(kAuThreads, 1) attn_mla_umma_kernel(
       // earlier tiles of this request are in O: rescale when any head's
       // reference moved (alpha_s published by the barrier)
       const bool rescale = sm100::named_bar_or(2, 128, need && !seg_first);
+      if (threadIdx.x == 128) SD_PROBE_MARK(3, 8, j);
       // O and the P buffer are free once the previous P V has completed
       if (j > 0) {
         bool okp = sm100::mbar_wait(pv_done, static_cast<uint32_t>((j - 1) & 1)) && !*abort_flag;
@@ -409,6 +417,7 @@ __global__ void __launch_bounds__(kAuThreads, 1) attn_mla_umma_kernel(
         if (!okp) { *abort_flag = 1; break; }
         sm100::tc_fence_after();
       }
+      if (threadIdx.x == 128) SD_PROBE_MARK(3, 9, j);
       if (rescale) {
 #pragma unroll 1
         for (int q8 = 0; q8 < 8; ++q8) {  // 4 value blocks x 2 halves of 32 head columns
@@ -438,6 +447,7 @@ __global__ void __launch_bounds__(kAuThreads, 1) attn_mla_umma_kernel(
       sm100::tc_fence_before();
       __syncwarp();
       if (lane == 0) sm100::mbar_arrive(p_full);
+      if (threadIdx.x == 128) SD_PROBE_MARK(3, 3, j);
 
       const int this_b = c.b;
       c.next(seqlens, B, seqlen_cap, k);
@@ -470,95 +480,103 @@ __global__ void __launch_bounds__(kAuThreads, 1) attn_mla_umma_kernel(
       ++j;
     }
   } else if (warp == 8) {
-    // ------------------------------ MMA issue ------------------------------
+    // ------------------------------ S issue ------------------------------
+    // S(i) needs tile i landed (and its request's Q) and S buffer i % 2 read
+    // out by the softmax. A second thread (warp 10) issues the P V products,
+    // so that neither kind waits behind the other's inputs; each issuer
+    // blocks on its own barriers in order.
     if (sm100::elect_one()) {
       constexpr uint32_t idesc_s = sm100::idesc_bf16(kAuHalfHeads, kAuTile, false, false);
-      constexpr uint32_t idesc_pv = sm100::idesc_bf16(128, kAuHalfHeads, true, false);
-      const uint32_t qa = smem_u32(qbuf), pa = smem_u32(pbuf);
-      // Issue S and P V in the order their inputs become ready: S(i) needs
-      // tile i landed (and its request's Q) and S buffer i%2 read out;
-      // P V(j) needs P(j). Polling both keeps P V(j) from waiting for the
-      // next tile's rows, so a tile buffer is released as soon as its own
-      // P V is done.
-      AttnCursor cs, cp;
+      const uint32_t qa = smem_u32(qbuf);
+      AttnCursor cs;
       cs.init(seqlens, B, seqlen_cap, k, first, count, breq);
-      cp.init(seqlens, B, seqlen_cap, k, first, count, breq);
-      long long is = 0, ip = 0;
-      int q_seen = 0, prev_bs = -1, prev_bp = -1;
-      uint32_t idle = 0;
+      int q_seen = 0, prev_bs = -1;
       bool ok = true;
-      while (ip < count && ok) {
-        bool progressed = false;
-        if (is < count) {
-          const bool seg_first = cs.b != prev_bs;
-          const int slot = static_cast<int>(is % kAuBufs);
-          const int sb = static_cast<int>(is & 1);
-          const bool ready = (!seg_first || sm100::mbar_test_wait(q_full, static_cast<uint32_t>(q_seen & 1))) &&
-                             sm100::mbar_test_wait(&tile_full[slot], static_cast<uint32_t>((is / kAuBufs) & 1)) &&
-                             (is < 2 || sm100::mbar_test_wait(&s_free[sb], static_cast<uint32_t>(((is - 2) >> 1) & 1)));
-          if (ready) {
-            sm100::tc_fence_after();
-            if (seg_first) ++q_seen;
-            prev_bs = cs.b;
-            // S = Q K^T (M = 64 heads) over the nine 64-column chunks
-            const uint32_t ta = smem_u32(ring + slot * kAuTileBytes);
+      for (long long is = 0; is < count && ok; ++is) {
+        const bool seg_first = cs.b != prev_bs;
+        const int slot = static_cast<int>(is % kAuBufs);
+        const int sb = static_cast<int>(is & 1);
+        ok = (!seg_first || sm100::mbar_wait(q_full, static_cast<uint32_t>(q_seen & 1))) &&
+             sm100::mbar_wait(&tile_full[slot], static_cast<uint32_t>((is / kAuBufs) & 1)) &&
+             (is < 2 || sm100::mbar_wait(&s_free[sb], static_cast<uint32_t>(((is - 2) >> 1) & 1))) && !*abort_flag;
+        if (!ok) break;
+        sm100::tc_fence_after();
+        if (seg_first) ++q_seen;
+        prev_bs = cs.b;
+        // S = Q K^T (M = 64 heads) over the nine 64-column chunks
+        const uint32_t ta = smem_u32(ring + slot * kAuTileBytes);
 #pragma unroll
-            for (int cc = 0; cc < kAuChunks; ++cc)
+        for (int cc = 0; cc < kAuChunks; ++cc)
 #pragma unroll
-              for (int kk = 0; kk < 4; ++kk)
-                sm100::mma_bf16_ss(tm_s + kAuTile * sb, sm100::smem_desc_k_sw128(qa + cc * kAuQChunkBytes + 32 * kk),
-                                   sm100::smem_desc_k_sw128(ta + cc * kAuChunkBytes + 32 * kk), idesc_s,
-                                   (cc | kk) != 0);
-            sm100::mma_commit(&s_full[sb]);
-            const int this_b = cs.b;
-            cs.next(seqlens, B, seqlen_cap, k);
-            if (is + 1 >= count || cs.b != this_b) sm100::mma_commit(q_empty);
-            ++is;
-            progressed = true;
-          }
-        }
-        if (ip < is && sm100::mbar_test_wait(p_full, static_cast<uint32_t>(ip & 1))) {
-          sm100::tc_fence_after();
-          const bool seg_first = cp.b != prev_bp;
-          prev_bp = cp.b;
-          const int slot = static_cast<int>(ip % kAuBufs);
-          const uint32_t ta = smem_u32(ring + slot * kAuTileBytes);
-          // O^T += V^T P^T (chunks 2v, 2v+1 are value block v)
-#pragma unroll
-          for (int v = 0; v < kAuVBlocks; ++v)
-#pragma unroll
-            for (int kk = 0; kk < kAuTile / 16; ++kk)
-              sm100::mma_bf16_ss(tm_o + 64 * v,
-                                 sm100::smem_desc_mn_sw128(ta + 2 * v * kAuChunkBytes + kk * 2048, kAuChunkBytes, 1024),
-                                 sm100::smem_desc_k_sw128(pa + 32 * kk), idesc_pv, !(seg_first && kk == 0));
-          sm100::mma_commit(&tile_empty[slot]);
-          sm100::mma_commit(pv_done);
-          cp.next(seqlens, B, seqlen_cap, k);
-          ++ip;
-          progressed = true;
-        }
-        if (progressed) {
-          idle = 0;
-        } else if (++idle >= sm100::kWaitLimit || *abort_flag) {
-          if (!*abort_flag) raise_error(SD_DEVERR_TIMEOUT);
-          ok = false;
-        } else {
-          __nanosleep(32);  // leave issue slots to the epilogue warp on this scheduler
-        }
+          for (int kk = 0; kk < 4; ++kk)
+            sm100::mma_bf16_ss(tm_s + kAuTile * sb, sm100::smem_desc_k_sw128(qa + cc * kAuQChunkBytes + 32 * kk),
+                               sm100::smem_desc_k_sw128(ta + cc * kAuChunkBytes + 32 * kk), idesc_s,
+                               (cc | kk) != 0);
+        sm100::mma_commit(&s_full[sb]);
+        SD_PROBE_MARK(3, 2, is);
+        const int this_b = cs.b;
+        cs.next(seqlens, B, seqlen_cap, k);
+        if (is + 1 >= count || cs.b != this_b) sm100::mma_commit(q_empty);
       }
       if (!ok) *abort_flag = 1;
       // every issued MMA completes before tensor memory is released
       sm100::mma_commit(mma_fin);
       sm100::mbar_wait(mma_fin, 0);
     }
-  } else {
+  } else if (warp == 10) {
+    // ----------------------------- P V issue -----------------------------
+    // P V(j) needs P(j) written (which follows S(j) and P V(j - 1)).
+    if (sm100::elect_one()) {
+      constexpr uint32_t idesc_pv = sm100::idesc_bf16(128, kAuHalfHeads, true, false);
+      const uint32_t pa = smem_u32(pbuf);
+      AttnCursor cp;
+      cp.init(seqlens, B, seqlen_cap, k, first, count, breq);
+      int prev_bp = -1;
+      bool ok = true;
+      for (long long ip = 0; ip < count && ok; ++ip) {
+        ok = sm100::mbar_wait(p_full, static_cast<uint32_t>(ip & 1)) && !*abort_flag;
+        if (!ok) break;
+        sm100::tc_fence_after();
+        const bool seg_first = cp.b != prev_bp;
+        prev_bp = cp.b;
+        const int slot = static_cast<int>(ip % kAuBufs);
+        const uint32_t ta = smem_u32(ring + slot * kAuTileBytes);
+        // O^T += V^T P^T (chunks 2v, 2v+1 are value block v)
+#pragma unroll
+        for (int v = 0; v < kAuVBlocks; ++v)
+#pragma unroll
+          for (int kk = 0; kk < kAuTile / 16; ++kk)
+            sm100::mma_bf16_ss(tm_o + 64 * v,
+                               sm100::smem_desc_mn_sw128(ta + 2 * v * kAuChunkBytes + kk * 2048, kAuChunkBytes, 1024),
+                               sm100::smem_desc_k_sw128(pa + 32 * kk), idesc_pv, !(seg_first && kk == 0));
+        sm100::mma_commit(&tile_empty[slot]);
+        sm100::mma_commit(pv_done);
+        SD_PROBE_MARK(3, 4, ip);
+        cp.next(seqlens, B, seqlen_cap, k);
+      }
+      if (!ok) *abort_flag = 1;
+      sm100::mma_commit(pv_fin);
+      sm100::mbar_wait(pv_fin, 0);
+    }
+  } else if (warp == 9) {
     // ------------------------------ row ids ------------------------------
     // Streams each tile's resolved pool rows into a small ring, kAuRidSlots
-    // tiles ahead of the copies and the softmax.
+    // tiles ahead of the copies and the softmax, and asks L2 to prefetch
+    // those rows (one bulk prefetch per 1152-byte row) as their ids enter the
+    // ring, so that the gathers, a few tiles later, find them in L2 instead
+    // of waiting for HBM. The ids a prefetch needs are loaded one iteration
+    // ahead, so their latency overlaps the wait for a free ring slot.
     AttnCursor c;
     c.init(seqlens, B, seqlen_cap, k, first, count, breq);
     long long n = 0;
     bool ok = true;
+    int ids[kAuTileWords];
+    auto load_ids = [&](const AttnCursor& cc) {
+      const int32_t* src = rows + (size_t)(cc.b % breq) * kpad + cc.tile * kAuTile;
+#pragma unroll
+      for (int w = 0; w < kAuTileWords; ++w) ids[w] = __ldg(src + 32 * w + lane);
+    };
+    if (c.valid()) load_ids(c);
     while (c.valid() && ok) {
       const int rs = static_cast<int>(n % kAuRidSlots);
       ok = sm100::mbar_wait(&rid_empty[rs], static_cast<uint32_t>((n / kAuRidSlots) & 1) ^ 1) && !*abort_flag;
@@ -567,8 +585,13 @@ __global__ void __launch_bounds__(kAuThreads, 1) attn_mla_umma_kernel(
 #pragma unroll
       for (int w = 0; w < kAuTileWords; ++w) cp_async_4(&rid[rs * kAuTile + 32 * w + lane], src + 32 * w + lane);
       sm100::cp_async_arrive_noinc(&rid_full[rs]);
+      const __nv_bfloat16* kv = kvl.p[c.b / breq];
+#pragma unroll
+      for (int w = 0; w < kAuTileWords; ++w)
+        if (ids[w] >= 0) sm100::prefetch_l2_bulk(kv + (long long)ids[w] * kAuDk, kAuDk * 2);
       ++n;
       c.next(seqlens, B, seqlen_cap, k);
+      if (c.valid()) load_ids(c);
     }
     cp_async_wait<0>();
     if (!ok) *abort_flag = 1;
@@ -577,99 +600,109 @@ __global__ void __launch_bounds__(kAuThreads, 1) attn_mla_umma_kernel(
   sm100::tc_fence_before();
   __syncthreads();
   sm100::tc_fence_after();
+  if (threadIdx.x == 0) SD_PROBE_MARK(3, 5, 0);
   if (warp == 8) {
     __syncwarp();
     sm100::tmem_dealloc(tmem, 512);
   }
 }
 
-// Merges the per-range partials into the bf16 output. One block per (request,
-// pair of heads), 128 threads per head of 4 value columns each. Warp 0 lists
-// the ranges that cover the request: a request has at most ceil(k / kAuTile)
-// tiles, and tile i of the list lies in range ((i + 1) * n_ranges - 1) /
-// total. Each thread then issues the loads of all its partials together.
+// Merges the per-range partials into the bf16 output: one warp per (request,
+// head), 16 heads per block, one wave. The ranges that cover a request follow
+// from the tile list in closed form: tile i lies in range ((i + 1) *
+// n_ranges - 1) / total, so with total >= n_ranges a request's tiles
+// [t0, t0 + n) span the consecutive ranges range(t0) .. range(t0 + n - 1),
+// and with fewer tiles than ranges each tile has a range of its own. Lane s
+// loads the (m, l) of segments s and s + 32 for the head; each lane then
+// merges 16 contiguous value columns over the segments.
 constexpr int kAuMaxSeg = kMaxTopK / kAuTile;
-constexpr int kAuCombineHeads = 2;
+constexpr int kAuCombineHeads = 16;  // heads (warps) per block
+constexpr int kAuSegPerLane = (kAuMaxSeg + 31) / 32;
 
-__global__ void __launch_bounds__(128 * kAuCombineHeads) attn_mla_umma_combine_kernel(
+__global__ void __launch_bounds__(32 * kAuCombineHeads) attn_mla_umma_combine_kernel(
     const float* __restrict__ part_o, const float2* __restrict__ part_ml, const int32_t* __restrict__ seqlens,
     int B, int breq, int k, int seqlen_cap, int n_ranges, __nv_bfloat16* __restrict__ out, float* __restrict__ lse) {
   pdl_wait();  // inputs come from earlier work in the stream
   pdl_trigger();
+  if (threadIdx.x == 0 && (blockIdx.x & 15) == 0) SD_PROBE_MARK(4, 0, 0);
   constexpr int HG = kAuHeads / kAuCombineHeads;
   const int b = blockIdx.x / HG;
-  const int h = (blockIdx.x % HG) * kAuCombineHeads + (threadIdx.x >> 7);
-  __shared__ int seg_r[kAuMaxSeg];
-  __shared__ float2 ml_s[kAuCombineHeads][kAuMaxSeg];
-  __shared__ int nseg_s;
-  const int tid = threadIdx.x & 127, lane = threadIdx.x & 31;
-  if (threadIdx.x < 32) {
-    uint32_t before = 0, total = 0, mine = 0;
-    for (int i = lane; i < B; i += 32) {
-      int L = seqlens[i % breq];
-      L = L < 0 ? 0 : (L > seqlen_cap ? seqlen_cap : L);
-      const uint32_t n = static_cast<uint32_t>(ceil_div(min(k, L), kAuTile));
-      before += i < b ? n : 0;
-      mine += i == b ? n : 0;
-      total += n;
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      before += __shfl_xor_sync(0xffffffffu, before, o);
-      total += __shfl_xor_sync(0xffffffffu, total, o);
-      mine += __shfl_xor_sync(0xffffffffu, mine, o);
-    }
-    const uint32_t nr = static_cast<uint32_t>(n_ranges);
-    const int h0 = (blockIdx.x % HG) * kAuCombineHeads;
-    uint32_t carry = 0xffffffffu;  // range of the previous tile
-    int nseg = 0;
-    for (uint32_t base = 0; base < mine; base += 32) {
-      const uint32_t t = base + lane;
-      const bool has = t < mine;
-      const uint32_t r = has ? static_cast<uint32_t>(((unsigned long long)(before + t + 1) * nr - 1) / total)
-                             : 0xffffffffu;
-      uint32_t prev = __shfl_up_sync(0xffffffffu, r, 1);
-      if (lane == 0) prev = carry;
-      const bool head_of_seg = has && r != prev;
-      const uint32_t bal = __ballot_sync(0xffffffffu, head_of_seg);
-      const int at = nseg + __popc(bal & ((1u << lane) - 1u));
-      if (head_of_seg) {
-        seg_r[at] = static_cast<int>(r);
-#pragma unroll
-        for (int hh = 0; hh < kAuCombineHeads; ++hh) ml_s[hh][at] = part_ml[((size_t)r + b) * kAuHeads + h0 + hh];
-      }
-      nseg += __popc(bal);
-      carry = __shfl_sync(0xffffffffu, r, 31);
-    }
-    if (lane == 0) nseg_s = nseg;
+  const int h = (blockIdx.x % HG) * kAuCombineHeads + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  uint32_t before = 0, total = 0, mine = 0;
+  for (int i = lane; i < B; i += 32) {
+    int L = seqlens[i % breq];
+    L = L < 0 ? 0 : (L > seqlen_cap ? seqlen_cap : L);
+    const uint32_t n = static_cast<uint32_t>(ceil_div(min(k, L), kAuTile));
+    before += i < b ? n : 0;
+    mine += i == b ? n : 0;
+    total += n;
   }
-  __syncthreads();
-  const int nseg = nseg_s;
-  const float2* ml = ml_s[threadIdx.x >> 7];
-  const int d0 = 4 * tid;  // value columns d0..d0+3
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    before += __shfl_xor_sync(0xffffffffu, before, o);
+    total += __shfl_xor_sync(0xffffffffu, total, o);
+    mine += __shfl_xor_sync(0xffffffffu, mine, o);
+  }
+  const unsigned long long nr = static_cast<unsigned long long>(n_ranges);
+  auto range_of = [&](uint32_t i) { return static_cast<uint32_t>(((i + 1ull) * nr - 1ull) / total); };
+  uint32_t nseg = 0, r0 = 0;
+  if (mine > 0) {
+    r0 = range_of(before);
+    nseg = total >= nr ? range_of(before + mine - 1) - r0 + 1 : mine;
+  }
+  auto seg_range = [&](uint32_t sg) { return total >= nr ? r0 + sg : range_of(before + sg); };
+  float2 ml[kAuSegPerLane];
   float M = -INFINITY;
-  for (int jj = 0; jj < nseg; ++jj) M = fmaxf(M, ml[jj].x);
-  float denom = 0.f;
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 4
-  for (int jj = 0; jj < nseg; ++jj) {
-    const float2 m_l = ml[jj];
-    if (m_l.x == -INFINITY) continue;
-    const size_t slot = static_cast<size_t>(seg_r[jj]) + b;
-    const float wgt = exp2f(m_l.x - M);
-    denom += wgt * m_l.y;
-    const float4 o = *reinterpret_cast<const float4*>(part_o + (slot * kAuHeads + h) * kAuDv + d0);
-    acc.x += wgt * o.x;
-    acc.y += wgt * o.y;
-    acc.z += wgt * o.z;
-    acc.w += wgt * o.w;
+#pragma unroll
+  for (int q = 0; q < kAuSegPerLane; ++q) {
+    const uint32_t sg = static_cast<uint32_t>(lane + 32 * q);
+    ml[q] = sg < nseg ? part_ml[((size_t)seg_range(sg) + b) * kAuHeads + h] : make_float2(-INFINITY, 0.f);
+    M = fmaxf(M, ml[q].x);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+  float wgt[kAuSegPerLane], denom = 0.f;
+#pragma unroll
+  for (int q = 0; q < kAuSegPerLane; ++q) {
+    wgt[q] = ml[q].x == -INFINITY ? 0.f : exp2f(ml[q].x - M);
+    denom += wgt[q] * ml[q].y;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) denom += __shfl_xor_sync(0xffffffffu, denom, o);
+  float acc[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) acc[i] = 0.f;
+  for (uint32_t sg = 0; sg < nseg; ++sg) {
+    float wq = wgt[0];
+#pragma unroll
+    for (int q = 1; q < kAuSegPerLane; ++q)
+      if ((sg >> 5) == static_cast<uint32_t>(q)) wq = wgt[q];
+    const float ws = __shfl_sync(0xffffffffu, wq, static_cast<int>(sg & 31));
+    if (ws == 0.f) continue;  // uniform over the warp
+    const float4* src =
+        reinterpret_cast<const float4*>(part_o + (((size_t)seg_range(sg) + b) * kAuHeads + h) * kAuDv + 16 * lane);
+    float4 v[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) v[i] = src[i];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      acc[4 * i] += ws * v[i].x;
+      acc[4 * i + 1] += ws * v[i].y;
+      acc[4 * i + 2] += ws * v[i].z;
+      acc[4 * i + 3] += ws * v[i].w;
+    }
   }
   const float inv = denom > 0.f ? 1.f / denom : 0.f;
-  __nv_bfloat162* o2 = reinterpret_cast<__nv_bfloat162*>(out + ((size_t)b * kAuHeads + h) * kAuDv + d0);
-  o2[0] = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
-  o2[1] = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
-  if (lse != nullptr && tid == 0)
+  uint32_t pk[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) pk[i] = pack_bf16x2(acc[2 * i] * inv, acc[2 * i + 1] * inv);
+  uint4* dst = reinterpret_cast<uint4*>(out + ((size_t)b * kAuHeads + h) * kAuDv + 16 * lane);
+  dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+  dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+  if (lse != nullptr && lane == 0)
     lse[(size_t)b * kAuHeads + h] = denom > 0.f ? (M + log2f(denom)) * 0.69314718055994530942f : -INFINITY;
+  if (threadIdx.x == 0 && (blockIdx.x & 15) == 0) SD_PROBE_MARK(4, 1, 0);
 }
 
 // Workspace: partial O [slots][128][512] fp32, (m, l) [slots][128], and the

@@ -4,11 +4,10 @@
 //
 // Keys are read in place from the paged int8 pool through the block table
 // (the pages' "direct paged-pool scoring ... no Torch gather" of the TriAttention
-// scorer, Key Design Decisions). This kernel is the general path: it serves
-// thin indexers (few heads per KV head, as in per-head selection) where the
-// [Hi x Di] x [Di x L] contraction is too narrow for tensor cores and the
-// stream of keys is the bound. Wide indexers (Hi = 64, Di = 128) go to the
-// tcgen05 kernel instead.
+// scorer, Key Design Decisions). This kernel is the general path, for every
+// shape the tensor-core kernel (indexer_umma.cuh) does not take: that one
+// serves the MLA indexer (one KV head, Hi = 64, Di = 128) and the per-head
+// indexer of 8 KV heads with Hi = 4, Di = 64.
 //
 // A CTA scores T consecutive tokens of one request for every KV head. Each
 // token's row base is looked up once; the tile's key rows (G x Di bytes per

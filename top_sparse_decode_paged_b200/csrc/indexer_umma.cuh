@@ -1,14 +1,20 @@
-// Indexer scores on the 5th-generation tensor cores (tcgen05, kind::i8) for a
-// single KV head with 128-byte key rows (Di = 128) and HI indexer heads:
+// Indexer scores on the 5th-generation tensor cores (tcgen05, kind::i8):
 //
-//   s[b,t] = sum_h w[b,h] * max(0, sum_d qi[b,h,d] * ki[t,d])
+//   s[b,g,t] = sum_h w[b,g,h] * max(0, sum_d qi[b,g,h,d] * ki[t,g,d])
 //
-// Per 128-token tile, the keys of the tile are the M = 128 operand A (K-major,
-// one 128-byte row per token, exactly the NHD page layout), the request's
-// queries are operand B (N = HI heads, K-major), and the int32 products
-// D[token, head] land in tensor memory, one TMEM lane per token. The ReLU and
-// the weighted head sum are then a per-thread loop over that thread's TMEM
-// row, and each warp writes 32 consecutive scores.
+// Per 128-token tile, the keys of the tile are the M = 128 operand A (K-major:
+// a token's G * Di bytes, exactly the NHD page layout, stored as 128-byte
+// column chunks of [128 tokens x 128 B]), the request's queries are operand B
+// (N = G * HPG heads, K = G * Di), and the int32 products D[token, head] land
+// in tensor memory, one TMEM lane per token. With one KV head (the MLA
+// indexer, G = 1, Di = 128) B is the request's [HPG x 128] query block, loaded
+// by TMA. With several KV heads (per-head selection) B is block-diagonal:
+// head (g, h) holds qi[b,g,h] in the K columns of KV head g and zeros
+// elsewhere, so one MMA chain scores every KV head's keys at once (the zeros
+// cost tensor time that stays far below the key stream); the producer warp
+// builds it in shared memory. The ReLU and the weighted head sums are then a
+// per-thread loop over that thread's TMEM row, and each warp writes 32
+// consecutive scores per KV head.
 //
 // Keys stream straight from the paged pool: the TMA engine copies each page
 // of the tile (P rows x 128 B, 128-byte swizzle) into a shared-memory stage,
@@ -18,9 +24,12 @@
 // the tiles of all requests form one list, and each CTA takes a contiguous
 // share of it (requests of any length, no host-side schedule).
 //
-// Roles (192 threads): warp 0 issues TMA, warp 1 owns tensor memory and issues
-// the MMAs, warps 2-5 run the epilogue (warp w reads TMEM lanes 32*(w%4)..+31).
-// Stages are recycled through mbarriers; accumulators are double-buffered.
+// Roles (320 threads): warp 0 issues TMA, warp 1 owns tensor memory and issues
+// the MMAs, warps 2-9 run the epilogue as two sets of four (set e takes the
+// tiles i = e mod 2; warp w reads TMEM lanes 32*(w%4)..+31). Stages are
+// recycled through mbarriers; tile i accumulates into one of kUmmaAccs
+// tensor-memory accumulators (i mod kUmmaAccs), so the MMAs run up to
+// kUmmaAccs - 1 tiles ahead of the epilogue.
 #pragma once
 
 #include "sm100.cuh"
@@ -28,27 +37,39 @@
 namespace sd {
 
 constexpr int kUmmaTile = 128;     // tokens per tile (MMA M)
-constexpr int kUmmaRowBytes = 128; // Di = 128 int8
-constexpr int kUmmaStages = 6;
-constexpr int kUmmaTilesPerStage = 2;  // consecutive tiles of one request share a stage
-constexpr int kUmmaAccs = 2;       // accumulators in tensor memory (tile i uses i % 2)
+constexpr int kUmmaChunk = 128;    // bytes of a K-major column chunk (the 128-byte swizzle)
+constexpr int kUmmaAccs = 4;       // accumulators in tensor memory (tile i uses i % 4)
 constexpr int kUmmaEpiSets = 2;   // epilogue warp sets; set e reads the tiles i = e (mod 2)
 constexpr int kUmmaThreads = 64 + 128 * kUmmaEpiSets;
 
-template <int HI>
-struct IndexerUmmaLayout {
-  static constexpr int kTileBytes = kUmmaTile * kUmmaRowBytes;  // 16 KB
-  static constexpr int kStageBytes = kUmmaTilesPerStage * kTileBytes;
-  static constexpr int kQBytes = HI * kUmmaRowBytes;
-  static constexpr int kAccCols = kUmmaAccs * HI;
+// G KV heads of Di-byte keys, HPG indexer heads per KV head; TPS tiles of one
+// request share a shared-memory stage, STAGES stages.
+template <int G, int HPG, int DI, int TPS, int STAGES>
+struct IndexerUmmaCfg {
+  static constexpr int kHeads = G * HPG;            // MMA N (accumulator columns)
+  static constexpr int kRowBytes = G * DI;          // key bytes per token (MMA K)
+  static constexpr int kChunks = kRowBytes / kUmmaChunk;
+  static constexpr int kTilesPerStage = TPS;
+  static constexpr int kStages = STAGES;
+  static constexpr int kChunkBytes = kUmmaTile * kUmmaChunk;  // 16 KB
+  static constexpr int kTileBytes = kChunks * kChunkBytes;
+  static constexpr int kStageBytes = TPS * kTileBytes;
+  static constexpr int kQBytes = kChunks * kHeads * kUmmaChunk;
+  static constexpr int kAccCols = kUmmaAccs * kHeads;
   static constexpr int kTmemCols = kAccCols <= 32 ? 32 : (kAccCols <= 64 ? 64 : (kAccCols <= 128 ? 128 : (kAccCols <= 256 ? 256 : 512)));
-  static constexpr int kOffQ = kUmmaStages * kStageBytes;
+  static constexpr int kOffQ = STAGES * kStageBytes;
   static constexpr int kOffBar = kOffQ + 2 * kQBytes;
-  static constexpr int kNumBars = 2 * kUmmaStages + 2 + 2 + 2 * kUmmaAccs;
+  static constexpr int kNumBars = 2 * STAGES + 2 + 2 + 2 * kUmmaAccs;
   static constexpr int kOffMisc = kOffBar + 8 * kNumBars;
   static constexpr int kBytes = kOffMisc + 16;
   static constexpr size_t kSmemAlloc = kBytes + 1024;  // slack to align the base to 1024 B
+  static_assert(kRowBytes % kUmmaChunk == 0 && kHeads % 16 == 0 && kHeads <= 256, "MMA shape");
+  static_assert(kAccCols <= 512 && kSmemAlloc <= 232448, "resources");
 };
+// The MLA indexer (one KV head, 64 heads of 128 bytes) and the per-head
+// indexer (8 KV heads of 64 bytes, 4 heads each).
+using IdxCfgMla = IndexerUmmaCfg<1, 64, 128, 2, 6>;
+using IdxCfgPerHead = IndexerUmmaCfg<8, 4, 64, 1, 3>;
 
 // Walks a contiguous range of the global tile list (request-major).
 
@@ -83,12 +104,12 @@ struct TileCursor {
 };
 
 // A stage takes the cursor's tile and the following ones of the same
-// request within the range, up to kUmmaTilesPerStage and to 32 pages (one
+// request within the range, up to tiles_per_stage and to 32 pages (one
 // block-table window); every tile but the stage's last is then a full 128
 // tokens.
-__device__ __forceinline__ int stage_tiles(const TileCursor& c, int pages_per_tile) {
+__device__ __forceinline__ int stage_tiles(const TileCursor& c, int pages_per_tile, int tiles_per_stage) {
   const long long left = c.remaining < (long long)(c.tiles_b - c.tile) ? c.remaining : (long long)(c.tiles_b - c.tile);
-  const int cap = min(kUmmaTilesPerStage, 32 / pages_per_tile);
+  const int cap = min(tiles_per_stage, 32 / pages_per_tile);
   return left < cap ? static_cast<int>(left) : cap;
 }
 
@@ -102,13 +123,15 @@ __device__ __forceinline__ long long total_tiles(const int32_t* seqlens, int B, 
   return n;
 }
 
-template <int HI>
+template <class Cfg, int G, int HPG, int DI>
 __global__ void __launch_bounds__(kUmmaThreads, 1) indexer_umma_kernel(
     const __grid_constant__ CUtensorMap tm_keys, const __grid_constant__ CUtensorMap tm_q,
-    const int32_t* __restrict__ w, const int32_t* __restrict__ block_table,
+    const int8_t* __restrict__ qi, const int32_t* __restrict__ w, const int32_t* __restrict__ block_table,
     const int32_t* __restrict__ seqlens, int32_t* __restrict__ scores, int B, int num_pages, int page_size,
     int max_pages, int max_seqlen) {
-  using Lay = IndexerUmmaLayout<HI>;
+  using Lay = Cfg;
+  constexpr int HI = Lay::kHeads;
+  constexpr int kUmmaStages = Lay::kStages;
   extern __shared__ uint8_t smem_dyn[];
   const uint32_t raw = smem_u32(smem_dyn);
   uint8_t* smem = smem_dyn + (((raw + 1023u) & ~1023u) - raw);
@@ -163,6 +186,7 @@ __global__ void __launch_bounds__(kUmmaThreads, 1) indexer_umma_kernel(
   const long long total = total_tiles(seqlens, B, cap);
   const long long first = total * blockIdx.x / gridDim.x;
   const long long count = total * (blockIdx.x + 1) / gridDim.x - first;
+  if (threadIdx.x == 0) SD_PROBE_MARK(1, 0, count);
 
   if (warp == 0) {
     // ---------------- TMA producer (whole warp) ----------------
@@ -179,7 +203,11 @@ __global__ void __launch_bounds__(kUmmaThreads, 1) indexer_umma_kernel(
     int stage = 0;
     uint32_t phase = 0;
     int nq = 0, cur_b = -1;
-    const uint32_t page_bytes = static_cast<uint32_t>(page_size) * kUmmaRowBytes;
+    const uint32_t page_bytes = static_cast<uint32_t>(page_size) * Lay::kRowBytes;
+    const int ppt_shift = 7 - pshift;  // log2 of the pages of a tile
+    // the keys are read once: keep them from evicting the scores, which the
+    // top-k rereads right after this kernel
+    const uint64_t evict_first = sm100::l2_policy_evict_first();
     const int oob_row = num_pages * page_size;
     int win_b = -1, win_p0 = 0, win_val = -1;
     int nxt_p0 = -1, nxt_val = -1;  // the following window of the same request, loaded ahead
@@ -187,23 +215,41 @@ __global__ void __launch_bounds__(kUmmaThreads, 1) indexer_umma_kernel(
       if (c.b != cur_b) {
         const int slot = nq & 1;
         bool ok = true;
-        if (lane == 0) {
-          ok = sm100::mbar_wait(&qempty[slot], ((nq >> 1) & 1) ^ 1) && !*abort_flag;
-          if (ok) {
-            sm100::mbar_arrive_expect_tx(&qfull[slot], Lay::kQBytes);
-            sm100::tma_load_2d(qbuf + slot * Lay::kQBytes, &tm_q, &qfull[slot], 0, c.b * HI);
-          }
-        }
+        if (lane == 0) ok = sm100::mbar_wait(&qempty[slot], ((nq >> 1) & 1) ^ 1) && !*abort_flag;
         if (!__shfl_sync(0xffffffffu, ok, 0)) {
           if (lane == 0) *abort_flag = 1;
           break;
+        }
+        if constexpr (G == 1) {
+          // the request's [HI x 128] query block, by TMA
+          if (lane == 0) {
+            sm100::mbar_arrive_expect_tx(&qfull[slot], Lay::kQBytes);
+            sm100::tma_load_2d(qbuf + slot * Lay::kQBytes, &tm_q, &qfull[slot], 0, c.b * HI);
+          }
+        } else {
+          // the block-diagonal query operand: 16-byte granule j of row n in
+          // chunk cc covers K bytes 128 cc + 16 j, which belong to KV head
+          // (128 cc + 16 j) / DI; row n = g * HPG + h is qi[b,g,h] there and
+          // zero elsewhere (rows in the 128-byte swizzle)
+          uint8_t* qs = qbuf + slot * Lay::kQBytes;
+          for (int idx = lane; idx < Lay::kChunks * HI * 8; idx += 32) {
+            const int cc = idx / (HI * 8), n = (idx / 8) % HI, j = idx % 8;
+            const int kb = kUmmaChunk * cc + 16 * j;
+            uint4 v = make_uint4(0u, 0u, 0u, 0u);
+            if (kb / DI == n / HPG)
+              v = __ldg(reinterpret_cast<const uint4*>(qi + ((size_t)c.b * HI + n) * DI + (kb % DI)));
+            *reinterpret_cast<uint4*>(qs + cc * HI * kUmmaChunk + n * kUmmaChunk + ((j ^ (n & 7)) << 4)) = v;
+          }
+          sm100::fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) sm100::mbar_arrive(&qfull[slot]);
         }
         cur_b = c.b;
         ++nq;
       }
       const int t0 = c.tile * kUmmaTile;
       const int p_first = t0 >> pshift;
-      const int nt = stage_tiles(c, kUmmaTile >> pshift);
+      const int nt = stage_tiles(c, kUmmaTile >> pshift, Lay::kTilesPerStage);
       const int npages = (min(kUmmaTile * nt, c.L - t0) + page_size - 1) >> pshift;
       if (c.b != win_b || p_first + npages > win_p0 + 32) {
         if (c.b == win_b && p_first == nxt_p0) {
@@ -229,12 +275,20 @@ __global__ void __launch_bounds__(kUmmaThreads, 1) indexer_umma_kernel(
         break;
       }
       if (off >= 0 && off < npages) {
+        // page `off` of the stage: tile off / ppt, rows (off % ppt) * P of
+        // each of its column chunks
         const int row = (win_val >= 0 && win_val < num_pages) ? win_val * page_size : oob_row;
-        sm100::tma_load_2d(kstage + stage * Lay::kStageBytes + off * page_bytes, &tm_keys, &full[stage], 0, row);
+        uint8_t* dst = kstage + stage * Lay::kStageBytes + (off >> ppt_shift) * Lay::kTileBytes +
+                       (off & ((1 << ppt_shift) - 1)) * page_size * kUmmaChunk;
+#pragma unroll
+        for (int cc = 0; cc < Lay::kChunks; ++cc)
+          sm100::tma_load_2d_hint(dst + cc * Lay::kChunkBytes, &tm_keys, &full[stage], cc * kUmmaChunk, row,
+                                  evict_first);
       }
       if (++stage == kUmmaStages) { stage = 0; phase ^= 1; }
       for (int j = 0; j < nt; ++j) c.next(seqlens, B, cap);
     }
+    if (lane == 0) SD_PROBE_MARK(1, 1, 0);
   } else if (warp == 1) {
     // ---------------- MMA issuer ----------------
     if (sm100::elect_one()) {
@@ -251,8 +305,9 @@ __global__ void __launch_bounds__(kUmmaThreads, 1) indexer_umma_kernel(
           ++nq;
         }
         const int slot = (nq - 1) & 1;
-        const int ntiles = stage_tiles(c, kUmmaTile >> pshift);
+        const int ntiles = stage_tiles(c, kUmmaTile >> pshift, Lay::kTilesPerStage);
         if (!sm100::mbar_wait(&full[stage], phase)) { *abort_flag = 1; break; }
+        if (blockIdx.x % 37 == 0) SD_PROBE_MARK(1, 10, 0);
         const uint32_t b0 = smem_u32(qbuf + slot * Lay::kQBytes);
         bool ok = true;
         for (int j = 0; j < ntiles; ++j) {
@@ -261,9 +316,11 @@ __global__ void __launch_bounds__(kUmmaThreads, 1) indexer_umma_kernel(
           const uint32_t a0 = smem_u32(kstage + stage * Lay::kStageBytes + j * Lay::kTileBytes);
           const uint32_t d = tmem_base + acc * HI;
 #pragma unroll
-          for (int k = 0; k < kUmmaRowBytes / 32; ++k)
-            sm100::mma_i8_ss(d, sm100::smem_desc_k_sw128(a0 + 32 * k), sm100::smem_desc_k_sw128(b0 + 32 * k),
-                             idesc, k > 0);
+          for (int cc = 0; cc < Lay::kChunks; ++cc)
+#pragma unroll
+            for (int k = 0; k < kUmmaChunk / 32; ++k)
+              sm100::mma_i8_ss(d, sm100::smem_desc_k_sw128(a0 + cc * Lay::kChunkBytes + 32 * k),
+                               sm100::smem_desc_k_sw128(b0 + cc * HI * kUmmaChunk + 32 * k), idesc, (cc | k) > 0);
           sm100::mma_commit(&accfull[acc]);
           if (++acc == kUmmaAccs) { acc = 0; accphase ^= 1; }
         }
@@ -274,6 +331,7 @@ __global__ void __launch_bounds__(kUmmaThreads, 1) indexer_umma_kernel(
         if (!c.valid() || c.b != this_b) sm100::mma_commit(&qempty[slot]);
         if (++stage == kUmmaStages) { stage = 0; phase ^= 1; }
       }
+      SD_PROBE_MARK(1, 2, 0);
     }
   } else {
     // ---------------- epilogue: ReLU, weighted head sum, store ----------------
@@ -282,12 +340,11 @@ __global__ void __launch_bounds__(kUmmaThreads, 1) indexer_umma_kernel(
     // its TMEM quadrant (warp % 4); the accumulator is released as soon as
     // its row is in registers; the block-table entry that validates this
     // thread's token is loaded one tile of the set ahead.
-    static_assert(kUmmaAccs == kUmmaEpiSets, "one accumulator per epilogue set");
+    static_assert(kUmmaAccs % kUmmaEpiSets == 0, "each set cycles through its own accumulators");
     const int set = (warp - 2) >> 2;
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
-    const int acc = set;
-    uint32_t accphase = 0;
+    int ti = set;  // this CTA's tile number: accumulator ti % kUmmaAccs
     TileCursor c;
     c.init(seqlens, B, cap, first, count);
     for (int i = 0; i < set; ++i) c.next(seqlens, B, cap);
@@ -309,9 +366,11 @@ __global__ void __launch_bounds__(kUmmaThreads, 1) indexer_umma_kernel(
       TileCursor cn = c;
       for (int i = 0; i < kUmmaEpiSets; ++i) cn.next(seqlens, B, cap);
       phys_next = page_of(cn);
-      const bool ok = sm100::mbar_wait(&accfull[acc], accphase);
+      const int acc = ti % kUmmaAccs;
+      const bool ok = sm100::mbar_wait(&accfull[acc], static_cast<uint32_t>((ti / kUmmaAccs) & 1));
       __syncwarp();  // tcgen05.ld is warp-collective: reconverge after the polling loop
       if (!ok) { *abort_flag = 1; break; }
+      if (blockIdx.x % 37 == 0 && quarter == 0 && lane == 0) SD_PROBE_MARK(1, 11 + set, 0);
       sm100::tc_fence_after();
       uint32_t r[HI];
 #pragma unroll
@@ -321,23 +380,29 @@ __global__ void __launch_bounds__(kUmmaThreads, 1) indexer_umma_kernel(
       sm100::tmem_ld_wait();
       sm100::tc_fence_before();
       sm100::mbar_arrive(&accempty[acc]);
-      // eight independent partial sums (a single chain would serialize 64 IMADs)
-      int32_t part[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-#pragma unroll
-      for (int i = 0; i < HI; ++i) part[i & 7] += wreg[i] * max(static_cast<int32_t>(r[i]), 0);
-      const int32_t s0 = (part[0] + part[1]) + (part[2] + part[3]);
-      const int32_t s1 = (part[4] + part[5]) + (part[6] + part[7]);
-      int32_t s = s0 + s1;
       if (t < c.L) {
-        if (phys < 0 || phys >= num_pages) {
-          raise_error(SD_DEVERR_PAGE);
-          s = INT32_MIN;
+        const bool bad = phys < 0 || phys >= num_pages;
+        if (bad) raise_error(SD_DEVERR_PAGE);
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+          // independent partial sums (a single chain would serialize the IMADs)
+          constexpr int kPart = HPG >= 8 ? 8 : HPG;
+          int32_t part[kPart];
+#pragma unroll
+          for (int i = 0; i < kPart; ++i) part[i] = 0;
+#pragma unroll
+          for (int i = 0; i < HPG; ++i)
+            part[i % kPart] += wreg[g * HPG + i] * max(static_cast<int32_t>(r[g * HPG + i]), 0);
+          int32_t s = 0;
+#pragma unroll
+          for (int i = 0; i < kPart; ++i) s += part[i];
+          scores[((size_t)c.b * G + g) * max_seqlen + t] = bad ? INT32_MIN : s;
         }
-        scores[(size_t)c.b * max_seqlen + t] = s;
       }
-      accphase ^= 1;
+      ti += kUmmaEpiSets;
       c = cn;
     }
+    if (quarter == 0 && lane == 0) SD_PROBE_MARK(1, 3 + set, 0);
   }
 
   sm100::tc_fence_before();

@@ -193,13 +193,14 @@ EncodeTiledFn encode_tiled_fn() {
   return fn;
 }
 
-// A 2-D int8 map over `rows` rows of 128 bytes, boxes of box_rows x 128 B,
-// 128-byte swizzle (the K-major UMMA operand layout).
-bool encode_rows128(CUtensorMap* map, const void* base, uint64_t rows, uint32_t box_rows) {
+// A 2-D int8 map over `rows` rows of row_bytes bytes, boxes of box_rows x 128 B
+// (one 128-byte column chunk), 128-byte swizzle (the K-major UMMA operand
+// layout).
+bool encode_rows128(CUtensorMap* map, const void* base, uint64_t rows, uint32_t box_rows, uint64_t row_bytes = 128) {
   EncodeTiledFn fn = encode_tiled_fn();
   if (fn == nullptr || (reinterpret_cast<uintptr_t>(base) & 15u) != 0) return false;
-  const cuuint64_t dims[2] = {128, rows};
-  const cuuint64_t strides[1] = {128};
+  const cuuint64_t dims[2] = {row_bytes, rows};
+  const cuuint64_t strides[1] = {row_bytes};
   const cuuint32_t box[2] = {128, box_rows};
   const cuuint32_t estride[2] = {1, 1};
   return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estride,
@@ -229,34 +230,51 @@ int sm_count() {
   return n;
 }
 
-// The tensor-core indexer covers one KV head of 128-byte keys with 64 heads and
-// pages that tile a 128-token block; everything else takes the dp4a kernel.
+// The tensor-core indexer covers one KV head of 128-byte keys with 64 heads
+// (MLA) and 8 KV heads of 64-byte keys with 4 heads each (per-head
+// selection), with pages that tile a 128-token block; everything else takes
+// the dp4a kernel.
+bool umma_indexer_mla(const sd_paged_desc& pd, int Hi, int Di) { return pd.kv_heads == 1 && Di == 128 && Hi == 64; }
+bool umma_indexer_perhead(const sd_paged_desc& pd, int Hi, int Di) { return pd.kv_heads == 8 && Di == 64 && Hi == 4; }
 bool umma_indexer_fits(const sd_paged_desc& pd, int Hi, int Di, const void* qi, const void* ki) {
   const int P = pd.page_size;
-  return pd.kv_heads == 1 && Di == 128 && Hi == 64 && P >= 8 && P <= 128 && (128 % P) == 0 &&
+  return (umma_indexer_mla(pd, Hi, Di) || umma_indexer_perhead(pd, Hi, Di)) && P >= 8 && P <= 128 && (128 % P) == 0 &&
          (long long)(pd.num_pages + 1) * P < (1ll << 31) &&  // TMA row coordinates, one page past the end included
          (reinterpret_cast<uintptr_t>(qi) & 15u) == 0 && (reinterpret_cast<uintptr_t>(ki) & 15u) == 0;
 }
 
-sd_status launch_indexer_umma(const int8_t* qi, const int32_t* w, const int8_t* ki, const int32_t* bt,
-                              const int32_t* seqlens, int32_t* scores, const sd_paged_desc& pd, int B,
-                              int max_seqlen, cudaStream_t st, bool* launched) {
-  constexpr int HI = 64;
-  using Lay = sd::IndexerUmmaLayout<HI>;
+template <class Cfg, int G, int HPG, int DI>
+sd_status launch_indexer_umma_t(const int8_t* qi, const int32_t* w, const int8_t* ki, const int32_t* bt,
+                                const int32_t* seqlens, int32_t* scores, const sd_paged_desc& pd, int B,
+                                int max_seqlen, cudaStream_t st, bool* launched) {
   *launched = false;
   CUtensorMap tm_keys, tm_q;
-  if (!encode_rows128(&tm_keys, ki, (uint64_t)pd.num_pages * pd.page_size, pd.page_size)) return SD_OK;
-  if (!encode_rows128(&tm_q, qi, (uint64_t)B * HI, HI)) return SD_OK;
-  auto kern = sd::indexer_umma_kernel<HI>;
+  if (!encode_rows128(&tm_keys, ki, (uint64_t)pd.num_pages * pd.page_size, pd.page_size, (uint64_t)G * DI)) return SD_OK;
+  if (G == 1) {
+    if (!encode_rows128(&tm_q, qi, (uint64_t)B * Cfg::kHeads, Cfg::kHeads)) return SD_OK;
+  } else {
+    tm_q = tm_keys;  // unused: the block-diagonal query operand is built in shared memory
+  }
+  auto kern = sd::indexer_umma_kernel<Cfg, G, HPG, DI>;
   sd_status s = cuda_check(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                static_cast<int>(Lay::kSmemAlloc)));
+                                                static_cast<int>(Cfg::kSmemAlloc)));
   if (s != SD_OK) return s;
   stage_mark(kStageIndexer, 0, st);
-  s = launch_k(kern, dim3(sm_count()), dim3(sd::kUmmaThreads), Lay::kSmemAlloc, st, tm_keys, tm_q, w, bt, seqlens,
-               scores, B, pd.num_pages, pd.page_size, pd.max_pages_per_req, max_seqlen);
+  s = launch_k(kern, dim3(sm_count()), dim3(sd::kUmmaThreads), Cfg::kSmemAlloc, st, tm_keys, tm_q, qi, w, bt,
+               seqlens, scores, B, pd.num_pages, pd.page_size, pd.max_pages_per_req, max_seqlen);
   stage_mark(kStageIndexer, 1, st);
   *launched = true;
   return s;
+}
+
+sd_status launch_indexer_umma(const int8_t* qi, const int32_t* w, const int8_t* ki, const int32_t* bt,
+                              const int32_t* seqlens, int32_t* scores, const sd_paged_desc& pd, int B, int Hi,
+                              int Di, int max_seqlen, cudaStream_t st, bool* launched) {
+  if (umma_indexer_mla(pd, Hi, Di))
+    return launch_indexer_umma_t<sd::IdxCfgMla, 1, 64, 128>(qi, w, ki, bt, seqlens, scores, pd, B, max_seqlen, st,
+                                                           launched);
+  return launch_indexer_umma_t<sd::IdxCfgPerHead, 8, 4, 64>(qi, w, ki, bt, seqlens, scores, pd, B, max_seqlen, st,
+                                                           launched);
 }
 
 template <int PER>
@@ -316,7 +334,7 @@ sd_status launch_indexer_topk(const int8_t* qi, const int32_t* w, const int8_t* 
   if (B == 0) return SD_OK;
   bool done = false;
   if (max_seqlen > 0 && umma_indexer_fits(pd, Hi, Di, qi, ki)) {
-    sd_status s = launch_indexer_umma(qi, w, ki, bt, seqlens, scores, pd, B, max_seqlen, st, &done);
+    sd_status s = launch_indexer_umma(qi, w, ki, bt, seqlens, scores, pd, B, Hi, Di, max_seqlen, st, &done);
     if (s != SD_OK) return s;
   }
   if (max_seqlen > 0 && !done) {
@@ -403,7 +421,7 @@ sd_status launch_attn_umma(const uint16_t* q, const uint16_t* const* kp_layers, 
   if (s != SD_OK) return s;
   stage_mark(kStageCombine, 0, st);
   s = launch_k(sd::attn_mla_umma_combine_kernel, dim3(Bv * (sd::kAuHeads / sd::kAuCombineHeads)),
-               dim3(128 * sd::kAuCombineHeads), 0, st, static_cast<const float*>(part_o),
+               dim3(32 * sd::kAuCombineHeads), 0, st, static_cast<const float*>(part_o),
                static_cast<const float2*>(part_ml), seqlens, Bv, B, k, seqlen_cap, sd::kAuRanges,
                reinterpret_cast<__nv_bfloat16*>(out), lse);
   stage_mark(kStageCombine, 1, st);
@@ -834,6 +852,21 @@ const char* sd_status_str(sd_status status) {
   }
   return "SD_ERR_UNKNOWN";
 }
+
+#ifdef SD_PROBE
+// Probe builds only: copies up to `max_records` probe records (4 x u64 each)
+// to host memory, resets the ring and returns how many were recorded.
+int64_t sd_probe_read(void* dst, int64_t max_records) {
+  unsigned int n = 0;
+  if (cudaDeviceSynchronize() != cudaSuccess || cudaMemcpyFromSymbol(&n, sd::g_probe_n, sizeof(n)) != cudaSuccess)
+    return -1;
+  const unsigned int m = static_cast<unsigned int>(std::min<int64_t>(std::min(n, sd::kProbeCap), max_records));
+  if (m > 0 && dst != nullptr && cudaMemcpyFromSymbol(dst, sd::g_probe, (size_t)m * 32) != cudaSuccess) return -1;
+  const unsigned int zero = 0;
+  if (cudaMemcpyToSymbol(sd::g_probe_n, &zero, sizeof(zero)) != cudaSuccess) return -1;
+  return n;
+}
+#endif
 
 int32_t sd_last_cuda_error(void) { return t_last_cuda_error; }
 int32_t sd_last_launch_count(void) { return t_launches; }

@@ -9,11 +9,39 @@
 
 namespace sd {
 
+constexpr int kMaxTopK = 2048;  // largest k the library accepts
+
 // Sticky per-device error word; kernels OR SD_DEVERR_* bits into it when
 // device-resident data (seqlens, block tables, indices) is out of range.
 __device__ unsigned int g_error_bits;
 
 __device__ __forceinline__ void raise_error(unsigned int bit) { atomicOr(&g_error_bits, bit); }
+
+// Timeline probes for tuning. Compiled out unless the library is built with
+// -DSD_PROBE; then each mark appends (globaltimer ns, SM clock, kernel / block
+// / event, value) to a device ring that sd_probe_read() copies out.
+#ifdef SD_PROBE
+constexpr unsigned int kProbeCap = 1u << 20;
+__device__ unsigned long long g_probe[kProbeCap][4];
+__device__ unsigned int g_probe_n;
+__device__ __forceinline__ void probe_mark(int kernel, int event, long long value) {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  const unsigned int i = atomicAdd(&g_probe_n, 1u);
+  if (i < kProbeCap) {
+    unsigned int smid;
+    asm volatile("mov.u32 %0, %%smid;" : "=r"(smid));
+    g_probe[i][0] = t;
+    g_probe[i][1] = clock64();
+    g_probe[i][2] = ((unsigned long long)kernel << 56) | ((unsigned long long)event << 48) |
+                    ((unsigned long long)smid << 32) | (blockIdx.x + blockIdx.y * gridDim.x);
+    g_probe[i][3] = static_cast<unsigned long long>(value);
+  }
+}
+#define SD_PROBE_MARK(k, e, v) ::sd::probe_mark((k), (e), (v))
+#else
+#define SD_PROBE_MARK(k, e, v) ((void)0)
+#endif
 
 // Clamp a device-resident sequence length to [0, cap]; flags the error bit.
 __device__ __forceinline__ int checked_seqlen(const int32_t* seqlens, int b, int cap) {
@@ -59,6 +87,16 @@ struct RowMap {
       } else {
         raise_error(SD_DEVERR_PAGE);
       }
+    }
+    rows[(size_t)row * kpad + slot] = r;
+  }
+  // The same for a token >= 0 whose block-table entry the caller loaded.
+  __device__ __forceinline__ void put_page(int row, int slot, int token, int page) const {
+    int r = -1;
+    if (page >= 0 && page < num_pages) {
+      r = page * page_size + token % page_size;
+    } else {
+      raise_error(SD_DEVERR_PAGE);
     }
     rows[(size_t)row * kpad + slot] = r;
   }

@@ -15,6 +15,16 @@
 //   - the final pass is an ordered compaction: per-thread counts of "greater"
 //     and "equal to the threshold" keys, one block scan, one cluster exchange
 //     of CTA totals, and each thread writes its picks in token order.
+// Candidate path (without a hint, whenever it applies, which is the common
+// case): after the first radix pass fixes the digit D holding the k-th
+// largest key, with A keys above it and c_D in it, and A + c_D <=
+// kTkCandCap, every CTA compacts its keys at or above D's range (in token
+// order), CTA 0 gathers the cluster's candidates and resolves the exact
+// threshold among the c_D keys of digit D by radix passes in its own shared
+// memory, then writes the output alone. That replaces the later cluster-wide
+// passes and the cluster compaction by one candidate exchange. Otherwise
+// (heavy ties, a digit holding too many keys, or a hint) the radix passes run
+// on the full slices as above.
 // No CTA waits on another except at hardware cluster barriers.
 #pragma once
 
@@ -30,19 +40,21 @@ constexpr int kTkThreads = 512;
 constexpr int kTkBinsBits = 11;
 constexpr int kTkBins = 1 << kTkBinsBits;
 constexpr int kTkMaxCluster = 8;
+constexpr int kTkCandCap = 4096;    // candidates (keys at or above the first pass's digit) the path takes
 
 // PER: scores per thread (16 or 32); a CTA holds a slice of 512 * PER scores.
 template <int PER>
 struct TopkClusterSmem {
   static constexpr int kStride = PER + 1;       // padded per-thread chunk (words)
   uint32_t keys[kTkThreads * kStride];          // thread t's chunk at t*(PER+1) (bank-conflict free)
-  uint32_t hist[kTkBins];                       // this CTA's histogram (read by the cluster)
-  uint32_t total[kTkBins];                      // cluster-wide histogram
+  uint32_t hist[kTkCandCap];                    // this CTA's histogram (read by the cluster); CTA 0's candidate keys
+  uint32_t total[kTkCandCap];                   // cluster-wide histogram; CTA 0's candidate tokens
   uint32_t red[kTkThreads / 32 * 2 + 8];        // block reduction / scan scratch
   uint32_t cta_vals[4];                         // values this CTA publishes to the cluster
-  uint32_t found[2];                            // threshold digit, remaining
+  uint32_t found[4];                            // threshold digit, remaining (and scratch)
   uint32_t mark[kTkThreads * PER / 32];         // hint tokens of this CTA's slice (one bit each)
   uint32_t hvals[4];                            // hint bounds this CTA publishes
+  static_assert(kTkThreads * kStride >= 2 * kTkCandCap, "candidate keys and tokens fit in the key area");
 };
 
 // Block-wide exclusive scan of 32-bit values (512 threads); returns the prefix,
@@ -75,6 +87,29 @@ __device__ __forceinline__ uint32_t tk_block_excl_scan(uint32_t v, uint32_t* scr
   return r;
 }
 
+// Block-wide minimum and maximum in one pass (two barriers).
+__device__ __forceinline__ void tk_block_minmax(uint32_t& mn, uint32_t& mx, uint32_t* scratch) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    mn = min(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+    mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  }
+  if (lane == 0) {
+    scratch[2 * warp] = mn;
+    scratch[2 * warp + 1] = mx;
+  }
+  __syncthreads();
+  mn = 0xffffffffu;
+  mx = 0u;
+#pragma unroll
+  for (int w = 0; w < kTkThreads / 32; ++w) {
+    mn = min(mn, scratch[2 * w]);
+    mx = max(mx, scratch[2 * w + 1]);
+  }
+  __syncthreads();
+}
+
 __device__ __forceinline__ uint32_t tk_block_reduce(uint32_t v, uint32_t* scratch, bool is_max) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 #pragma unroll
@@ -99,12 +134,233 @@ __device__ __forceinline__ uint32_t tk_block_reduce(uint32_t v, uint32_t* scratc
   return v;
 }
 
+// total[i] = sum over the cluster's CTAs of hist[i] (2048 bins), with every
+// remote read of a thread in flight together; ends with a block barrier.
+template <typename Smem>
+__device__ __forceinline__ void tk_merge_hist(Smem& sm, cg::cluster_group& cluster, int CS) {
+  constexpr int kPer = kTkBins / kTkThreads;
+  uint32_t v[kTkMaxCluster][kPer];
+#pragma unroll
+  for (int r = 0; r < kTkMaxCluster; ++r) {
+    if (r < CS) {
+      const uint32_t* h = cluster.map_shared_rank(sm.hist, r);
+#pragma unroll
+      for (int j = 0; j < kPer; ++j) v[r][j] = h[threadIdx.x + j * kTkThreads];
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < kPer; ++j) {
+    uint32_t t = 0;
+#pragma unroll
+    for (int r = 0; r < kTkMaxCluster; ++r)
+      if (r < CS) t += v[r][j];
+    sm.total[threadIdx.x + j * kTkThreads] = t;
+  }
+  __syncthreads();
+}
+
+// Finds the threshold digit of one radix pass: thread t owns bins 4t..4t+3 of
+// `h` (2048 bins); returns (digit, remaining) through found[0..1] and the
+// count of the digit's bin through the return value.
+__device__ __forceinline__ uint32_t tk_find_digit(const uint32_t* h, uint32_t remaining, uint32_t* red,
+                                                  uint32_t* found) {
+  const int tid = threadIdx.x;
+  uint32_t c4[4], mine = 0;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    c4[i] = h[4 * tid + i];
+    mine += c4[i];
+  }
+  uint32_t all;
+  const uint32_t rev = tk_block_excl_scan(mine, red, &all);  // keys in higher bins (reverse order)
+  const uint32_t above = all - rev - mine;
+  if (above < remaining && above + mine >= remaining) {
+    uint32_t acc = above;
+#pragma unroll
+    for (int i = 3; i >= 0; --i) {
+      if (acc < remaining && acc + c4[i] >= remaining) {
+        found[0] = 4u * tid + i;
+        found[1] = remaining - acc;
+      }
+      acc += c4[i];
+    }
+  }
+  __syncthreads();
+  const uint32_t bin_count = h[found[0]];
+  return bin_count;
+}
+
+// The candidate path (see the file comment). On entry the first radix pass
+// has fixed the digit D of the k-th largest key: its keys are those with
+// (u & pmask1) == prefix1 (bin_count of them, over the cluster), every key
+// >= prefix1 is at or above D, and `need` keys are to be taken from D. Every
+// CTA holds its slice's keys in its per-thread chunks. Ends with CTA 0
+// writing the row's output; the other CTAs return after the third cluster
+// barrier.
+template <int PER>
+__device__ __forceinline__ void topk_candidates(TopkClusterSmem<PER>& sm, cg::cluster_group& cluster, int CS,
+                                                int crank, int row, int b, int k, int s0, int nvalid,
+                                                uint32_t prefix1, uint32_t pmask1, int shift, uint32_t need,
+                                                uint32_t bin_count, int32_t* out, const RowMap& rm) {
+  const int tid = threadIdx.x;
+  // 1. this CTA's keys >= prefix1, in token order, into the key area
+  uint32_t kv[PER];
+  uint32_t pick = 0, nc = 0;
+  const uint32_t* chunk = sm.keys + tid * (PER + 1);
+#pragma unroll
+  for (int j = 0; j < PER; ++j) {
+    kv[j] = chunk[j];
+    const bool c = j < nvalid && kv[j] >= prefix1;
+    pick |= static_cast<uint32_t>(c) << j;
+    nc += c;
+  }
+  uint32_t ctot;
+  uint32_t pos = tk_block_excl_scan(nc, sm.red, &ctot);  // its barriers order every chunk read before the writes
+  uint32_t* ck = sm.keys;               // candidate keys, token order
+  uint32_t* ct = sm.keys + kTkCandCap;  // their tokens
+#pragma unroll
+  for (int j = 0; j < PER; ++j) {
+    if ((pick >> j) & 1u) {
+      ck[pos] = kv[j];
+      ct[pos] = static_cast<uint32_t>(s0 + tid * PER + j);
+      ++pos;
+    }
+  }
+  if (tid == 0) sm.cta_vals[2] = ctot;
+  cluster.sync();  // every CTA's candidates and count are in place (and every histogram read)
+  uint32_t* gk = sm.hist;   // CTA 0: the cluster's candidates in token order (CTA slices are in order)
+  uint32_t* gt = sm.total;
+  if (crank == 0) {
+    uint32_t cnt[kTkMaxCluster];
+#pragma unroll
+    for (int r = 0; r < kTkMaxCluster; ++r) cnt[r] = r < CS ? cluster.map_shared_rank(sm.cta_vals, r)[2] : 0u;
+    uint32_t off = 0;
+#pragma unroll
+    for (int r = 0; r < kTkMaxCluster; ++r) {
+      if (r < CS) {
+        const uint32_t* rk = cluster.map_shared_rank(sm.keys, r);
+        for (uint32_t i = tid; i < cnt[r]; i += kTkThreads) {
+          gk[off + i] = rk[i];
+          gt[off + i] = rk[kTkCandCap + i];
+        }
+      }
+      off += cnt[r];
+    }
+    if (tid == 0) sm.found[0] = off;
+  }
+  cluster.sync();  // CTA 0 holds every candidate: the others may leave
+  if (crank != 0) return;
+  const uint32_t nC = sm.found[0];
+
+  // 2. the exact threshold key Tk among the keys of digit D (radix passes over
+  // the candidates, histogram in the now free key area)
+  uint32_t Tk = prefix1, need_eq;
+  if (shift == 0) {
+    need_eq = need;                 // D is a single key value
+  } else if (bin_count == need) {
+    need_eq = 0xffffffffu;          // all of D is taken: every key >= prefix1 is in
+  } else {
+    uint32_t* rh = sm.keys;
+    uint32_t prefix = prefix1, pmask = pmask1, remaining = need;
+    int top = shift - 1;
+    for (;;) {
+      const int nbits = min(kTkBinsBits, top + 1);
+      const int sh = top + 1 - nbits;
+      const uint32_t dmask = (1u << nbits) - 1u;
+      for (int i = tid; i < kTkBins; i += kTkThreads) rh[i] = 0u;
+      __syncthreads();
+      for (uint32_t i = tid; i < nC; i += kTkThreads) {
+        const uint32_t u = gk[i];
+        if ((u & pmask) == prefix) atomicAdd(&rh[(u >> sh) & dmask], 1u);
+      }
+      __syncthreads();
+      const uint32_t cnt = tk_find_digit(rh, remaining, sm.red, sm.found + 2);
+      const uint32_t digit = sm.found[2], rem = sm.found[3];
+      __syncthreads();
+      prefix |= digit << sh;
+      pmask |= dmask << sh;
+      top = sh - 1;
+      if (sh == 0) {  // every bit fixed: Tk is exact
+        Tk = prefix;
+        need_eq = rem;
+        break;
+      }
+      if (cnt == rem) {  // the whole digit bin is taken: every key >= prefix is in
+        Tk = prefix;
+        need_eq = 0xffffffffu;
+        break;
+      }
+      remaining = rem;
+    }
+  }
+
+  // 3. ordered output: candidate i is taken if its key is above Tk (every key
+  // of a digit above D is), or equal to Tk and among the first need_eq of
+  // those in token order; thread t handles candidates 8t..8t+7
+  constexpr int kPerThr = kTkCandCap / kTkThreads;
+  uint32_t n_gt = 0, n_eq = 0;
+#pragma unroll
+  for (int j = 0; j < kPerThr; ++j) {
+    const uint32_t i = kPerThr * tid + j;
+    if (i < nC) {
+      const uint32_t u = gk[i];
+      n_gt += u > Tk;
+      n_eq += u == Tk;
+    }
+  }
+  uint32_t tot_packed;
+  const uint32_t pre = tk_block_excl_scan((n_gt << 16) | n_eq, sm.red, &tot_packed);
+  uint32_t gt_before = pre >> 16, eq_before = pre & 0xffffu;
+  if (tid == 0) SD_PROBE_MARK(2, 3, nC);
+  // the taken tokens in output order, staged in the free key area (k <= 2048)
+  uint32_t* sel = sm.keys;
+#pragma unroll
+  for (int j = 0; j < kPerThr; ++j) {
+    const uint32_t i = kPerThr * tid + j;
+    if (i < nC) {
+      const uint32_t u = gk[i];
+      if (u > Tk) {
+        sel[gt_before + min(eq_before, need_eq)] = gt[i];
+        ++gt_before;
+      } else if (u == Tk) {
+        if (eq_before < need_eq) sel[gt_before + eq_before] = gt[i];
+        ++eq_before;
+      }
+    }
+  }
+  __syncthreads();
+  // coalesced output; the pool rows' block-table loads of a thread are
+  // independent of each other, so they are all in flight together
+  constexpr int kOutPerThr = (kMaxTopK + kTkThreads - 1) / kTkThreads;
+  int pages[kOutPerThr];
+#pragma unroll
+  for (int j = 0; j < kOutPerThr; ++j) {
+    const int o = tid + j * kTkThreads;
+    pages[j] = -1;
+    if (o < k) {
+      const int tok = static_cast<int>(sel[o]);
+      out[o] = tok;
+      if (rm.rows != nullptr) pages[j] = rm.block_table[(size_t)b * rm.max_pages + tok / rm.page_size];
+    }
+  }
+  if (rm.rows != nullptr) {
+#pragma unroll
+    for (int j = 0; j < kOutPerThr; ++j) {
+      const int o = tid + j * kTkThreads;
+      if (o < k) rm.put_page(row, o, static_cast<int>(sel[o]), pages[j]);
+    }
+    for (int i = k + tid; i < rm.kpad; i += kTkThreads) rm.rows[(size_t)row * rm.kpad + i] = -1;
+  }
+  if (tid == 0) SD_PROBE_MARK(2, 5, nC);
+}
+
 template <int PER>
 __global__ void __launch_bounds__(kTkThreads, 2) topk_cluster_kernel(
     const int32_t* __restrict__ scores, const int32_t* __restrict__ seqlens, int32_t* __restrict__ indices,
     int G, int max_seqlen, int seqlen_cap, int k, RowMap rm, const int32_t* __restrict__ hint) {
   pdl_wait();  // inputs come from earlier work in the stream
   pdl_trigger();
+  if (threadIdx.x == 0) SD_PROBE_MARK(2, 0, 0);
 
   constexpr int kTkPerThread = PER;
   constexpr int kTkChunkStride = PER + 1;
@@ -151,8 +407,7 @@ __global__ void __launch_bounds__(kTkThreads, 2) topk_cluster_kernel(
   }
   if (hint != nullptr)
     for (int i = tid; i < kTkThreads * PER / 32; i += kTkThreads) sm.mark[i] = 0u;
-  kmin = tk_block_reduce(kmin, sm.red, false);
-  kmax = tk_block_reduce(kmax, sm.red, true);
+  tk_block_minmax(kmin, kmax, sm.red);
   if (tid == 0) {
     sm.cta_vals[0] = kmin;
     sm.cta_vals[1] = kmax;
@@ -176,9 +431,42 @@ __global__ void __launch_bounds__(kTkThreads, 2) topk_cluster_kernel(
     }
   }
   __syncthreads();
+  if (threadIdx.x == 0) SD_PROBE_MARK(2, 1, 0);
   uint32_t gmin = sm.found[0], gmax = sm.found[1];
   uint32_t hi_cut = 0xffffffffu;              // keys above it are all selected
   uint32_t remaining0 = static_cast<uint32_t>(k);
+
+  // ---- candidate path: first radix pass, then one candidate exchange ----
+  if (hint == nullptr && gmin != gmax) {
+    const int hb = 31 - __clz(gmin ^ gmax);
+    const uint32_t prefix0 = hb == 31 ? 0u : (gmax >> (hb + 1)) << (hb + 1);
+    const uint32_t pmask0 = hb == 31 ? 0u : ~((2u << hb) - 1u);
+    const int nbits = min(kTkBinsBits, hb + 1);
+    const int shift = hb + 1 - nbits;
+    const uint32_t dmask = (1u << nbits) - 1u;
+    for (int i = tid; i < kTkBins; i += kTkThreads) sm.hist[i] = 0u;
+    __syncthreads();
+    {
+      const uint32_t* chunk = sm.keys + tid * kTkChunkStride;
+      for (int j = 0; j < nvalid; ++j) atomicAdd(&sm.hist[(chunk[j] >> shift) & dmask], 1u);
+    }
+    cluster.sync();  // every CTA's histogram is complete
+    tk_merge_hist(sm, cluster, CS);
+    const uint32_t bin_count = tk_find_digit(sm.total, static_cast<uint32_t>(k), sm.red, sm.found + 2);
+    const uint32_t digit = sm.found[2], rem = sm.found[3];
+    __syncthreads();
+    const uint32_t above = static_cast<uint32_t>(k) - rem;
+    const uint32_t prefix1 = prefix0 | (digit << shift), pmask1 = pmask0 | (dmask << shift);
+    if (above + bin_count <= static_cast<uint32_t>(kTkCandCap)) {
+      if (threadIdx.x == 0) SD_PROBE_MARK(2, 2, bin_count);
+      topk_candidates<PER>(sm, cluster, CS, crank, row, b, k, s0, nvalid, prefix1, pmask1, shift, rem,
+                           bin_count, out, rm);
+      return;
+    }
+    // the full passes below start over and rewrite this CTA's histogram:
+    // first let every CTA finish reading it
+    cluster.sync();
+  }
 
   // ---- previous selection as a hint (exact for any hint) ----
   // P = the hint's distinct tokens below L. If |P| = k, the k-th largest key
@@ -295,11 +583,7 @@ __global__ void __launch_bounds__(kTkThreads, 2) topk_cluster_kernel(
         if ((u & pmask) == prefix && u <= hi_cut) atomicAdd(&sm.hist[(u >> shift) & dmask], 1u);
       }
       cluster.sync();  // every CTA's histogram is complete
-      for (int i = tid; i < kTkBins; i += kTkThreads) {
-        uint32_t v = 0;
-        for (int r = 0; r < CS; ++r) v += cluster.map_shared_rank(sm.hist, r)[i];
-        sm.total[i] = v;
-      }
+      tk_merge_hist(sm, cluster, CS);
       cluster.sync();  // nobody rewrites its histogram before all have read it
       // thread t owns bins 4t..4t+3; find the digit where the count of keys with
       // a larger-or-equal digit first reaches `remaining`
@@ -332,6 +616,7 @@ __global__ void __launch_bounds__(kTkThreads, 2) topk_cluster_kernel(
       prefix |= digit << shift;
       pmask |= dmask << shift;
       top = shift - 1;
+      if (threadIdx.x == 0) SD_PROBE_MARK(2, 2, bin_count);
       if (shift == 0) {            // every bit fixed: T is exact
         T = prefix;
         need_eq = rem;
@@ -380,11 +665,13 @@ __global__ void __launch_bounds__(kTkThreads, 2) topk_cluster_kernel(
       ++eq_before;
     }
   }
+  if (threadIdx.x == 0) SD_PROBE_MARK(2, 3, 0);
   cluster.sync();  // no CTA leaves while others may still read its shared memory
   // optional row ids: a separate pass over the finished output (written by
   // the whole cluster before the barrier), one block-table load per page run
   if (rm.rows != nullptr)
     for (int i = crank * kTkThreads + tid; i < rm.kpad; i += CS * kTkThreads) rm.put(row, b, i, i < k ? out[i] : -1, pc);
+  if (threadIdx.x == 0) SD_PROBE_MARK(2, 4, 0);
 }
 
 // Cluster size for rows of up to max_seqlen scores with PER scores per thread

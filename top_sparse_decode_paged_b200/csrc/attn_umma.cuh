@@ -34,7 +34,9 @@
 // zeros. Measured on the part: scattered 1152-byte rows stream from HBM at
 // about 3.1 TB/s by cp.async and 2.8 TB/s by 1-D bulk copies; pushing half of
 // each tile to the partner CTA over distributed shared memory was slower than
-// reading it twice through L2.
+// reading it twice through L2. Neither an L2 prefetch of upcoming rows nor
+// staging the next tile in the copy threads' registers shortened the tile
+// period.
 //
 // Softmax: a 16-lane tensor-memory load spreads each warp's 16 heads over all
 // 32 threads (2 heads x 16 tokens each); max and sum are combined over the 4
@@ -50,7 +52,7 @@
 // 4-7 run the softmax, rescale and write partials (warp w owns TMEM lanes
 // 32*(w%4)..+31), warp 8 owns tensor memory and issues the S products, warp
 // 10 issues the P V products (each issuer blocks on its own inputs, in
-// order), warp 9 streams row ids and has their rows prefetched into L2.
+// order), warp 9 streams row ids.
 // Every wait is bounded (a timeout flags SD_DEVERR_TIMEOUT).
 #pragma once
 
@@ -69,10 +71,10 @@ constexpr int kAuChunkBytes = kAuTile * 128;              // 8 KB
 constexpr int kAuTileBytes = kAuChunks * kAuChunkBytes;   // 72 KB
 constexpr int kAuQChunkBytes = kAuHalfHeads * 128;        // 8 KB
 constexpr int kAuQBytes = kAuChunks * kAuQChunkBytes;     // 72 KB
-constexpr int kAuPBytes = kAuHalfHeads * 128;             // 8 KB: 64 head rows of up to 64 tokens
+constexpr int kAuPChunk = kAuChunks - 1;  // P^T (64 heads x 64 tokens) goes into the tile's rope chunk once S is done
 constexpr int kAuBufs = 2;
 constexpr int kAuThreads = 352;
-constexpr int kAuRidSlots = 4;             // row-id lookahead (tiles); rows are prefetched into L2 as their ids enter the ring
+constexpr int kAuRidSlots = 4;             // row-id lookahead (tiles)
 constexpr int kAuRanges = 74;              // CTA pairs: 148 CTAs, one per SM
 constexpr float kAuRescaleLog2 = 8.0f;     // lazy rescale threshold (log2 units)
 static_assert(kAuTile % 32 == 0 && kAuTile <= 64, "tile of 32 or 64 tokens");
@@ -83,9 +85,8 @@ __host__ __device__ constexpr int attn_kpad(int k) { return (k + kAuTile - 1) / 
 struct AttnUmmaLayout {
   static constexpr int kOffQ = 0;
   static constexpr int kOffRing = kOffQ + kAuQBytes;
-  static constexpr int kOffP = kOffRing + kAuBufs * kAuTileBytes;
-  static constexpr int kOffBar = kOffP + kAuPBytes;
-  static constexpr int kNumBars = 2 * kAuBufs + 10 + 2 * kAuRidSlots;
+  static constexpr int kOffBar = kOffRing + kAuBufs * kAuTileBytes;
+  static constexpr int kNumBars = 4 * kAuBufs + 8 + 2 * kAuRidSlots;
   static constexpr int kOffRid = kOffBar + 8 * kNumBars;             // [slots][tile] pool row ids (-1: skip)
   static constexpr int kOffAlpha = kOffRid + 4 * kAuTile * kAuRidSlots;  // [64] rescale factors
   static constexpr int kOffMisc = kOffAlpha + 4 * kAuHalfHeads;
@@ -194,19 +195,18 @@ __global__ void __launch_bounds__(kAuThreads, 1) attn_mla_umma_kernel(
   uint8_t* smem = smem_dyn + (((raw + 1023u) & ~1023u) - raw);
   uint8_t* qbuf = smem + Lay::kOffQ;
   uint8_t* ring = smem + Lay::kOffRing;
-  uint8_t* pbuf = smem + Lay::kOffP;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::kOffBar);
   uint64_t* tile_full = bars;                    // [bufs] 128 copy-thread arrivals (cp.async)
   uint64_t* tile_empty = bars + kAuBufs;         // [bufs] MMA commit after the tile's P V
-  uint64_t* q_full = bars + 2 * kAuBufs;         // 1 arrival + the Q bytes (TMA)
+  uint64_t* p_full = bars + 2 * kAuBufs;         // [bufs] the four softmax warps: P^T of the slot's tile written
+  uint64_t* pv_done = bars + 3 * kAuBufs;        // [bufs] MMA commit after the slot's tile's P V
+  uint64_t* q_full = bars + 4 * kAuBufs;         // 1 arrival + the Q bytes (TMA)
   uint64_t* q_empty = q_full + 1;                // MMA commit after a request's last S
   uint64_t* s_full = q_full + 2;                 // [2] MMA commit
   uint64_t* s_free = q_full + 4;                 // [2] the four softmax warps have read S
-  uint64_t* p_full = q_full + 6;                 // the four epilogue warps: P written, O rescaled/read out
-  uint64_t* pv_done = q_full + 7;                // MMA commit after P V
-  uint64_t* mma_fin = q_full + 8;                // S issuer's commit at exit
-  uint64_t* pv_fin = q_full + 9;                 // P V issuer's commit at exit
-  uint64_t* rid_full = q_full + 10;              // [slots] 32 row-id lanes (cp.async)
+  uint64_t* mma_fin = q_full + 6;                // S issuer's commit at exit
+  uint64_t* pv_fin = q_full + 7;                 // P V issuer's commit at exit
+  uint64_t* rid_full = q_full + 8;               // [slots] 32 row-id lanes (cp.async)
   uint64_t* rid_empty = rid_full + kAuRidSlots;  // [slots] 4 copy warps + the epilogue
   int32_t* rid = reinterpret_cast<int32_t*>(smem + Lay::kOffRid);
   float* alpha_s = reinterpret_cast<float*>(smem + Lay::kOffAlpha);
@@ -223,6 +223,8 @@ __global__ void __launch_bounds__(kAuThreads, 1) attn_mla_umma_kernel(
     for (int i = 0; i < kAuBufs; ++i) {
       sm100::mbar_init(&tile_full[i], 128);
       sm100::mbar_init(&tile_empty[i], 1);
+      sm100::mbar_init(&p_full[i], 4);
+      sm100::mbar_init(&pv_done[i], 1);
     }
     sm100::mbar_init(q_full, 1);
     sm100::mbar_init(q_empty, 1);
@@ -230,8 +232,6 @@ __global__ void __launch_bounds__(kAuThreads, 1) attn_mla_umma_kernel(
       sm100::mbar_init(&s_full[i], 1);
       sm100::mbar_init(&s_free[i], 4);
     }
-    sm100::mbar_init(p_full, 4);
-    sm100::mbar_init(pv_done, 1);
     sm100::mbar_init(mma_fin, 1);
     sm100::mbar_init(pv_fin, 1);
     for (int i = 0; i < kAuRidSlots; ++i) {
@@ -375,44 +375,70 @@ __global__ void __launch_bounds__(kAuThreads, 1) attn_mla_umma_kernel(
       }
       uint32_t pk[2][kReps];  // [head][rr]: bf16 pair of tokens 8 rr + 2 tq + {0, 1}
       bool need = false;
+      // scaled logits (log2 units) of this thread's 2 heads x 2 kReps tokens;
+      // skipped tokens are -inf, which the exponential maps to 0
+      float y[2][2 * kReps];
+#pragma unroll
+      for (int e = 0; e < 2; ++e)
+#pragma unroll
+        for (int q = 0; q < 2 * kReps; ++q)
+          y[e][q] = ((vb >> q) & 1u) ? __uint_as_float(r[4 * (q >> 1) + 2 * e + (q & 1)]) * scale_log2 : -INFINITY;
+      float mx[2];
 #pragma unroll
       for (int e = 0; e < 2; ++e) {
-        float mx = -INFINITY;
+        float a[kReps];
 #pragma unroll
-        for (int rr = 0; rr < kReps; ++rr) {
-          if ((vb >> (2 * rr)) & 1u) mx = fmaxf(mx, __uint_as_float(r[4 * rr + 2 * e]) * scale_log2);
-          if ((vb >> (2 * rr + 1)) & 1u) mx = fmaxf(mx, __uint_as_float(r[4 * rr + 2 * e + 1]) * scale_log2);
-        }
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-        const bool ne = mx > m_ref[e] + kAuRescaleLog2 || (m_ref[e] == -INFINITY && mx > -INFINITY);
+        for (int i = 0; i < kReps; ++i) a[i] = fmaxf(y[e][2 * i], y[e][2 * i + 1]);
+#pragma unroll
+        for (int w2 = kReps / 2; w2 > 0; w2 >>= 1)
+#pragma unroll
+          for (int i = 0; i < w2; ++i) a[i] = fmaxf(a[i], a[i + w2]);
+        mx[e] = a[0];
+      }
+#pragma unroll
+      for (int e = 0; e < 2; ++e) mx[e] = fmaxf(mx[e], __shfl_xor_sync(0xffffffffu, mx[e], 1));
+#pragma unroll
+      for (int e = 0; e < 2; ++e) mx[e] = fmaxf(mx[e], __shfl_xor_sync(0xffffffffu, mx[e], 2));
+      float m_use[2];
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const bool ne = mx[e] > m_ref[e] + kAuRescaleLog2 || (m_ref[e] == -INFINITY && mx[e] > -INFINITY);
         float alpha = 1.f;
         if (ne) {
-          alpha = exp2f(m_ref[e] - mx);  // 0 when m_ref is -inf
+          alpha = exp2f(m_ref[e] - mx[e]);  // 0 when m_ref is -inf
           l_sum[e] *= alpha;
-          m_ref[e] = mx;
+          m_ref[e] = mx[e];
         }
         need = need || ne;
         if (tq == 0) alpha_s[h0 + 8 * e] = alpha;
-        const float m_use = m_ref[e] == -INFINITY ? 0.f : m_ref[e];
+        m_use[e] = m_ref[e] == -INFINITY ? 0.f : m_ref[e];
+      }
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        float l0 = 0.f, l1 = 0.f;
 #pragma unroll
         for (int rr = 0; rr < kReps; ++rr) {
-          const float p0 = ((vb >> (2 * rr)) & 1u)
-                               ? sm100::ex2_approx(__uint_as_float(r[4 * rr + 2 * e]) * scale_log2 - m_use) : 0.f;
-          const float p1 = ((vb >> (2 * rr + 1)) & 1u)
-                               ? sm100::ex2_approx(__uint_as_float(r[4 * rr + 2 * e + 1]) * scale_log2 - m_use) : 0.f;
+          const float p0 = sm100::ex2_approx(y[e][2 * rr] - m_use[e]);
+          const float p1 = sm100::ex2_approx(y[e][2 * rr + 1] - m_use[e]);
           const __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
-          l_sum[e] += __low2float(h2) + __high2float(h2);
+          l0 += __low2float(h2);
+          l1 += __high2float(h2);
           pk[e][rr] = *reinterpret_cast<const uint32_t*>(&h2);
         }
+        l_sum[e] += l0 + l1;
       }
       // earlier tiles of this request are in O: rescale when any head's
       // reference moved (alpha_s published by the barrier)
       const bool rescale = sm100::named_bar_or(2, 128, need && !seg_first);
       if (threadIdx.x == 128) SD_PROBE_MARK(3, 8, j);
-      // O and the P buffer are free once the previous P V has completed
-      if (j > 0) {
-        bool okp = sm100::mbar_wait(pv_done, static_cast<uint32_t>((j - 1) & 1)) && !*abort_flag;
+      // P^T goes into this tile's rope chunk, which S has finished reading:
+      // no wait. A rescale of O waits for the previous tile's P V first (each
+      // slot's P V barrier is never waited more than one phase behind: the
+      // slot's next P V needs a P^T not yet written).
+      if (rescale && j > 0) {
+        const long long jp = j - 1;
+        bool okp = sm100::mbar_wait(&pv_done[jp % kAuBufs], static_cast<uint32_t>((jp / kAuBufs) & 1)) &&
+                   !*abort_flag;
         okp = sm100::named_bar_and(3, 128, okp);
         if (!okp) { *abort_flag = 1; break; }
         sm100::tc_fence_after();
@@ -438,7 +464,8 @@ __global__ void __launch_bounds__(kAuThreads, 1) attn_mla_umma_kernel(
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
           const int h = h0 + 8 * e;
-          uint8_t* prow = pbuf + (h >> 3) * 1024 + (h & 7) * 128 + 4 * tq;
+          uint8_t* prow = ring + (j % kAuBufs) * kAuTileBytes + kAuPChunk * kAuChunkBytes + (h >> 3) * 1024 +
+                          (h & 7) * 128 + 4 * tq;
 #pragma unroll
           for (int rr = 0; rr < kReps; ++rr) *reinterpret_cast<uint32_t*>(prow + ((rr ^ (h & 7)) << 4)) = pk[e][rr];
         }
@@ -446,14 +473,15 @@ __global__ void __launch_bounds__(kAuThreads, 1) attn_mla_umma_kernel(
       }
       sm100::tc_fence_before();
       __syncwarp();
-      if (lane == 0) sm100::mbar_arrive(p_full);
+      if (lane == 0) sm100::mbar_arrive(&p_full[j % kAuBufs]);
       if (threadIdx.x == 128) SD_PROBE_MARK(3, 3, j);
+      if (lane == 0 && warp > 4) SD_PROBE_MARK(3, 5 + warp, j);  // events 10-12: the other warps' P
 
       const int this_b = c.b;
       c.next(seqlens, B, seqlen_cap, k);
       const bool seg_last = !c.valid() || c.b != this_b;
       if (seg_last) {
-        bool okd = sm100::mbar_wait(pv_done, static_cast<uint32_t>(j & 1)) && !*abort_flag;
+        bool okd = sm100::mbar_wait(&pv_done[j % kAuBufs], static_cast<uint32_t>((j / kAuBufs) & 1)) && !*abort_flag;
         okd = sm100::named_bar_and(4, 128, okd);
         if (!okd) { *abort_flag = 1; break; }
         sm100::tc_fence_after();
@@ -528,19 +556,20 @@ __global__ void __launch_bounds__(kAuThreads, 1) attn_mla_umma_kernel(
     // P V(j) needs P(j) written (which follows S(j) and P V(j - 1)).
     if (sm100::elect_one()) {
       constexpr uint32_t idesc_pv = sm100::idesc_bf16(128, kAuHalfHeads, true, false);
-      const uint32_t pa = smem_u32(pbuf);
       AttnCursor cp;
       cp.init(seqlens, B, seqlen_cap, k, first, count, breq);
       int prev_bp = -1;
       bool ok = true;
       for (long long ip = 0; ip < count && ok; ++ip) {
-        ok = sm100::mbar_wait(p_full, static_cast<uint32_t>(ip & 1)) && !*abort_flag;
+        ok = sm100::mbar_wait(&p_full[ip % kAuBufs], static_cast<uint32_t>((ip / kAuBufs) & 1)) && !*abort_flag;
         if (!ok) break;
+        SD_PROBE_MARK(3, 13, ip);
         sm100::tc_fence_after();
         const bool seg_first = cp.b != prev_bp;
         prev_bp = cp.b;
         const int slot = static_cast<int>(ip % kAuBufs);
         const uint32_t ta = smem_u32(ring + slot * kAuTileBytes);
+        const uint32_t pa = ta + kAuPChunk * kAuChunkBytes;
         // O^T += V^T P^T (chunks 2v, 2v+1 are value block v)
 #pragma unroll
         for (int v = 0; v < kAuVBlocks; ++v)
@@ -550,7 +579,7 @@ __global__ void __launch_bounds__(kAuThreads, 1) attn_mla_umma_kernel(
                                sm100::smem_desc_mn_sw128(ta + 2 * v * kAuChunkBytes + kk * 2048, kAuChunkBytes, 1024),
                                sm100::smem_desc_k_sw128(pa + 32 * kk), idesc_pv, !(seg_first && kk == 0));
         sm100::mma_commit(&tile_empty[slot]);
-        sm100::mma_commit(pv_done);
+        sm100::mma_commit(&pv_done[slot]);
         SD_PROBE_MARK(3, 4, ip);
         cp.next(seqlens, B, seqlen_cap, k);
       }
@@ -561,22 +590,11 @@ __global__ void __launch_bounds__(kAuThreads, 1) attn_mla_umma_kernel(
   } else if (warp == 9) {
     // ------------------------------ row ids ------------------------------
     // Streams each tile's resolved pool rows into a small ring, kAuRidSlots
-    // tiles ahead of the copies and the softmax, and asks L2 to prefetch
-    // those rows (one bulk prefetch per 1152-byte row) as their ids enter the
-    // ring, so that the gathers, a few tiles later, find them in L2 instead
-    // of waiting for HBM. The ids a prefetch needs are loaded one iteration
-    // ahead, so their latency overlaps the wait for a free ring slot.
+    // tiles ahead of the copies and the softmax.
     AttnCursor c;
     c.init(seqlens, B, seqlen_cap, k, first, count, breq);
     long long n = 0;
     bool ok = true;
-    int ids[kAuTileWords];
-    auto load_ids = [&](const AttnCursor& cc) {
-      const int32_t* src = rows + (size_t)(cc.b % breq) * kpad + cc.tile * kAuTile;
-#pragma unroll
-      for (int w = 0; w < kAuTileWords; ++w) ids[w] = __ldg(src + 32 * w + lane);
-    };
-    if (c.valid()) load_ids(c);
     while (c.valid() && ok) {
       const int rs = static_cast<int>(n % kAuRidSlots);
       ok = sm100::mbar_wait(&rid_empty[rs], static_cast<uint32_t>((n / kAuRidSlots) & 1) ^ 1) && !*abort_flag;
@@ -585,13 +603,8 @@ __global__ void __launch_bounds__(kAuThreads, 1) attn_mla_umma_kernel(
 #pragma unroll
       for (int w = 0; w < kAuTileWords; ++w) cp_async_4(&rid[rs * kAuTile + 32 * w + lane], src + 32 * w + lane);
       sm100::cp_async_arrive_noinc(&rid_full[rs]);
-      const __nv_bfloat16* kv = kvl.p[c.b / breq];
-#pragma unroll
-      for (int w = 0; w < kAuTileWords; ++w)
-        if (ids[w] >= 0) sm100::prefetch_l2_bulk(kv + (long long)ids[w] * kAuDk, kAuDk * 2);
       ++n;
       c.next(seqlens, B, seqlen_cap, k);
-      if (c.valid()) load_ids(c);
     }
     cp_async_wait<0>();
     if (!ok) *abort_flag = 1;

@@ -123,6 +123,17 @@ __device__ __forceinline__ long long total_tiles(const int32_t* seqlens, int B, 
   return n;
 }
 
+// max(0, x) for an int32 dot product |x| < 2^31 - 2^23, on the FP32 pipe
+// (twice the INT32 pipe's rate, which the weighted sum keeps busy): as a
+// float, a nonnegative x is a nonnegative number (subnormals kept: no .ftz),
+// a negative x a negative number or a NaN, and max.f32 returns +0 for both.
+// Here |x| <= 128 * 128 * 128 = 2^21.
+__device__ __forceinline__ int32_t relu_on_fp_pipe(uint32_t x) {
+  uint32_t y;
+  asm("max.f32 %0, %1, %2;" : "=r"(y) : "r"(x), "r"(0u));
+  return static_cast<int32_t>(y);
+}
+
 template <class Cfg, int G, int HPG, int DI>
 __global__ void __launch_bounds__(kUmmaThreads, 1) indexer_umma_kernel(
     const __grid_constant__ CUtensorMap tm_keys, const __grid_constant__ CUtensorMap tm_q,
@@ -307,7 +318,7 @@ __global__ void __launch_bounds__(kUmmaThreads, 1) indexer_umma_kernel(
         const int slot = (nq - 1) & 1;
         const int ntiles = stage_tiles(c, kUmmaTile >> pshift, Lay::kTilesPerStage);
         if (!sm100::mbar_wait(&full[stage], phase)) { *abort_flag = 1; break; }
-        if (blockIdx.x % 37 == 0) SD_PROBE_MARK(1, 10, 0);
+        if (blockIdx.x % 37 == 0) SD_PROBE_MARK(1, 10, stage + kUmmaStages * static_cast<int>(phase));
         const uint32_t b0 = smem_u32(qbuf + slot * Lay::kQBytes);
         bool ok = true;
         for (int j = 0; j < ntiles; ++j) {
@@ -370,7 +381,7 @@ __global__ void __launch_bounds__(kUmmaThreads, 1) indexer_umma_kernel(
       const bool ok = sm100::mbar_wait(&accfull[acc], static_cast<uint32_t>((ti / kUmmaAccs) & 1));
       __syncwarp();  // tcgen05.ld is warp-collective: reconverge after the polling loop
       if (!ok) { *abort_flag = 1; break; }
-      if (blockIdx.x % 37 == 0 && quarter == 0 && lane == 0) SD_PROBE_MARK(1, 11 + set, 0);
+      if (blockIdx.x % 37 == 0 && quarter == 0 && lane == 0) SD_PROBE_MARK(1, 11 + set, ti >> 1);
       sm100::tc_fence_after();
       uint32_t r[HI];
 #pragma unroll
@@ -392,7 +403,7 @@ __global__ void __launch_bounds__(kUmmaThreads, 1) indexer_umma_kernel(
           for (int i = 0; i < kPart; ++i) part[i] = 0;
 #pragma unroll
           for (int i = 0; i < HPG; ++i)
-            part[i % kPart] += wreg[g * HPG + i] * max(static_cast<int32_t>(r[g * HPG + i]), 0);
+            part[i % kPart] += wreg[g * HPG + i] * relu_on_fp_pipe(r[g * HPG + i]);
           int32_t s = 0;
 #pragma unroll
           for (int i = 0; i < kPart; ++i) s += part[i];

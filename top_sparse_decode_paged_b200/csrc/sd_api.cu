@@ -854,17 +854,17 @@ const char* sd_status_str(sd_status status) {
 }
 
 #ifdef SD_PROBE
-// Probe builds only: copies up to `max_records` probe records (4 x u64 each)
-// to host memory, resets the ring and returns how many were recorded.
-int64_t sd_probe_read(void* dst, int64_t max_records) {
-  unsigned int n = 0;
-  if (cudaDeviceSynchronize() != cudaSuccess || cudaMemcpyFromSymbol(&n, sd::g_probe_n, sizeof(n)) != cudaSuccess)
+// Probe builds only: copies the probe slots (u64 ns, [4][1024][16][64], 0 =
+// not recorded) to host memory if dst is not NULL, then clears them.
+int64_t sd_probe_read(void* dst, int64_t max_bytes) {
+  const size_t n = sizeof(sd::g_probe);
+  if (cudaDeviceSynchronize() != cudaSuccess) return -1;
+  if (dst != nullptr && max_bytes >= (int64_t)n && cudaMemcpyFromSymbol(dst, sd::g_probe, n) != cudaSuccess) return -1;
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, sd::g_probe) != cudaSuccess || cudaMemset(p, 0, n) != cudaSuccess ||
+      cudaDeviceSynchronize() != cudaSuccess)
     return -1;
-  const unsigned int m = static_cast<unsigned int>(std::min<int64_t>(std::min(n, sd::kProbeCap), max_records));
-  if (m > 0 && dst != nullptr && cudaMemcpyFromSymbol(dst, sd::g_probe, (size_t)m * 32) != cudaSuccess) return -1;
-  const unsigned int zero = 0;
-  if (cudaMemcpyToSymbol(sd::g_probe_n, &zero, sizeof(zero)) != cudaSuccess) return -1;
-  return n;
+  return (int64_t)n;
 }
 #endif
 

@@ -18,25 +18,18 @@ __device__ unsigned int g_error_bits;
 __device__ __forceinline__ void raise_error(unsigned int bit) { atomicOr(&g_error_bits, bit); }
 
 // Timeline probes for tuning. Compiled out unless the library is built with
-// -DSD_PROBE; then each mark appends (globaltimer ns, SM clock, kernel / block
-// / event, value) to a device ring that sd_probe_read() copies out.
+// -DSD_PROBE; then a mark stores the globaltimer (ns) into a fixed slot
+// [kernel][block][event][index % 64] (a plain store: nothing waits on it),
+// which sd_probe_read() copies out.
 #ifdef SD_PROBE
-constexpr unsigned int kProbeCap = 1u << 20;
-__device__ unsigned long long g_probe[kProbeCap][4];
-__device__ unsigned int g_probe_n;
+constexpr int kProbeKernels = 4, kProbeBlocks = 1024, kProbeEvents = 16, kProbeIdx = 64;
+__device__ unsigned long long g_probe[kProbeKernels][kProbeBlocks][kProbeEvents][kProbeIdx];
 __device__ __forceinline__ void probe_mark(int kernel, int event, long long value) {
   unsigned long long t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  const unsigned int i = atomicAdd(&g_probe_n, 1u);
-  if (i < kProbeCap) {
-    unsigned int smid;
-    asm volatile("mov.u32 %0, %%smid;" : "=r"(smid));
-    g_probe[i][0] = t;
-    g_probe[i][1] = clock64();
-    g_probe[i][2] = ((unsigned long long)kernel << 56) | ((unsigned long long)event << 48) |
-                    ((unsigned long long)smid << 32) | (blockIdx.x + blockIdx.y * gridDim.x);
-    g_probe[i][3] = static_cast<unsigned long long>(value);
-  }
+  const unsigned int blk = blockIdx.x + blockIdx.y * gridDim.x;
+  if (kernel >= 1 && kernel <= kProbeKernels && blk < kProbeBlocks && event < kProbeEvents)
+    g_probe[kernel - 1][blk][event][static_cast<unsigned int>(value) % kProbeIdx] = t;
 }
 #define SD_PROBE_MARK(k, e, v) ::sd::probe_mark((k), (e), (v))
 #else

@@ -41,6 +41,9 @@
  *     be captured in a CUDA graph. Buffers keep the addresses the caller gives.
  *   - `workspace` is caller-owned device scratch of at least the size that
  *     sd_workspace_size() returns for the same shape (256-byte aligned).
+ *   - The library sets each kernel's shared-memory limit once per device and
+ *     remembers it. A device reset (cudaDeviceReset) clears such settings:
+ *     unload the library (or restart the process) after one.
  *   - Argument errors are found on the host before any launch and returned as
  *     a status; nothing is enqueued then. Errors in device-resident data (a
  *     seqlen beyond the block table, a block-table entry outside the pool, an

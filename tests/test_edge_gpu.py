@@ -153,15 +153,18 @@ def _indices_vs_oracle(wl):
     return got
 
 
-def test_topk_two_level_ties_at_the_threshold():
+@pytest.mark.parametrize("n_hot", [3000, 5000])
+def test_topk_two_level_ties_at_the_threshold(n_hot):
     """Scores take two values; more tokens hold the high value than k, so the
-    threshold is the high value and the lowest-index ones must win."""
+    threshold is the high value and the lowest-index ones must win. With 3000
+    tied keys the top-k resolves them as candidates in one CTA; with 5000
+    (more than its candidate capacity) it takes the full radix passes."""
     wl = W.make(W.spec("b4_l4096_mla", B=2, seqlens=(20000, 9000), seed=41))
     rng = np.random.default_rng(5)
     wl.ki_pages[:] = 0
     row = rng.integers(-64, 65, size=128).astype(np.int8)
     for b, L in enumerate(wl.seqlens):
-        hot = rng.choice(int(L), size=3000, replace=False)   # > k = 2048
+        hot = rng.choice(int(L), size=n_hot, replace=False)   # > k = 2048
         for t in hot:
             wl.ki_pages[wl.block_table[b, t // 64], t % 64, 0] = row
     _indices_vs_oracle(wl)

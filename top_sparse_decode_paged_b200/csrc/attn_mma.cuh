@@ -9,8 +9,11 @@
 // sparse attention", Walkthrough: selected-token MLA over NHD latent caches).
 //
 // Work split: one CTA per (request, KV head, block of HB query heads, split of
-// the k index slots). Each CTA streams its slots in tiles of 64 rows, gathered
-// with cp.async into padded shared rows (double buffered). Per tile:
+// the k index slots). Each CTA first resolves all of its slots to pool rows
+// (index load, then block-table load: every thread's lookups in flight
+// together, into shared memory), then streams its slots in tiles of 64 rows,
+// gathered with cp.async into padded shared rows (double buffered), so no
+// dependent lookup sits between two tiles. Per tile:
 //   S = Q K^T on tensor cores (warps split the 64 tokens), an online softmax
 //   whose row maxima and sums are shared through shared memory, P written to
 //   shared memory as bf16, then O += P V (warps split the value columns).
@@ -34,15 +37,14 @@ struct AttnMmaCfg {
   static constexpr int PS = kAttnTile + 8;
   static constexpr int DV_PER_WARP = DV / 4;  // value columns per warp
   static constexpr int NV8 = DV_PER_WARP / 8; // n8 tiles per warp in P.V
-  static size_t smem_bytes(bool separate_v) {
-    size_t s = 0;
+  // shared memory for a split of `slots` index slots
+  static size_t smem_bytes(bool separate_v, int slots) {
+    size_t s = sizeof(long long) * ((slots + kAttnTile - 1) / kAttnTile) * kAttnTile;  // resolved rows
     s += sizeof(__nv_bfloat16) * HB * KS;                        // Q
     s += sizeof(__nv_bfloat16) * 2 * kAttnTile * KS;             // K tiles
     if (separate_v) s += sizeof(__nv_bfloat16) * 2 * kAttnTile * VS;  // V tiles
     s += sizeof(__nv_bfloat16) * HB * PS;                        // P
     s += sizeof(float) * 2 * 4 * HB;                             // row max / sum partials
-    s += sizeof(long long) * 2 * kAttnTile;                      // row ids
-    s += sizeof(int) * 2;                                        // tile has rows
     return s;
   }
 };
@@ -63,14 +65,14 @@ __global__ void __launch_bounds__(AttnMmaCfg<DK, DV, MT>::THREADS) attn_split_mm
   const bool separate_v = v_pages != nullptr;
 
   extern __shared__ __align__(16) unsigned char smem_raw[];
-  __nv_bfloat16* sQ = reinterpret_cast<__nv_bfloat16*>(smem_raw);
+  long long* sRow = reinterpret_cast<long long*>(smem_raw);  // the split's resolved pool rows (-1: skip)
+  __nv_bfloat16* sQ = reinterpret_cast<__nv_bfloat16*>(
+      smem_raw + sizeof(long long) * ((slots_per_split + kAttnTile - 1) / kAttnTile) * kAttnTile);
   __nv_bfloat16* sK = sQ + HB * KS;
   __nv_bfloat16* sV = sK + 2 * kAttnTile * KS;
   __nv_bfloat16* sP = separate_v ? sV + 2 * kAttnTile * VS : sV;
   float* sMax = reinterpret_cast<float*>(sP + HB * PS);
   float* sSum = sMax + 4 * HB;
-  long long* sRow = reinterpret_cast<long long*>(sSum + 4 * HB);
-  int* sAny = reinterpret_cast<int*>(sRow + 2 * kAttnTile);
 
   const int split = blockIdx.x;
   const int hb = blockIdx.y;
@@ -96,45 +98,40 @@ __global__ void __launch_bounds__(AttnMmaCfg<DK, DV, MT>::THREADS) attn_split_mm
   }
   cp_async_commit();
 
+  // every slot of the split resolved to its pool row, lookups in flight together
   const int32_t* idx_row = indices + (size_t)bg * k;
-  auto load_rows = [&](int tile, int buf) {
-    int any = 0;
-    if (tid < kAttnTile) {
-      const int slot = slot0 + tile * kAttnTile + tid;
-      long long rid = -1;
-      if (slot < slot1) {
-        const int t = idx_row[slot];
-        if (t >= 0) {
-          if (t >= L) {
-            raise_error(SD_DEVERR_INDEX);
+  for (int i = tid; i < ntiles * kAttnTile; i += C::THREADS) {
+    const int slot = slot0 + i;
+    long long rid = -1;
+    if (slot < slot1) {
+      const int t = idx_row[slot];
+      if (t >= 0) {
+        if (t >= L) {
+          raise_error(SD_DEVERR_INDEX);
+        } else {
+          const int page = block_table[(size_t)b * max_pages + t / page_size];
+          if (page < 0 || page >= num_pages) {
+            raise_error(SD_DEVERR_PAGE);
           } else {
-            const int page = block_table[(size_t)b * max_pages + t / page_size];
-            if (page < 0 || page >= num_pages) {
-              raise_error(SD_DEVERR_PAGE);
-            } else {
-              rid = ((long long)page * page_size + (t % page_size)) * G + g;
-            }
+            rid = ((long long)page * page_size + (t % page_size)) * G + g;
           }
         }
       }
-      sRow[buf * kAttnTile + tid] = rid;
-      any = rid >= 0;
     }
-    any = __syncthreads_or(any);  // uniform result
-    if (tid == 0) sAny[buf] = any;  // read again only after a later barrier
-    return any;
-  };
-  auto issue_copy = [&](int buf) {
+    sRow[i] = rid;
+  }
+  __syncthreads();
+  auto issue_copy = [&](int tile, int buf) {
     for (int c = tid; c < kAttnTile * (DK / 8); c += C::THREADS) {
       const int r = c / (DK / 8), ch = c % (DK / 8);
-      const long long rid = sRow[buf * kAttnTile + r];
+      const long long rid = sRow[tile * kAttnTile + r];
       const __nv_bfloat16* src = k_pages + (rid >= 0 ? rid : 0) * DK + ch * 8;
       cp_async_16(sK + (buf * kAttnTile + r) * KS + ch * 8, src, rid >= 0 ? 16 : 0);
     }
     if (separate_v) {
       for (int c = tid; c < kAttnTile * (DV / 8); c += C::THREADS) {
         const int r = c / (DV / 8), ch = c % (DV / 8);
-        const long long rid = sRow[buf * kAttnTile + r];
+        const long long rid = sRow[tile * kAttnTile + r];
         const __nv_bfloat16* src = v_pages + (rid >= 0 ? rid : 0) * DV + ch * 8;
         cp_async_16(sV + (buf * kAttnTile + r) * VS + ch * 8, src, rid >= 0 ? 16 : 0);
       }
@@ -149,20 +146,19 @@ __global__ void __launch_bounds__(AttnMmaCfg<DK, DV, MT>::THREADS) attn_split_mm
   for (int i = 0; i < C::NV8; ++i) o_acc[i][0] = o_acc[i][1] = o_acc[i][2] = o_acc[i][3] = 0.f;
 
   if (ntiles > 0) {
-    if (load_rows(0, 0)) issue_copy(0);
+    issue_copy(0, 0);
     cp_async_commit();
   }
   for (int tile = 0; tile < ntiles; ++tile) {
     const int buf = tile & 1, nb = buf ^ 1;
     if (tile + 1 < ntiles) {
-      if (load_rows(tile + 1, nb)) issue_copy(nb);  // includes a barrier
+      issue_copy(tile + 1, nb);  // buffer nb (tile - 1) was released by the last barrier of that tile
       cp_async_commit();
       cp_async_wait<1>();
     } else {
       cp_async_wait<0>();
     }
     __syncthreads();
-    if (!sAny[buf]) continue;  // uniform: every row of this tile was skipped
 
     const __nv_bfloat16* kt = sK + buf * kAttnTile * KS;
     const __nv_bfloat16* vt = separate_v ? sV + buf * kAttnTile * VS : kt;
@@ -185,7 +181,7 @@ __global__ void __launch_bounds__(AttnMmaCfg<DK, DV, MT>::THREADS) attn_split_mm
     }
 
     // ---- online softmax across the 4 token quarters ----
-    const long long* rows = sRow + buf * kAttnTile;
+    const long long* rows = sRow + tile * kAttnTile;
     float tmax[2] = {-INFINITY, -INFINITY};
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt) {

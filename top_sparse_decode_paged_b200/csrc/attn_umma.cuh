@@ -632,7 +632,7 @@ constexpr int kAuMaxSeg = kMaxTopK / kAuTile;
 constexpr int kAuCombineHeads = 16;  // heads (warps) per block
 constexpr int kAuSegPerLane = (kAuMaxSeg + 31) / 32;
 
-__global__ void __launch_bounds__(32 * kAuCombineHeads) attn_mla_umma_combine_kernel(
+__global__ void __launch_bounds__(32 * kAuCombineHeads, 2) attn_mla_umma_combine_kernel(
     const float* __restrict__ part_o, const float2* __restrict__ part_ml, const int32_t* __restrict__ seqlens,
     int B, int breq, int k, int seqlen_cap, int n_ranges, __nv_bfloat16* __restrict__ out, float* __restrict__ lse) {
   pdl_wait();  // inputs come from earlier work in the stream
@@ -686,25 +686,38 @@ __global__ void __launch_bounds__(32 * kAuCombineHeads) attn_mla_umma_combine_ke
   float acc[16];
 #pragma unroll
   for (int i = 0; i < 16; ++i) acc[i] = 0.f;
-  for (uint32_t sg = 0; sg < nseg; ++sg) {
-    float wq = wgt[0];
+  // two segments' loads in flight at a time
+  for (uint32_t s0 = 0; s0 < nseg; s0 += 2) {
+    float4 v[2][4];
+    float ws[2];
 #pragma unroll
-    for (int q = 1; q < kAuSegPerLane; ++q)
-      if ((sg >> 5) == static_cast<uint32_t>(q)) wq = wgt[q];
-    const float ws = __shfl_sync(0xffffffffu, wq, static_cast<int>(sg & 31));
-    if (ws == 0.f) continue;  // uniform over the warp
-    const float4* src =
-        reinterpret_cast<const float4*>(part_o + (((size_t)seg_range(sg) + b) * kAuHeads + h) * kAuDv + 16 * lane);
-    float4 v[4];
+    for (int u = 0; u < 2; ++u) {
+      const uint32_t sg = s0 + u;
+      float wq = wgt[0];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) v[i] = src[i];
+      for (int q = 1; q < kAuSegPerLane; ++q)
+        if ((sg >> 5) == static_cast<uint32_t>(q)) wq = wgt[q];
+      ws[u] = __shfl_sync(0xffffffffu, wq, static_cast<int>(sg & 31));
+      if (sg < nseg && ws[u] != 0.f) {
+        const float4* src = reinterpret_cast<const float4*>(
+            part_o + (((size_t)seg_range(sg) + b) * kAuHeads + h) * kAuDv + 16 * lane);
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      acc[4 * i] += ws * v[i].x;
-      acc[4 * i + 1] += ws * v[i].y;
-      acc[4 * i + 2] += ws * v[i].z;
-      acc[4 * i + 3] += ws * v[i].w;
+        for (int i = 0; i < 4; ++i) v[u][i] = src[i];
+      } else {
+        ws[u] = 0.f;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) v[u][i] = make_float4(0.f, 0.f, 0.f, 0.f);
+      }
     }
+#pragma unroll
+    for (int u = 0; u < 2; ++u)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        acc[4 * i] += ws[u] * v[u][i].x;
+        acc[4 * i + 1] += ws[u] * v[u][i].y;
+        acc[4 * i + 2] += ws[u] * v[u][i].z;
+        acc[4 * i + 3] += ws[u] * v[u][i].w;
+      }
   }
   const float inv = denom > 0.f ? 1.f / denom : 0.f;
   uint32_t pk[8];

@@ -68,7 +68,7 @@ struct IndexerUmmaCfg {
 };
 // The MLA indexer (one KV head, 64 heads of 128 bytes) and the per-head
 // indexer (8 KV heads of 64 bytes, 4 heads each).
-using IdxCfgMla = IndexerUmmaCfg<1, 64, 128, 2, 6>;
+using IdxCfgMla = IndexerUmmaCfg<1, 64, 128, 4, 3>;
 using IdxCfgPerHead = IndexerUmmaCfg<8, 4, 64, 1, 3>;
 
 // Walks a contiguous range of the global tile list (request-major).

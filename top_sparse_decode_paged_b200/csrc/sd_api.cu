@@ -55,6 +55,31 @@ sd_status cuda_check(cudaError_t e) {
   return SD_ERR_CUDA;
 }
 
+// cudaFuncSetAttribute(MaxDynamicSharedMemorySize) once per (device, kernel,
+// size): the attribute outlives the call, and setting it on every launch
+// costs host time on the decode loop.
+sd_status set_smem_limit(const void* kern, size_t bytes) {
+  struct Entry { const void* k; int dev; size_t bytes; };
+  static std::mutex mu;
+  static Entry done[64];
+  static int n_done = 0;
+  int dev = 0;
+  sd_status s = cuda_check(cudaGetDevice(&dev));
+  if (s != SD_OK) return s;
+  std::lock_guard<std::mutex> lock(mu);
+  for (int i = 0; i < n_done; ++i)
+    if (done[i].k == kern && done[i].dev == dev && done[i].bytes >= bytes) return SD_OK;
+  s = cuda_check(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes)));
+  if (s != SD_OK) return s;
+  for (int i = 0; i < n_done; ++i)
+    if (done[i].k == kern && done[i].dev == dev) {
+      done[i].bytes = bytes;
+      return SD_OK;
+    }
+  if (n_done < 64) done[n_done++] = Entry{kern, dev, bytes};
+  return SD_OK;
+}
+
 sd_status after_launch() {
   ++t_launches;
   return cuda_check(cudaGetLastError());
@@ -162,8 +187,7 @@ sd_status launch_indexer_t(const int8_t* qi, const int32_t* w, const int8_t* ki,
                            int Hi, int max_seqlen, cudaStream_t st) {
   const size_t smem = sd::indexer_dp4a_smem(pd.kv_heads, Hi, DI);
   if (smem > 48 * 1024) {
-    const sd_status s = cuda_check(cudaFuncSetAttribute(sd::indexer_dp4a_kernel<DI>,
-                                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+    const sd_status s = set_smem_limit(reinterpret_cast<const void*>(sd::indexer_dp4a_kernel<DI>), smem);
     if (s != SD_OK) return s;
   }
   dim3 grid(sd::ceil_div(max_seqlen, sd::indexer_dp4a_tokens(pd.kv_heads, DI)), B);
@@ -256,8 +280,7 @@ sd_status launch_indexer_umma_t(const int8_t* qi, const int32_t* w, const int8_t
     tm_q = tm_keys;  // unused: the block-diagonal query operand is built in shared memory
   }
   auto kern = sd::indexer_umma_kernel<Cfg, G, HPG, DI>;
-  sd_status s = cuda_check(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                static_cast<int>(Cfg::kSmemAlloc)));
+  sd_status s = set_smem_limit(reinterpret_cast<const void*>(kern), Cfg::kSmemAlloc);
   if (s != SD_OK) return s;
   stage_mark(kStageIndexer, 0, st);
   s = launch_k(kern, dim3(sm_count()), dim3(sd::kUmmaThreads), Cfg::kSmemAlloc, st, tm_keys, tm_q, qi, w, bt,
@@ -282,8 +305,7 @@ sd_status launch_topk_cluster(const int32_t* scores, const int32_t* seqlens, int
                               int max_seqlen, int cap, int k, int cs, const sd::RowMap& rm, const int32_t* hint,
                               cudaStream_t st) {
   const size_t smem = sizeof(sd::TopkClusterSmem<PER>);
-  sd_status s = cuda_check(cudaFuncSetAttribute(sd::topk_cluster_kernel<PER>,
-                                                cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)));
+  sd_status s = set_smem_limit(reinterpret_cast<const void*>(sd::topk_cluster_kernel<PER>), smem);
   if (s != SD_OK) return s;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(cs, rows, 1);
@@ -355,10 +377,9 @@ sd_status launch_attn_t(const uint16_t* q, const uint16_t* kp, const uint16_t* v
                         const AttnPlan& p, float* part_o, float2* part_ml, int seqlen_cap,
                         cudaStream_t st) {
   using C = sd::AttnMmaCfg<DK, DV, MT>;
-  const size_t smem = C::smem_bytes(vp != nullptr);
+  const size_t smem = C::smem_bytes(vp != nullptr, p.slots_per_split);
   auto kern = sd::attn_split_mma_kernel<DK, DV, MT>;
-  sd_status s = cuda_check(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                static_cast<int>(smem)));
+  sd_status s = set_smem_limit(reinterpret_cast<const void*>(kern), smem);
   if (s != SD_OK) return s;
   const float scale_log2 = scale * 1.4426950408889634f;
   dim3 grid(p.n_splits, p.n_hb, B * pd.kv_heads);
@@ -404,8 +425,7 @@ sd_status launch_attn_umma(const uint16_t* q, const uint16_t* const* kp_layers, 
     if (kp_layers[l] == nullptr || (reinterpret_cast<uintptr_t>(kp_layers[l]) & 15u) != 0) return SD_ERR_UNSUPPORTED;
     kvl.p[l] = reinterpret_cast<const __nv_bfloat16*>(kp_layers[l]);
   }
-  sd_status s = cuda_check(cudaFuncSetAttribute(sd::attn_mla_umma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                static_cast<int>(Lay::kSmemAlloc)));
+  sd_status s = set_smem_limit(reinterpret_cast<const void*>(sd::attn_mla_umma_kernel), Lay::kSmemAlloc);
   if (s != SD_OK) return s;
   const float scale_log2 = scale * 1.4426950408889634f;
   stage_mark(kStageAttn, 0, st);
@@ -870,7 +890,7 @@ int64_t sd_probe_read(void* dst, int64_t max_bytes) {
 
 int32_t sd_last_cuda_error(void) { return t_last_cuda_error; }
 int32_t sd_last_launch_count(void) { return t_launches; }
-int32_t sd_version(void) { return (0 << 16) | 4; }
+int32_t sd_version(void) { return (0 << 16) | 5; }
 
 }  // extern "C"
 

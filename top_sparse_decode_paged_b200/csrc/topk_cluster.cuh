@@ -15,16 +15,16 @@
 //   - the final pass is an ordered compaction: per-thread counts of "greater"
 //     and "equal to the threshold" keys, one block scan, one cluster exchange
 //     of CTA totals, and each thread writes its picks in token order.
-// Candidate path (without a hint, whenever it applies, which is the common
-// case): after the first radix pass fixes the digit D holding the k-th
-// largest key, with A keys above it and c_D in it, and A + c_D <=
-// kTkCandCap, every CTA compacts its keys at or above D's range (in token
-// order), CTA 0 gathers the cluster's candidates and resolves the exact
-// threshold among the c_D keys of digit D by radix passes in its own shared
-// memory, then writes the output alone. That replaces the later cluster-wide
-// passes and the cluster compaction by one candidate exchange. Otherwise
-// (heavy ties, a digit holding too many keys, or a hint) the radix passes run
-// on the full slices as above.
+// Digit path (without a hint, the common case): the first radix pass fixes
+// the digit D holding the k-th largest key (A keys above it, c_D in it). When
+// c_D <= kTkDigitCap (a few dozen keys here), every CTA publishes its keys of
+// D and its count above D, gathers the cluster's keys of D over DSMEM, ranks
+// them to get the exact threshold, and writes its own slice's picks in token
+// order: four cluster barriers in all, no pass over the full row after the
+// first. When D holds more keys but A + c_D <= kTkCandCap, the candidate path
+// has CTA 0 gather every key at or above D and resolve the threshold alone.
+// Otherwise (heavy ties, or a hint) the radix passes run on the full slices
+// as above.
 // No CTA waits on another except at hardware cluster barriers.
 #pragma once
 
@@ -41,6 +41,7 @@ constexpr int kTkBinsBits = 11;
 constexpr int kTkBins = 1 << kTkBinsBits;
 constexpr int kTkMaxCluster = 8;
 constexpr int kTkCandCap = 4096;    // candidates (keys at or above the first pass's digit) the path takes
+constexpr int kTkDigitCap = 512;    // keys of the threshold digit the digit path resolves in every CTA
 
 // PER: scores per thread (16 or 32); a CTA holds a slice of 512 * PER scores.
 template <int PER>
@@ -188,6 +189,161 @@ __device__ __forceinline__ uint32_t tk_find_digit(const uint32_t* h, uint32_t re
   __syncthreads();
   const uint32_t bin_count = h[found[0]];
   return bin_count;
+}
+
+// The digit path (see the file comment): the first radix pass has fixed the
+// digit D of the k-th largest key, whose keys are those with (u & pmask1) ==
+// prefix1 (c_D <= kTkDigitCap of them over the cluster); `need` of them are
+// to be taken. Every CTA publishes its keys of D (in token order) and its
+// count of keys above D, gathers the cluster's keys of D (typically a few
+// dozen), ranks them to find
+// the exact threshold key Tk and how many keys equal to it to take, then
+// writes its own slice's picks in token order at the offset the earlier
+// CTAs' counts give.
+template <int PER>
+__device__ __forceinline__ void topk_digit_path(TopkClusterSmem<PER>& sm, cg::cluster_group& cluster, int CS,
+                                                int crank, int row, int b, int k, int s0, int nvalid,
+                                                uint32_t prefix1, uint32_t pmask1, uint32_t need, int32_t* out,
+                                                const RowMap& rm) {
+  const int tid = threadIdx.x;
+  const uint32_t hiD = prefix1 | ~pmask1;  // the largest key of digit D
+  uint32_t* dkey = sm.total;                // this CTA's keys of D
+  uint32_t* gkey = sm.total + kTkDigitCap;  // the cluster's keys of D
+  const uint32_t* chunk = sm.keys + tid * (PER + 1);
+  // 1. this CTA's counts above D and its keys of D
+  uint32_t kv[PER];
+  uint32_t n_above = 0, n_d = 0;
+#pragma unroll
+  for (int j = 0; j < PER; ++j) {
+    kv[j] = chunk[j];
+    if (j < nvalid) {
+      n_above += kv[j] > hiD;
+      n_d += (kv[j] & pmask1) == prefix1;
+    }
+  }
+  uint32_t tot;
+  const uint32_t pre = tk_block_excl_scan((n_above << 16) | n_d, sm.red, &tot);
+  uint32_t pos = pre & 0xffffu;
+#pragma unroll
+  for (int j = 0; j < PER; ++j)
+    if (j < nvalid && (kv[j] & pmask1) == prefix1) dkey[pos++] = kv[j];
+  if (tid == 0) {
+    sm.cta_vals[2] = tot >> 16;
+    sm.cta_vals[3] = tot & 0xffffu;
+  }
+  cluster.sync();  // every CTA's keys of D and counts are in place
+  uint32_t a_r[kTkMaxCluster], d_r[kTkMaxCluster];
+#pragma unroll
+  for (int r = 0; r < kTkMaxCluster; ++r) {
+    a_r[r] = 0u;
+    d_r[r] = 0u;
+    if (r < CS) {
+      const uint32_t* rv = cluster.map_shared_rank(sm.cta_vals, r);
+      a_r[r] = rv[2];
+      d_r[r] = rv[3];
+    }
+  }
+  uint32_t base_above = 0, base_d = 0, cD = 0;
+#pragma unroll
+  for (int r = 0; r < kTkMaxCluster; ++r) {
+    base_above += r < crank ? a_r[r] : 0u;
+    base_d += r < crank ? d_r[r] : 0u;
+    cD += d_r[r];
+  }
+  {
+    uint32_t off = 0;
+#pragma unroll
+    for (int r = 0; r < kTkMaxCluster; ++r) {
+      if (r < CS) {
+        const uint32_t* rk = cluster.map_shared_rank(dkey, r);
+        for (uint32_t i = tid; i < d_r[r]; i += kTkThreads) gkey[off + i] = rk[i];
+      }
+      off += d_r[r];
+    }
+  }
+  cluster.sync();  // every CTA has gathered: no more remote reads, any CTA may leave after this
+  // 2. the exact threshold: key x of D is Tk when fewer than `need` keys of D
+  // are above it and at least `need` are at or above it
+  for (uint32_t i = tid; i < cD; i += kTkThreads) {
+    const uint32_t x = gkey[i];
+    uint32_t gt = 0, ge = 0;
+    for (uint32_t q = 0; q < cD; ++q) {
+      const uint32_t y = gkey[q];
+      gt += y > x;
+      ge += y >= x;
+    }
+    if (gt < need && need <= ge) {
+      sm.found[0] = x;         // every such thread writes the same two values
+      sm.found[1] = need - gt;
+    }
+  }
+  __syncthreads();
+  const uint32_t Tk = sm.found[0], need_eq = sm.found[1];
+  // keys of D in earlier CTAs above / equal to Tk
+  uint32_t gtD = 0, eqD = 0;
+  for (uint32_t i = tid; i < base_d; i += kTkThreads) {
+    gtD += gkey[i] > Tk;
+    eqD += gkey[i] == Tk;
+  }
+  uint32_t tot2;
+  tk_block_excl_scan((gtD << 16) | eqD, sm.red, &tot2);
+  const uint32_t gt_base = base_above + (tot2 >> 16), eq_base = tot2 & 0xffffu;
+  // 3. this slice's picks in token order: every key above Tk, then the first
+  // need_eq keys equal to it over the cluster. They fill the output range
+  // [o0, o0 + n_out) of this CTA; they are staged in shared memory, then the
+  // indices and (in a decode step) the pool rows are written with every
+  // block-table load of a thread in flight together.
+  uint32_t n_gt = 0, n_eq = 0;
+#pragma unroll
+  for (int j = 0; j < PER; ++j) {
+    if (j < nvalid) {
+      n_gt += kv[j] > Tk;
+      n_eq += kv[j] == Tk;
+    }
+  }
+  uint32_t tot3;
+  const uint32_t pre3 = tk_block_excl_scan((n_gt << 16) | n_eq, sm.red, &tot3);
+  const uint32_t o0 = gt_base + min(eq_base, need_eq);
+  const uint32_t n_out = (tot3 >> 16) + min(eq_base + (tot3 & 0xffffu), need_eq) - min(eq_base, need_eq);
+  uint32_t gt_before = gt_base + (pre3 >> 16), eq_before = eq_base + (pre3 & 0xffffu);
+  uint32_t* stage = sm.hist;  // read by no CTA any more (the histogram merge is long done)
+#pragma unroll
+  for (int j = 0; j < PER; ++j) {
+    if (j < nvalid) {
+      const uint32_t u = kv[j];
+      const uint32_t g = static_cast<uint32_t>(s0 + tid * PER + j);
+      if (u > Tk) {
+        stage[gt_before + min(eq_before, need_eq) - o0] = g;
+        ++gt_before;
+      } else if (u == Tk) {
+        if (eq_before < need_eq) stage[gt_before + eq_before - o0] = g;
+        ++eq_before;
+      }
+    }
+  }
+  __syncthreads();
+  constexpr int kOutPerThr = (kMaxTopK + kTkThreads - 1) / kTkThreads;
+  int pages[kOutPerThr];
+#pragma unroll
+  for (int q = 0; q < kOutPerThr; ++q) {
+    const uint32_t i = tid + q * kTkThreads;
+    pages[q] = -1;
+    if (i < n_out) {
+      const int tok = static_cast<int>(stage[i]);
+      out[o0 + i] = tok;
+      if (rm.rows != nullptr) pages[q] = rm.block_table[(size_t)b * rm.max_pages + tok / rm.page_size];
+    }
+  }
+  if (rm.rows != nullptr) {
+#pragma unroll
+    for (int q = 0; q < kOutPerThr; ++q) {
+      const uint32_t i = tid + q * kTkThreads;
+      if (i < n_out) rm.put_page(row, static_cast<int>(o0 + i), static_cast<int>(stage[i]), pages[q]);
+    }
+    if (crank == 0)
+      for (int i = k + tid; i < rm.kpad; i += kTkThreads) rm.rows[(size_t)row * rm.kpad + i] = -1;
+  }
+  if (tid == 0) SD_PROBE_MARK(2, 5, cD);
 }
 
 // The candidate path (see the file comment). On entry the first radix pass
@@ -457,6 +613,11 @@ __global__ void __launch_bounds__(kTkThreads, 2) topk_cluster_kernel(
     __syncthreads();
     const uint32_t above = static_cast<uint32_t>(k) - rem;
     const uint32_t prefix1 = prefix0 | (digit << shift), pmask1 = pmask0 | (dmask << shift);
+    if (bin_count <= static_cast<uint32_t>(kTkDigitCap)) {
+      if (threadIdx.x == 0) SD_PROBE_MARK(2, 2, bin_count);
+      topk_digit_path<PER>(sm, cluster, CS, crank, row, b, k, s0, nvalid, prefix1, pmask1, rem, out, rm);
+      return;
+    }
     if (above + bin_count <= static_cast<uint32_t>(kTkCandCap)) {
       if (threadIdx.x == 0) SD_PROBE_MARK(2, 2, bin_count);
       topk_candidates<PER>(sm, cluster, CS, crank, row, b, k, s0, nvalid, prefix1, pmask1, shift, rem,

@@ -177,8 +177,8 @@ def test_topk_cluster_slices_with_ragged_rows():
 
 
 def test_topk_single_cta_fallback_beyond_cluster_capacity():
-    """max_seqlen above 8 x 16384 takes the one-CTA-per-row kernel."""
-    _indices_vs_oracle(W.make(W.spec("b4_l4096_mla", seqlens=(131073, 5000), seed=43)))
+    """max_seqlen above 8 x 32768 takes the one-CTA-per-row kernel."""
+    _indices_vs_oracle(W.make(W.spec("b4_l4096_mla", seqlens=(262145, 5000), seed=43)))
 
 
 def test_h128_k_at_least_seqlen_equals_dense_and_empty_request():

@@ -326,7 +326,7 @@ sd_status launch_topk_cluster(const int32_t* scores, const int32_t* seqlens, int
 }
 
 // Top-k: one thread-block cluster per row when the row fits in the cluster's
-// shared memory (max_seqlen <= 8 x 512 x 32), else one CTA per row over L2.
+// shared memory (max_seqlen <= 8 x 1024 x 32), else one CTA per row over L2.
 sd_status launch_topk(const int32_t* scores, const int32_t* seqlens, int32_t* indices, int B, int G,
                       int max_seqlen, int cap, int k, const sd::RowMap& rm, const int32_t* hint, cudaStream_t st) {
   const int rows = B * G;
@@ -334,10 +334,12 @@ sd_status launch_topk(const int32_t* scores, const int32_t* seqlens, int32_t* in
   const int cs32 = sd::topk_cluster_size(max_seqlen, 32);
   stage_mark(kStageTopk, 0, st);
   if ((cs16 > 0 || cs32 > 0) && rows <= 65535) {
-    // 32 scores per thread measured faster than 16 (fewer CTAs per cluster)
+    // Every CTA takes a whole SM: 16 scores per thread (more CTAs per row)
+    // while all rows' CTAs fit in one wave, else 32 (half the CTAs)
+    const bool per16 = cs16 > 0 && ((long long)rows * cs16 <= sm_count() || cs32 == 0);
     const sd_status s =
-        cs32 > 0 ? launch_topk_cluster<32>(scores, seqlens, indices, rows, G, max_seqlen, cap, k, cs32, rm, hint, st)
-                 : launch_topk_cluster<16>(scores, seqlens, indices, rows, G, max_seqlen, cap, k, cs16, rm, hint, st);
+        per16 ? launch_topk_cluster<16>(scores, seqlens, indices, rows, G, max_seqlen, cap, k, cs16, rm, hint, st)
+              : launch_topk_cluster<32>(scores, seqlens, indices, rows, G, max_seqlen, cap, k, cs32, rm, hint, st);
     stage_mark(kStageTopk, 1, st);
     ++t_launches;
     return s;

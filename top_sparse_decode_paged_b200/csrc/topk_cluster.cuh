@@ -3,7 +3,7 @@
 // Same result as topk_radix_kernel (score descending, ties to the lower token,
 // output in ascending token order, -1 padded), organised for B200:
 //   - a row of L scores is split over a cluster of CS CTAs (CS <= 8); each CTA
-//     copies its slice (512 threads x 16 or 32 scores) once from L2 into shared
+//     copies its slice (1024 threads x 16 or 32 scores) once from L2 into shared
 //     memory and never touches global memory again until it writes its part of
 //     the output;
 //   - a cluster-wide min/max fixes the highest bit in which the keys differ,
@@ -36,14 +36,15 @@ namespace sd {
 
 namespace cg = cooperative_groups;
 
-constexpr int kTkThreads = 512;
+constexpr int kTkThreads = 1024;  // one CTA per SM: 32 warps keep the latency-bound phases busy
 constexpr int kTkBinsBits = 11;
 constexpr int kTkBins = 1 << kTkBinsBits;
+constexpr int kTkBinsPerThr = kTkBins / kTkThreads;  // bins a thread owns when finding a digit
 constexpr int kTkMaxCluster = 8;
 constexpr int kTkCandCap = 4096;    // candidates (keys at or above the first pass's digit) the path takes
 constexpr int kTkDigitCap = 512;    // keys of the threshold digit the digit path resolves in every CTA
 
-// PER: scores per thread (16 or 32); a CTA holds a slice of 512 * PER scores.
+// PER: scores per thread (16 or 32); a CTA holds a slice of kTkThreads * PER scores.
 template <int PER>
 struct TopkClusterSmem {
   static constexpr int kStride = PER + 1;       // padded per-thread chunk (words)
@@ -58,7 +59,7 @@ struct TopkClusterSmem {
   static_assert(kTkThreads * kStride >= 2 * kTkCandCap, "candidate keys and tokens fit in the key area");
 };
 
-// Block-wide exclusive scan of 32-bit values (512 threads); returns the prefix,
+// Block-wide exclusive scan of 32-bit values (kTkThreads <= 1024); returns the prefix,
 // writes the total to *total.
 __device__ __forceinline__ uint32_t tk_block_excl_scan(uint32_t v, uint32_t* scratch, uint32_t* total) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -160,30 +161,32 @@ __device__ __forceinline__ void tk_merge_hist(Smem& sm, cg::cluster_group& clust
   __syncthreads();
 }
 
-// Finds the threshold digit of one radix pass: thread t owns bins 4t..4t+3 of
-// `h` (2048 bins); returns (digit, remaining) through found[0..1] and the
-// count of the digit's bin through the return value.
+// Finds the threshold digit of one radix pass: thread t owns the
+// kTkBinsPerThr bins from kTkBinsPerThr * t of `h` (2048 bins); the digit is
+// the bin where the count of keys in it and all higher bins first reaches
+// `remaining`. Returns (digit, remaining within it) through found[0..1] and
+// the count of the digit's bin through the return value.
 __device__ __forceinline__ uint32_t tk_find_digit(const uint32_t* h, uint32_t remaining, uint32_t* red,
                                                   uint32_t* found) {
   const int tid = threadIdx.x;
-  uint32_t c4[4], mine = 0;
+  uint32_t c[kTkBinsPerThr], mine = 0;
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    c4[i] = h[4 * tid + i];
-    mine += c4[i];
+  for (int i = 0; i < kTkBinsPerThr; ++i) {
+    c[i] = h[kTkBinsPerThr * tid + i];
+    mine += c[i];
   }
   uint32_t all;
-  const uint32_t rev = tk_block_excl_scan(mine, red, &all);  // keys in higher bins (reverse order)
-  const uint32_t above = all - rev - mine;
+  const uint32_t before = tk_block_excl_scan(mine, red, &all);  // keys in lower bins
+  const uint32_t above = all - before - mine;                   // keys in higher bins
   if (above < remaining && above + mine >= remaining) {
     uint32_t acc = above;
 #pragma unroll
-    for (int i = 3; i >= 0; --i) {
-      if (acc < remaining && acc + c4[i] >= remaining) {
-        found[0] = 4u * tid + i;
+    for (int i = kTkBinsPerThr - 1; i >= 0; --i) {
+      if (acc < remaining && acc + c[i] >= remaining) {
+        found[0] = static_cast<uint32_t>(kTkBinsPerThr * tid + i);
         found[1] = remaining - acc;
       }
-      acc += c4[i];
+      acc += c[i];
     }
   }
   __syncthreads();
@@ -232,6 +235,7 @@ __device__ __forceinline__ void topk_digit_path(TopkClusterSmem<PER>& sm, cg::cl
     sm.cta_vals[3] = tot & 0xffffu;
   }
   cluster.sync();  // every CTA's keys of D and counts are in place
+  if (tid == 0) SD_PROBE_MARK(2, 9, 0);
   uint32_t a_r[kTkMaxCluster], d_r[kTkMaxCluster];
 #pragma unroll
   for (int r = 0; r < kTkMaxCluster; ++r) {
@@ -262,6 +266,7 @@ __device__ __forceinline__ void topk_digit_path(TopkClusterSmem<PER>& sm, cg::cl
     }
   }
   cluster.sync();  // every CTA has gathered: no more remote reads, any CTA may leave after this
+  if (tid == 0) SD_PROBE_MARK(2, 10, 0);
   // 2. the exact threshold: key x of D is Tk when fewer than `need` keys of D
   // are above it and at least `need` are at or above it
   for (uint32_t i = tid; i < cD; i += kTkThreads) {
@@ -278,6 +283,7 @@ __device__ __forceinline__ void topk_digit_path(TopkClusterSmem<PER>& sm, cg::cl
     }
   }
   __syncthreads();
+  if (tid == 0) SD_PROBE_MARK(2, 11, 0);
   const uint32_t Tk = sm.found[0], need_eq = sm.found[1];
   // keys of D in earlier CTAs above / equal to Tk
   uint32_t gtD = 0, eqD = 0;
@@ -322,6 +328,7 @@ __device__ __forceinline__ void topk_digit_path(TopkClusterSmem<PER>& sm, cg::cl
     }
   }
   __syncthreads();
+  if (tid == 0) SD_PROBE_MARK(2, 12, 0);
   constexpr int kOutPerThr = (kMaxTopK + kTkThreads - 1) / kTkThreads;
   int pages[kOutPerThr];
 #pragma unroll
@@ -452,7 +459,7 @@ __device__ __forceinline__ void topk_candidates(TopkClusterSmem<PER>& sm, cg::cl
 
   // 3. ordered output: candidate i is taken if its key is above Tk (every key
   // of a digit above D is), or equal to Tk and among the first need_eq of
-  // those in token order; thread t handles candidates 8t..8t+7
+  // those in token order; thread t handles kPerThr consecutive candidates
   constexpr int kPerThr = kTkCandCap / kTkThreads;
   uint32_t n_gt = 0, n_eq = 0;
 #pragma unroll
@@ -511,7 +518,7 @@ __device__ __forceinline__ void topk_candidates(TopkClusterSmem<PER>& sm, cg::cl
 }
 
 template <int PER>
-__global__ void __launch_bounds__(kTkThreads, 2) topk_cluster_kernel(
+__global__ void __launch_bounds__(kTkThreads, 1) topk_cluster_kernel(
     const int32_t* __restrict__ scores, const int32_t* __restrict__ seqlens, int32_t* __restrict__ indices,
     int G, int max_seqlen, int seqlen_cap, int k, RowMap rm, const int32_t* __restrict__ hint) {
   pdl_wait();  // inputs come from earlier work in the stream
@@ -563,6 +570,7 @@ __global__ void __launch_bounds__(kTkThreads, 2) topk_cluster_kernel(
   }
   if (hint != nullptr)
     for (int i = tid; i < kTkThreads * PER / 32; i += kTkThreads) sm.mark[i] = 0u;
+  if (tid == 0) SD_PROBE_MARK(2, 6, 0);
   tk_block_minmax(kmin, kmax, sm.red);
   if (tid == 0) {
     sm.cta_vals[0] = kmin;
@@ -606,8 +614,10 @@ __global__ void __launch_bounds__(kTkThreads, 2) topk_cluster_kernel(
       const uint32_t* chunk = sm.keys + tid * kTkChunkStride;
       for (int j = 0; j < nvalid; ++j) atomicAdd(&sm.hist[(chunk[j] >> shift) & dmask], 1u);
     }
+    if (tid == 0) SD_PROBE_MARK(2, 7, 0);
     cluster.sync();  // every CTA's histogram is complete
     tk_merge_hist(sm, cluster, CS);
+    if (tid == 0) SD_PROBE_MARK(2, 8, 0);
     const uint32_t bin_count = tk_find_digit(sm.total, static_cast<uint32_t>(k), sm.red, sm.found + 2);
     const uint32_t digit = sm.found[2], rem = sm.found[3];
     __syncthreads();
@@ -746,33 +756,11 @@ __global__ void __launch_bounds__(kTkThreads, 2) topk_cluster_kernel(
       cluster.sync();  // every CTA's histogram is complete
       tk_merge_hist(sm, cluster, CS);
       cluster.sync();  // nobody rewrites its histogram before all have read it
-      // thread t owns bins 4t..4t+3; find the digit where the count of keys with
-      // a larger-or-equal digit first reaches `remaining`
-      uint32_t c4[4], mine = 0;
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        c4[i] = sm.total[4 * tid + i];
-        mine += c4[i];
-      }
-      uint32_t all;
-      // exclusive scan in reverse thread order = count of keys in higher bins
-      const uint32_t rev = tk_block_excl_scan(mine, sm.red, &all);
-      const uint32_t above = all - rev - mine;
-      if (above < remaining && above + mine >= remaining) {
-        uint32_t acc = above;
-#pragma unroll
-        for (int i = 3; i >= 0; --i) {
-          if (acc < remaining && acc + c4[i] >= remaining) {
-            sm.found[0] = 4u * tid + i;
-            sm.found[1] = remaining - acc;
-          }
-          acc += c4[i];
-        }
-      }
-      __syncthreads();
+      // the digit where the count of keys with a larger-or-equal digit first
+      // reaches `remaining`
+      const uint32_t bin_count = tk_find_digit(sm.total, remaining, sm.red, sm.found);
       const uint32_t digit = sm.found[0];
       const uint32_t rem = sm.found[1];
-      const uint32_t bin_count = sm.total[digit];
       __syncthreads();
       prefix |= digit << shift;
       pmask |= dmask << shift;

@@ -43,8 +43,8 @@ L2_FLUSH_BYTES = 256 << 20
 NCU_TRAFFIC = {
     # captured at --batch 16 (half the workload's 32 requests) and scaled by 2:
     # both kernels' traffic grows with the requests they process
-    ("b32_l65536_mla", "indexer"): (0x00000006, 2 * (134.464768e6 + 4.152320e6)),
-    ("b32_l65536_mla", "attn"): (0x00000006, 2 * (40.339712e6 + 1.163776e6)),
+    ("b32_l65536_mla", "indexer"): (0x00000007, 2 * (134.464000e6 + 4.018176e6)),
+    ("b32_l65536_mla", "attn"): (0x00000007, 2 * (40.339456e6 + 1.273856e6)),
 }
 
 

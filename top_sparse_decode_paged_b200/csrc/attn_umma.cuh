@@ -249,16 +249,19 @@ __global__ void __launch_bounds__(kAuThreads, 1) attn_mla_umma_kernel(
   sm100::tc_fence_before();
   __syncthreads();
   sm100::tc_fence_after();
-  // the set-up above reads no input: the previous kernel may still be running
+  // This range of the tile list follows from the sequence lengths alone. The
+  // caller owns them and no kernel of the library writes them, so they are
+  // read while the previous kernel may still be running; everything else
+  // waits for it.
+  const long long total = attn_total_tiles(seqlens, B, seqlen_cap, k, breq);
+  const long long first = total * range / n_ranges;
+  const long long count = total * (range + 1) / n_ranges - first;
   pdl_wait();
   pdl_trigger();
   const uint32_t tmem = *tmem_slot;
   const uint32_t tm_o = tmem;          // cols [0,256): O^T, block j at 64j
   const uint32_t tm_s = tmem + 256;    // S, two buffers of kAuTile columns
 
-  const long long total = attn_total_tiles(seqlens, B, seqlen_cap, k, breq);
-  const long long first = total * range / n_ranges;
-  const long long count = total * (range + 1) / n_ranges - first;
   if (threadIdx.x == 0) SD_PROBE_MARK(3, 0, count);
 
   if (warp < 4) {
@@ -635,9 +638,6 @@ constexpr int kAuSegPerLane = (kAuMaxSeg + 31) / 32;
 __global__ void __launch_bounds__(32 * kAuCombineHeads, 2) attn_mla_umma_combine_kernel(
     const float* __restrict__ part_o, const float2* __restrict__ part_ml, const int32_t* __restrict__ seqlens,
     int B, int breq, int k, int seqlen_cap, int n_ranges, __nv_bfloat16* __restrict__ out, float* __restrict__ lse) {
-  pdl_wait();  // inputs come from earlier work in the stream
-  pdl_trigger();
-  if (threadIdx.x == 0 && (blockIdx.x & 15) == 0) SD_PROBE_MARK(4, 0, 0);
   constexpr int HG = kAuHeads / kAuCombineHeads;
   const int b = blockIdx.x / HG;
   const int h = (blockIdx.x % HG) * kAuCombineHeads + (threadIdx.x >> 5);
@@ -665,6 +665,28 @@ __global__ void __launch_bounds__(32 * kAuCombineHeads, 2) attn_mla_umma_combine
     nseg = total >= nr ? range_of(before + mine - 1) - r0 + 1 : mine;
   }
   auto seg_range = [&](uint32_t sg) { return total >= nr ? r0 + sg : range_of(before + sg); };
+  // The segments above follow from the caller's sequence lengths, which no
+  // kernel of the library writes; the partials come from the attention.
+  pdl_wait();
+  pdl_trigger();
+  if (threadIdx.x == 0 && (blockIdx.x & 15) == 0) SD_PROBE_MARK(4, 0, 0);
+  // a segment's 16 values of this lane's columns (zeros past the last one):
+  // every written partial is finite, so rows of zero weight add nothing
+  auto load_seg = [&](uint32_t sg, float4 (&v)[4]) {
+    if (sg < nseg) {
+      const float4* src = reinterpret_cast<const float4*>(
+          part_o + (((size_t)seg_range(sg) + b) * kAuHeads + h) * kAuDv + 16 * lane);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) v[i] = src[i];
+    } else {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) v[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+  };
+  // the first segment's row loads together with every segment's (m, l): it
+  // does not depend on the weights
+  float4 v0[4];
+  load_seg(0, v0);
   float2 ml[kAuSegPerLane];
   float M = -INFINITY;
 #pragma unroll
@@ -683,41 +705,41 @@ __global__ void __launch_bounds__(32 * kAuCombineHeads, 2) attn_mla_umma_combine
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) denom += __shfl_xor_sync(0xffffffffu, denom, o);
-  float acc[16];
+  auto weight_of = [&](uint32_t sg) {
+    float wq = wgt[0];
 #pragma unroll
-  for (int i = 0; i < 16; ++i) acc[i] = 0.f;
-  // two segments' loads in flight at a time
-  for (uint32_t s0 = 0; s0 < nseg; s0 += 2) {
+    for (int q = 1; q < kAuSegPerLane; ++q)
+      if ((sg >> 5) == static_cast<uint32_t>(q)) wq = wgt[q];
+    const float ws = __shfl_sync(0xffffffffu, wq, static_cast<int>(sg & 31));
+    return sg < nseg ? ws : 0.f;
+  };
+  float acc[16];
+  {
+    const float w0 = weight_of(0);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      acc[4 * i] = w0 * v0[i].x;
+      acc[4 * i + 1] = w0 * v0[i].y;
+      acc[4 * i + 2] = w0 * v0[i].z;
+      acc[4 * i + 3] = w0 * v0[i].w;
+    }
+  }
+  // the other segments two at a time
+  for (uint32_t s0 = 1; s0 < nseg; s0 += 2) {
     float4 v[2][4];
-    float ws[2];
+    load_seg(s0, v[0]);
+    load_seg(s0 + 1, v[1]);
 #pragma unroll
     for (int u = 0; u < 2; ++u) {
-      const uint32_t sg = s0 + u;
-      float wq = wgt[0];
-#pragma unroll
-      for (int q = 1; q < kAuSegPerLane; ++q)
-        if ((sg >> 5) == static_cast<uint32_t>(q)) wq = wgt[q];
-      ws[u] = __shfl_sync(0xffffffffu, wq, static_cast<int>(sg & 31));
-      if (sg < nseg && ws[u] != 0.f) {
-        const float4* src = reinterpret_cast<const float4*>(
-            part_o + (((size_t)seg_range(sg) + b) * kAuHeads + h) * kAuDv + 16 * lane);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) v[u][i] = src[i];
-      } else {
-        ws[u] = 0.f;
-#pragma unroll
-        for (int i = 0; i < 4; ++i) v[u][i] = make_float4(0.f, 0.f, 0.f, 0.f);
-      }
-    }
-#pragma unroll
-    for (int u = 0; u < 2; ++u)
+      const float ws = weight_of(s0 + u);
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        acc[4 * i] += ws[u] * v[u][i].x;
-        acc[4 * i + 1] += ws[u] * v[u][i].y;
-        acc[4 * i + 2] += ws[u] * v[u][i].z;
-        acc[4 * i + 3] += ws[u] * v[u][i].w;
+        acc[4 * i] += ws * v[u][i].x;
+        acc[4 * i + 1] += ws * v[u][i].y;
+        acc[4 * i + 2] += ws * v[u][i].z;
+        acc[4 * i + 3] += ws * v[u][i].w;
       }
+    }
   }
   const float inv = denom > 0.f ? 1.f / denom : 0.f;
   uint32_t pk[8];

@@ -892,7 +892,7 @@ int64_t sd_probe_read(void* dst, int64_t max_bytes) {
 
 int32_t sd_last_cuda_error(void) { return t_last_cuda_error; }
 int32_t sd_last_launch_count(void) { return t_launches; }
-int32_t sd_version(void) { return (0 << 16) | 6; }
+int32_t sd_version(void) { return (0 << 16) | 7; }
 
 }  // extern "C"
 

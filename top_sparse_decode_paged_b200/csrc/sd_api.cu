@@ -300,16 +300,16 @@ sd_status launch_indexer_umma(const int8_t* qi, const int32_t* w, const int8_t* 
                                                            launched);
 }
 
-template <int PER>
+template <int PER, int NT>
 sd_status launch_topk_cluster(const int32_t* scores, const int32_t* seqlens, int32_t* indices, int rows, int G,
                               int max_seqlen, int cap, int k, int cs, const sd::RowMap& rm, const int32_t* hint,
                               cudaStream_t st) {
-  const size_t smem = sizeof(sd::TopkClusterSmem<PER>);
-  sd_status s = set_smem_limit(reinterpret_cast<const void*>(sd::topk_cluster_kernel<PER>), smem);
+  const size_t smem = sizeof(sd::TopkClusterSmem<PER, NT>);
+  sd_status s = set_smem_limit(reinterpret_cast<const void*>(sd::topk_cluster_kernel<PER, NT>), smem);
   if (s != SD_OK) return s;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(cs, rows, 1);
-  cfg.blockDim = dim3(sd::kTkThreads, 1, 1);
+  cfg.blockDim = dim3(NT, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
   cudaLaunchAttribute attr[2];
@@ -321,7 +321,7 @@ sd_status launch_topk_cluster(const int32_t* scores, const int32_t* seqlens, int
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = t_stage_count == 0 ? 2 : 1;  // see launch_k
-  return cuda_check(cudaLaunchKernelEx(&cfg, sd::topk_cluster_kernel<PER>, scores, seqlens, indices, G,
+  return cuda_check(cudaLaunchKernelEx(&cfg, sd::topk_cluster_kernel<PER, NT>, scores, seqlens, indices, G,
                                        std::max(max_seqlen, 1), cap, k, rm, hint));
 }
 
@@ -330,16 +330,22 @@ sd_status launch_topk_cluster(const int32_t* scores, const int32_t* seqlens, int
 sd_status launch_topk(const int32_t* scores, const int32_t* seqlens, int32_t* indices, int B, int G,
                       int max_seqlen, int cap, int k, const sd::RowMap& rm, const int32_t* hint, cudaStream_t st) {
   const int rows = B * G;
-  const int cs16 = sd::topk_cluster_size(max_seqlen, 16);
-  const int cs32 = sd::topk_cluster_size(max_seqlen, 32);
+  const long long sms = sm_count();
+  const int cs16 = sd::topk_cluster_size(max_seqlen, 16, 1024);   // 1024 threads, one CTA per SM
+  const int cs32 = sd::topk_cluster_size(max_seqlen, 32, 1024);
+  const int cs32h = sd::topk_cluster_size(max_seqlen, 32, 512);   // 512 threads, two CTAs per SM
   stage_mark(kStageTopk, 0, st);
   if ((cs16 > 0 || cs32 > 0) && rows <= 65535) {
-    // Every CTA takes a whole SM: 16 scores per thread (more CTAs per row)
-    // while all rows' CTAs fit in one wave, else 32 (half the CTAs)
-    const bool per16 = cs16 > 0 && ((long long)rows * cs16 <= sm_count() || cs32 == 0);
-    const sd_status s =
-        per16 ? launch_topk_cluster<16>(scores, seqlens, indices, rows, G, max_seqlen, cap, k, cs16, rm, hint, st)
-              : launch_topk_cluster<32>(scores, seqlens, indices, rows, G, max_seqlen, cap, k, cs32, rm, hint, st);
+    // All rows' CTAs in one wave if possible: 1024 threads x 16 scores (the
+    // most warps per row) when a CTA per SM is enough, else 512 x 32 when two
+    // per SM are, else 1024 x 32 (the fewest CTAs)
+    sd_status s;
+    if (cs16 > 0 && (long long)rows * cs16 <= sms)
+      s = launch_topk_cluster<16, 1024>(scores, seqlens, indices, rows, G, max_seqlen, cap, k, cs16, rm, hint, st);
+    else if (cs32h > 0 && (long long)rows * cs32h <= 2 * sms)
+      s = launch_topk_cluster<32, 512>(scores, seqlens, indices, rows, G, max_seqlen, cap, k, cs32h, rm, hint, st);
+    else  // cs32 > 0 here: a row that fits at 16 scores per thread fits at 32
+      s = launch_topk_cluster<32, 1024>(scores, seqlens, indices, rows, G, max_seqlen, cap, k, cs32, rm, hint, st);
     stage_mark(kStageTopk, 1, st);
     ++t_launches;
     return s;

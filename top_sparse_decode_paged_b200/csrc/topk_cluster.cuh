@@ -3,7 +3,7 @@
 // Same result as topk_radix_kernel (score descending, ties to the lower token,
 // output in ascending token order, -1 padded), organised for B200:
 //   - a row of L scores is split over a cluster of CS CTAs (CS <= 8); each CTA
-//     copies its slice (1024 threads x 16 or 32 scores) once from L2 into shared
+//     copies its slice (NT = 1024 or 512 threads x 16 or 32 scores) once from L2 into shared
 //     memory and never touches global memory again until it writes its part of
 //     the output;
 //   - a cluster-wide min/max fixes the highest bit in which the keys differ,
@@ -36,31 +36,33 @@ namespace sd {
 
 namespace cg = cooperative_groups;
 
-constexpr int kTkThreads = 1024;  // one CTA per SM: 32 warps keep the latency-bound phases busy
+// NT: threads per CTA, 1024 (one CTA per SM: 32 warps keep the latency-bound
+// phases busy) or 512 (two per SM, when that keeps every row in one wave).
+constexpr int kTkMaxThreads = 1024;
 constexpr int kTkBinsBits = 11;
 constexpr int kTkBins = 1 << kTkBinsBits;
-constexpr int kTkBinsPerThr = kTkBins / kTkThreads;  // bins a thread owns when finding a digit
 constexpr int kTkMaxCluster = 8;
 constexpr int kTkCandCap = 4096;    // candidates (keys at or above the first pass's digit) the path takes
 constexpr int kTkDigitCap = 512;    // keys of the threshold digit the digit path resolves in every CTA
 
-// PER: scores per thread (16 or 32); a CTA holds a slice of kTkThreads * PER scores.
-template <int PER>
+// PER: scores per thread (16 or 32); a CTA holds a slice of NT * PER scores.
+template <int PER, int NT>
 struct TopkClusterSmem {
   static constexpr int kStride = PER + 1;       // padded per-thread chunk (words)
-  uint32_t keys[kTkThreads * kStride];          // thread t's chunk at t*(PER+1) (bank-conflict free)
+  uint32_t keys[NT * kStride];          // thread t's chunk at t*(PER+1) (bank-conflict free)
   uint32_t hist[kTkCandCap];                    // this CTA's histogram (read by the cluster); CTA 0's candidate keys
   uint32_t total[kTkCandCap];                   // cluster-wide histogram; CTA 0's candidate tokens
-  uint32_t red[kTkThreads / 32 * 2 + 8];        // block reduction / scan scratch
+  uint32_t red[NT / 32 * 2 + 8];        // block reduction / scan scratch
   uint32_t cta_vals[4];                         // values this CTA publishes to the cluster
   uint32_t found[4];                            // threshold digit, remaining (and scratch)
-  uint32_t mark[kTkThreads * PER / 32];         // hint tokens of this CTA's slice (one bit each)
+  uint32_t mark[NT * PER / 32];         // hint tokens of this CTA's slice (one bit each)
   uint32_t hvals[4];                            // hint bounds this CTA publishes
-  static_assert(kTkThreads * kStride >= 2 * kTkCandCap, "candidate keys and tokens fit in the key area");
+  static_assert(NT * kStride >= 2 * kTkCandCap, "candidate keys and tokens fit in the key area");
 };
 
-// Block-wide exclusive scan of 32-bit values (kTkThreads <= 1024); returns the prefix,
+// Block-wide exclusive scan of 32-bit values (NT <= 1024); returns the prefix,
 // writes the total to *total.
+template <int NT>
 __device__ __forceinline__ uint32_t tk_block_excl_scan(uint32_t v, uint32_t* scratch, uint32_t* total) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   uint32_t incl = v;
@@ -72,24 +74,25 @@ __device__ __forceinline__ uint32_t tk_block_excl_scan(uint32_t v, uint32_t* scr
   if (lane == 31) scratch[warp] = incl;
   __syncthreads();
   if (warp == 0) {
-    const uint32_t w = lane < kTkThreads / 32 ? scratch[lane] : 0u;
+    const uint32_t w = lane < NT / 32 ? scratch[lane] : 0u;
     uint32_t wi = w;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       const uint32_t n = __shfl_up_sync(0xffffffffu, wi, o);
       if (lane >= o) wi += n;
     }
-    if (lane < kTkThreads / 32) scratch[lane] = wi - w;
-    if (lane == 31) scratch[kTkThreads / 32] = wi;
+    if (lane < NT / 32) scratch[lane] = wi - w;
+    if (lane == 31) scratch[NT / 32] = wi;
   }
   __syncthreads();
   const uint32_t r = scratch[warp] + incl - v;
-  *total = scratch[kTkThreads / 32];
+  *total = scratch[NT / 32];
   __syncthreads();
   return r;
 }
 
 // Block-wide minimum and maximum in one pass (two barriers).
+template <int NT>
 __device__ __forceinline__ void tk_block_minmax(uint32_t& mn, uint32_t& mx, uint32_t* scratch) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 #pragma unroll
@@ -105,13 +108,14 @@ __device__ __forceinline__ void tk_block_minmax(uint32_t& mn, uint32_t& mx, uint
   mn = 0xffffffffu;
   mx = 0u;
 #pragma unroll
-  for (int w = 0; w < kTkThreads / 32; ++w) {
+  for (int w = 0; w < NT / 32; ++w) {
     mn = min(mn, scratch[2 * w]);
     mx = max(mx, scratch[2 * w + 1]);
   }
   __syncthreads();
 }
 
+template <int NT>
 __device__ __forceinline__ uint32_t tk_block_reduce(uint32_t v, uint32_t* scratch, bool is_max) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 #pragma unroll
@@ -122,32 +126,32 @@ __device__ __forceinline__ uint32_t tk_block_reduce(uint32_t v, uint32_t* scratc
   if (lane == 0) scratch[warp] = v;
   __syncthreads();
   if (warp == 0) {
-    v = lane < kTkThreads / 32 ? scratch[lane] : (is_max ? 0u : 0xffffffffu);
+    v = lane < NT / 32 ? scratch[lane] : (is_max ? 0u : 0xffffffffu);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
       const uint32_t n = __shfl_xor_sync(0xffffffffu, v, o);
       v = is_max ? max(v, n) : min(v, n);
     }
-    if (lane == 0) scratch[kTkThreads / 32] = v;
+    if (lane == 0) scratch[NT / 32] = v;
   }
   __syncthreads();
-  v = scratch[kTkThreads / 32];
+  v = scratch[NT / 32];
   __syncthreads();
   return v;
 }
 
 // total[i] = sum over the cluster's CTAs of hist[i] (2048 bins), with every
 // remote read of a thread in flight together; ends with a block barrier.
-template <typename Smem>
+template <int NT, typename Smem>
 __device__ __forceinline__ void tk_merge_hist(Smem& sm, cg::cluster_group& cluster, int CS) {
-  constexpr int kPer = kTkBins / kTkThreads;
+  constexpr int kPer = kTkBins / NT;
   uint32_t v[kTkMaxCluster][kPer];
 #pragma unroll
   for (int r = 0; r < kTkMaxCluster; ++r) {
     if (r < CS) {
       const uint32_t* h = cluster.map_shared_rank(sm.hist, r);
 #pragma unroll
-      for (int j = 0; j < kPer; ++j) v[r][j] = h[threadIdx.x + j * kTkThreads];
+      for (int j = 0; j < kPer; ++j) v[r][j] = h[threadIdx.x + j * NT];
     }
   }
 #pragma unroll
@@ -156,34 +160,35 @@ __device__ __forceinline__ void tk_merge_hist(Smem& sm, cg::cluster_group& clust
 #pragma unroll
     for (int r = 0; r < kTkMaxCluster; ++r)
       if (r < CS) t += v[r][j];
-    sm.total[threadIdx.x + j * kTkThreads] = t;
+    sm.total[threadIdx.x + j * NT] = t;
   }
   __syncthreads();
 }
 
 // Finds the threshold digit of one radix pass: thread t owns the
-// kTkBinsPerThr bins from kTkBinsPerThr * t of `h` (2048 bins); the digit is
+// (kTkBins / NT) bins from (kTkBins / NT) * t of `h` (2048 bins); the digit is
 // the bin where the count of keys in it and all higher bins first reaches
 // `remaining`. Returns (digit, remaining within it) through found[0..1] and
 // the count of the digit's bin through the return value.
+template <int NT>
 __device__ __forceinline__ uint32_t tk_find_digit(const uint32_t* h, uint32_t remaining, uint32_t* red,
                                                   uint32_t* found) {
   const int tid = threadIdx.x;
-  uint32_t c[kTkBinsPerThr], mine = 0;
+  uint32_t c[(kTkBins / NT)], mine = 0;
 #pragma unroll
-  for (int i = 0; i < kTkBinsPerThr; ++i) {
-    c[i] = h[kTkBinsPerThr * tid + i];
+  for (int i = 0; i < (kTkBins / NT); ++i) {
+    c[i] = h[(kTkBins / NT) * tid + i];
     mine += c[i];
   }
   uint32_t all;
-  const uint32_t before = tk_block_excl_scan(mine, red, &all);  // keys in lower bins
+  const uint32_t before = tk_block_excl_scan<NT>(mine, red, &all);  // keys in lower bins
   const uint32_t above = all - before - mine;                   // keys in higher bins
   if (above < remaining && above + mine >= remaining) {
     uint32_t acc = above;
 #pragma unroll
-    for (int i = kTkBinsPerThr - 1; i >= 0; --i) {
+    for (int i = (kTkBins / NT) - 1; i >= 0; --i) {
       if (acc < remaining && acc + c[i] >= remaining) {
-        found[0] = static_cast<uint32_t>(kTkBinsPerThr * tid + i);
+        found[0] = static_cast<uint32_t>((kTkBins / NT) * tid + i);
         found[1] = remaining - acc;
       }
       acc += c[i];
@@ -203,8 +208,8 @@ __device__ __forceinline__ uint32_t tk_find_digit(const uint32_t* h, uint32_t re
 // the exact threshold key Tk and how many keys equal to it to take, then
 // writes its own slice's picks in token order at the offset the earlier
 // CTAs' counts give.
-template <int PER>
-__device__ __forceinline__ void topk_digit_path(TopkClusterSmem<PER>& sm, cg::cluster_group& cluster, int CS,
+template <int PER, int NT>
+__device__ __forceinline__ void topk_digit_path(TopkClusterSmem<PER, NT>& sm, cg::cluster_group& cluster, int CS,
                                                 int crank, int row, int b, int k, int s0, int nvalid,
                                                 uint32_t prefix1, uint32_t pmask1, uint32_t need, int32_t* out,
                                                 const RowMap& rm) {
@@ -225,7 +230,7 @@ __device__ __forceinline__ void topk_digit_path(TopkClusterSmem<PER>& sm, cg::cl
     }
   }
   uint32_t tot;
-  const uint32_t pre = tk_block_excl_scan((n_above << 16) | n_d, sm.red, &tot);
+  const uint32_t pre = tk_block_excl_scan<NT>((n_above << 16) | n_d, sm.red, &tot);
   uint32_t pos = pre & 0xffffu;
 #pragma unroll
   for (int j = 0; j < PER; ++j)
@@ -260,7 +265,7 @@ __device__ __forceinline__ void topk_digit_path(TopkClusterSmem<PER>& sm, cg::cl
     for (int r = 0; r < kTkMaxCluster; ++r) {
       if (r < CS) {
         const uint32_t* rk = cluster.map_shared_rank(dkey, r);
-        for (uint32_t i = tid; i < d_r[r]; i += kTkThreads) gkey[off + i] = rk[i];
+        for (uint32_t i = tid; i < d_r[r]; i += NT) gkey[off + i] = rk[i];
       }
       off += d_r[r];
     }
@@ -269,7 +274,7 @@ __device__ __forceinline__ void topk_digit_path(TopkClusterSmem<PER>& sm, cg::cl
   if (tid == 0) SD_PROBE_MARK(2, 10, 0);
   // 2. the exact threshold: key x of D is Tk when fewer than `need` keys of D
   // are above it and at least `need` are at or above it
-  for (uint32_t i = tid; i < cD; i += kTkThreads) {
+  for (uint32_t i = tid; i < cD; i += NT) {
     const uint32_t x = gkey[i];
     uint32_t gt = 0, ge = 0;
     for (uint32_t q = 0; q < cD; ++q) {
@@ -287,12 +292,12 @@ __device__ __forceinline__ void topk_digit_path(TopkClusterSmem<PER>& sm, cg::cl
   const uint32_t Tk = sm.found[0], need_eq = sm.found[1];
   // keys of D in earlier CTAs above / equal to Tk
   uint32_t gtD = 0, eqD = 0;
-  for (uint32_t i = tid; i < base_d; i += kTkThreads) {
+  for (uint32_t i = tid; i < base_d; i += NT) {
     gtD += gkey[i] > Tk;
     eqD += gkey[i] == Tk;
   }
   uint32_t tot2;
-  tk_block_excl_scan((gtD << 16) | eqD, sm.red, &tot2);
+  tk_block_excl_scan<NT>((gtD << 16) | eqD, sm.red, &tot2);
   const uint32_t gt_base = base_above + (tot2 >> 16), eq_base = tot2 & 0xffffu;
   // 3. this slice's picks in token order: every key above Tk, then the first
   // need_eq keys equal to it over the cluster. They fill the output range
@@ -308,7 +313,7 @@ __device__ __forceinline__ void topk_digit_path(TopkClusterSmem<PER>& sm, cg::cl
     }
   }
   uint32_t tot3;
-  const uint32_t pre3 = tk_block_excl_scan((n_gt << 16) | n_eq, sm.red, &tot3);
+  const uint32_t pre3 = tk_block_excl_scan<NT>((n_gt << 16) | n_eq, sm.red, &tot3);
   const uint32_t o0 = gt_base + min(eq_base, need_eq);
   const uint32_t n_out = (tot3 >> 16) + min(eq_base + (tot3 & 0xffffu), need_eq) - min(eq_base, need_eq);
   uint32_t gt_before = gt_base + (pre3 >> 16), eq_before = eq_base + (pre3 & 0xffffu);
@@ -329,11 +334,11 @@ __device__ __forceinline__ void topk_digit_path(TopkClusterSmem<PER>& sm, cg::cl
   }
   __syncthreads();
   if (tid == 0) SD_PROBE_MARK(2, 12, 0);
-  constexpr int kOutPerThr = (kMaxTopK + kTkThreads - 1) / kTkThreads;
+  constexpr int kOutPerThr = (kMaxTopK + NT - 1) / NT;
   int pages[kOutPerThr];
 #pragma unroll
   for (int q = 0; q < kOutPerThr; ++q) {
-    const uint32_t i = tid + q * kTkThreads;
+    const uint32_t i = tid + q * NT;
     pages[q] = -1;
     if (i < n_out) {
       const int tok = static_cast<int>(stage[i]);
@@ -344,11 +349,11 @@ __device__ __forceinline__ void topk_digit_path(TopkClusterSmem<PER>& sm, cg::cl
   if (rm.rows != nullptr) {
 #pragma unroll
     for (int q = 0; q < kOutPerThr; ++q) {
-      const uint32_t i = tid + q * kTkThreads;
+      const uint32_t i = tid + q * NT;
       if (i < n_out) rm.put_page(row, static_cast<int>(o0 + i), static_cast<int>(stage[i]), pages[q]);
     }
     if (crank == 0)
-      for (int i = k + tid; i < rm.kpad; i += kTkThreads) rm.rows[(size_t)row * rm.kpad + i] = -1;
+      for (int i = k + tid; i < rm.kpad; i += NT) rm.rows[(size_t)row * rm.kpad + i] = -1;
   }
   if (tid == 0) SD_PROBE_MARK(2, 5, cD);
 }
@@ -360,8 +365,8 @@ __device__ __forceinline__ void topk_digit_path(TopkClusterSmem<PER>& sm, cg::cl
 // CTA holds its slice's keys in its per-thread chunks. Ends with CTA 0
 // writing the row's output; the other CTAs return after the third cluster
 // barrier.
-template <int PER>
-__device__ __forceinline__ void topk_candidates(TopkClusterSmem<PER>& sm, cg::cluster_group& cluster, int CS,
+template <int PER, int NT>
+__device__ __forceinline__ void topk_candidates(TopkClusterSmem<PER, NT>& sm, cg::cluster_group& cluster, int CS,
                                                 int crank, int row, int b, int k, int s0, int nvalid,
                                                 uint32_t prefix1, uint32_t pmask1, int shift, uint32_t need,
                                                 uint32_t bin_count, int32_t* out, const RowMap& rm) {
@@ -378,7 +383,7 @@ __device__ __forceinline__ void topk_candidates(TopkClusterSmem<PER>& sm, cg::cl
     nc += c;
   }
   uint32_t ctot;
-  uint32_t pos = tk_block_excl_scan(nc, sm.red, &ctot);  // its barriers order every chunk read before the writes
+  uint32_t pos = tk_block_excl_scan<NT>(nc, sm.red, &ctot);  // its barriers order every chunk read before the writes
   uint32_t* ck = sm.keys;               // candidate keys, token order
   uint32_t* ct = sm.keys + kTkCandCap;  // their tokens
 #pragma unroll
@@ -402,7 +407,7 @@ __device__ __forceinline__ void topk_candidates(TopkClusterSmem<PER>& sm, cg::cl
     for (int r = 0; r < kTkMaxCluster; ++r) {
       if (r < CS) {
         const uint32_t* rk = cluster.map_shared_rank(sm.keys, r);
-        for (uint32_t i = tid; i < cnt[r]; i += kTkThreads) {
+        for (uint32_t i = tid; i < cnt[r]; i += NT) {
           gk[off + i] = rk[i];
           gt[off + i] = rk[kTkCandCap + i];
         }
@@ -430,14 +435,14 @@ __device__ __forceinline__ void topk_candidates(TopkClusterSmem<PER>& sm, cg::cl
       const int nbits = min(kTkBinsBits, top + 1);
       const int sh = top + 1 - nbits;
       const uint32_t dmask = (1u << nbits) - 1u;
-      for (int i = tid; i < kTkBins; i += kTkThreads) rh[i] = 0u;
+      for (int i = tid; i < kTkBins; i += NT) rh[i] = 0u;
       __syncthreads();
-      for (uint32_t i = tid; i < nC; i += kTkThreads) {
+      for (uint32_t i = tid; i < nC; i += NT) {
         const uint32_t u = gk[i];
         if ((u & pmask) == prefix) atomicAdd(&rh[(u >> sh) & dmask], 1u);
       }
       __syncthreads();
-      const uint32_t cnt = tk_find_digit(rh, remaining, sm.red, sm.found + 2);
+      const uint32_t cnt = tk_find_digit<NT>(rh, remaining, sm.red, sm.found + 2);
       const uint32_t digit = sm.found[2], rem = sm.found[3];
       __syncthreads();
       prefix |= digit << sh;
@@ -460,7 +465,7 @@ __device__ __forceinline__ void topk_candidates(TopkClusterSmem<PER>& sm, cg::cl
   // 3. ordered output: candidate i is taken if its key is above Tk (every key
   // of a digit above D is), or equal to Tk and among the first need_eq of
   // those in token order; thread t handles kPerThr consecutive candidates
-  constexpr int kPerThr = kTkCandCap / kTkThreads;
+  constexpr int kPerThr = kTkCandCap / NT;
   uint32_t n_gt = 0, n_eq = 0;
 #pragma unroll
   for (int j = 0; j < kPerThr; ++j) {
@@ -472,7 +477,7 @@ __device__ __forceinline__ void topk_candidates(TopkClusterSmem<PER>& sm, cg::cl
     }
   }
   uint32_t tot_packed;
-  const uint32_t pre = tk_block_excl_scan((n_gt << 16) | n_eq, sm.red, &tot_packed);
+  const uint32_t pre = tk_block_excl_scan<NT>((n_gt << 16) | n_eq, sm.red, &tot_packed);
   uint32_t gt_before = pre >> 16, eq_before = pre & 0xffffu;
   if (tid == 0) SD_PROBE_MARK(2, 3, nC);
   // the taken tokens in output order, staged in the free key area (k <= 2048)
@@ -494,11 +499,11 @@ __device__ __forceinline__ void topk_candidates(TopkClusterSmem<PER>& sm, cg::cl
   __syncthreads();
   // coalesced output; the pool rows' block-table loads of a thread are
   // independent of each other, so they are all in flight together
-  constexpr int kOutPerThr = (kMaxTopK + kTkThreads - 1) / kTkThreads;
+  constexpr int kOutPerThr = (kMaxTopK + NT - 1) / NT;
   int pages[kOutPerThr];
 #pragma unroll
   for (int j = 0; j < kOutPerThr; ++j) {
-    const int o = tid + j * kTkThreads;
+    const int o = tid + j * NT;
     pages[j] = -1;
     if (o < k) {
       const int tok = static_cast<int>(sel[o]);
@@ -509,16 +514,16 @@ __device__ __forceinline__ void topk_candidates(TopkClusterSmem<PER>& sm, cg::cl
   if (rm.rows != nullptr) {
 #pragma unroll
     for (int j = 0; j < kOutPerThr; ++j) {
-      const int o = tid + j * kTkThreads;
+      const int o = tid + j * NT;
       if (o < k) rm.put_page(row, o, static_cast<int>(sel[o]), pages[j]);
     }
-    for (int i = k + tid; i < rm.kpad; i += kTkThreads) rm.rows[(size_t)row * rm.kpad + i] = -1;
+    for (int i = k + tid; i < rm.kpad; i += NT) rm.rows[(size_t)row * rm.kpad + i] = -1;
   }
   if (tid == 0) SD_PROBE_MARK(2, 5, nC);
 }
 
-template <int PER>
-__global__ void __launch_bounds__(kTkThreads, 1) topk_cluster_kernel(
+template <int PER, int NT>
+__global__ void __launch_bounds__(NT, kTkMaxThreads / NT) topk_cluster_kernel(
     const int32_t* __restrict__ scores, const int32_t* __restrict__ seqlens, int32_t* __restrict__ indices,
     int G, int max_seqlen, int seqlen_cap, int k, RowMap rm, const int32_t* __restrict__ hint) {
   pdl_wait();  // inputs come from earlier work in the stream
@@ -528,7 +533,7 @@ __global__ void __launch_bounds__(kTkThreads, 1) topk_cluster_kernel(
   constexpr int kTkPerThread = PER;
   constexpr int kTkChunkStride = PER + 1;
   extern __shared__ __align__(16) uint8_t tk_smem_raw[];
-  TopkClusterSmem<PER>& sm = *reinterpret_cast<TopkClusterSmem<PER>*>(tk_smem_raw);
+  TopkClusterSmem<PER, NT>& sm = *reinterpret_cast<TopkClusterSmem<PER, NT>*>(tk_smem_raw);
   cg::cluster_group cluster = cg::this_cluster();
   const int CS = static_cast<int>(cluster.num_blocks());
   const int crank = static_cast<int>(cluster.block_rank());
@@ -541,7 +546,7 @@ __global__ void __launch_bounds__(kTkThreads, 1) topk_cluster_kernel(
 
   if (L <= k) {  // uniform over the cluster: no cluster barrier is reached
     const int n = rm.rows != nullptr ? max(k, rm.kpad) : k;
-    for (int i = crank * kTkThreads + tid; i < n; i += CS * kTkThreads) {
+    for (int i = crank * NT + tid; i < n; i += CS * NT) {
       if (i < k) out[i] = i < L ? i : -1;
       rm.put(row, b, i, i < L ? i : -1, pc);
     }
@@ -549,7 +554,7 @@ __global__ void __launch_bounds__(kTkThreads, 1) topk_cluster_kernel(
   }
 
 
-  const int slice = ceil_div(ceil_div(L, CS), kTkThreads) * kTkThreads;  // <= kTkSlice by launch
+  const int slice = ceil_div(ceil_div(L, CS), NT) * NT;  // <= kTkSlice by launch
   const int s0 = crank * slice;
   const int lim = max(0, min(slice, L - s0));                 // valid elements of this slice
   const int nvalid = max(0, min(kTkPerThread, lim - tid * kTkPerThread));  // in this thread's chunk
@@ -559,7 +564,7 @@ __global__ void __launch_bounds__(kTkThreads, 1) topk_cluster_kernel(
   uint32_t kmin = 0xffffffffu, kmax = 0u;
 #pragma unroll
   for (int j = 0; j < kTkPerThread; ++j) {
-    const int e = j * kTkThreads + tid;           // element within the slice
+    const int e = j * NT + tid;           // element within the slice
     uint32_t u = 0u;                               // past the slice: never read again
     if (e < lim) {
       u = static_cast<uint32_t>(src[s0 + e]) ^ 0x80000000u;
@@ -569,9 +574,9 @@ __global__ void __launch_bounds__(kTkThreads, 1) topk_cluster_kernel(
     sm.keys[(e / kTkPerThread) * kTkChunkStride + (e % kTkPerThread)] = u;
   }
   if (hint != nullptr)
-    for (int i = tid; i < kTkThreads * PER / 32; i += kTkThreads) sm.mark[i] = 0u;
+    for (int i = tid; i < NT * PER / 32; i += NT) sm.mark[i] = 0u;
   if (tid == 0) SD_PROBE_MARK(2, 6, 0);
-  tk_block_minmax(kmin, kmax, sm.red);
+  tk_block_minmax<NT>(kmin, kmax, sm.red);
   if (tid == 0) {
     sm.cta_vals[0] = kmin;
     sm.cta_vals[1] = kmax;
@@ -608,7 +613,7 @@ __global__ void __launch_bounds__(kTkThreads, 1) topk_cluster_kernel(
     const int nbits = min(kTkBinsBits, hb + 1);
     const int shift = hb + 1 - nbits;
     const uint32_t dmask = (1u << nbits) - 1u;
-    for (int i = tid; i < kTkBins; i += kTkThreads) sm.hist[i] = 0u;
+    for (int i = tid; i < kTkBins; i += NT) sm.hist[i] = 0u;
     __syncthreads();
     {
       const uint32_t* chunk = sm.keys + tid * kTkChunkStride;
@@ -616,21 +621,21 @@ __global__ void __launch_bounds__(kTkThreads, 1) topk_cluster_kernel(
     }
     if (tid == 0) SD_PROBE_MARK(2, 7, 0);
     cluster.sync();  // every CTA's histogram is complete
-    tk_merge_hist(sm, cluster, CS);
+    tk_merge_hist<NT>(sm, cluster, CS);
     if (tid == 0) SD_PROBE_MARK(2, 8, 0);
-    const uint32_t bin_count = tk_find_digit(sm.total, static_cast<uint32_t>(k), sm.red, sm.found + 2);
+    const uint32_t bin_count = tk_find_digit<NT>(sm.total, static_cast<uint32_t>(k), sm.red, sm.found + 2);
     const uint32_t digit = sm.found[2], rem = sm.found[3];
     __syncthreads();
     const uint32_t above = static_cast<uint32_t>(k) - rem;
     const uint32_t prefix1 = prefix0 | (digit << shift), pmask1 = pmask0 | (dmask << shift);
     if (bin_count <= static_cast<uint32_t>(kTkDigitCap)) {
       if (threadIdx.x == 0) SD_PROBE_MARK(2, 2, bin_count);
-      topk_digit_path<PER>(sm, cluster, CS, crank, row, b, k, s0, nvalid, prefix1, pmask1, rem, out, rm);
+      topk_digit_path<PER, NT>(sm, cluster, CS, crank, row, b, k, s0, nvalid, prefix1, pmask1, rem, out, rm);
       return;
     }
     if (above + bin_count <= static_cast<uint32_t>(kTkCandCap)) {
       if (threadIdx.x == 0) SD_PROBE_MARK(2, 2, bin_count);
-      topk_candidates<PER>(sm, cluster, CS, crank, row, b, k, s0, nvalid, prefix1, pmask1, shift, rem,
+      topk_candidates<PER, NT>(sm, cluster, CS, crank, row, b, k, s0, nvalid, prefix1, pmask1, shift, rem,
                            bin_count, out, rm);
       return;
     }
@@ -647,7 +652,7 @@ __global__ void __launch_bounds__(kTkThreads, 1) topk_cluster_kernel(
   // taking every key above that range.
   if (hint != nullptr) {
     const int32_t* hr = hint + (size_t)row * k;
-    for (int i = crank * kTkThreads + tid; i < k; i += CS * kTkThreads) {
+    for (int i = crank * NT + tid; i < k; i += CS * NT) {
       const int t = hr[i];
       if (t >= 0 && t < L) {
         const int owner = t / slice, off = t - owner * slice;
@@ -669,10 +674,10 @@ __global__ void __launch_bounds__(kTkThreads, 1) topk_cluster_kernel(
         }
       }
     }
-    lo = tk_block_reduce(lo, sm.red, false);
-    hi = tk_block_reduce(hi, sm.red, true);
+    lo = tk_block_reduce<NT>(lo, sm.red, false);
+    hi = tk_block_reduce<NT>(hi, sm.red, true);
     uint32_t np_tot;
-    tk_block_excl_scan(np, sm.red, &np_tot);
+    tk_block_excl_scan<NT>(np, sm.red, &np_tot);
     if (tid == 0) {
       sm.hvals[0] = lo;
       sm.hvals[1] = hi;
@@ -709,7 +714,7 @@ __global__ void __launch_bounds__(kTkThreads, 1) topk_cluster_kernel(
       const uint32_t* chunk = sm.keys + tid * kTkChunkStride;
       for (int j = 0; j < nvalid; ++j) above += chunk[j] > x;
       uint32_t above_cta;
-      tk_block_excl_scan(above, sm.red, &above_cta);
+      tk_block_excl_scan<NT>(above, sm.red, &above_cta);
       if (tid == 0) sm.hvals[3] = above_cta;
       cluster.sync();
       if (tid < 32) {
@@ -746,7 +751,7 @@ __global__ void __launch_bounds__(kTkThreads, 1) topk_cluster_kernel(
       const int nbits = min(kTkBinsBits, top + 1);
       const int shift = top + 1 - nbits;
       const uint32_t dmask = (1u << nbits) - 1u;
-      for (int i = tid; i < kTkBins; i += kTkThreads) sm.hist[i] = 0u;
+      for (int i = tid; i < kTkBins; i += NT) sm.hist[i] = 0u;
       __syncthreads();
       const uint32_t* chunk = sm.keys + tid * kTkChunkStride;
       for (int j = 0; j < nvalid; ++j) {
@@ -754,11 +759,11 @@ __global__ void __launch_bounds__(kTkThreads, 1) topk_cluster_kernel(
         if ((u & pmask) == prefix && u <= hi_cut) atomicAdd(&sm.hist[(u >> shift) & dmask], 1u);
       }
       cluster.sync();  // every CTA's histogram is complete
-      tk_merge_hist(sm, cluster, CS);
+      tk_merge_hist<NT>(sm, cluster, CS);
       cluster.sync();  // nobody rewrites its histogram before all have read it
       // the digit where the count of keys with a larger-or-equal digit first
       // reaches `remaining`
-      const uint32_t bin_count = tk_find_digit(sm.total, remaining, sm.red, sm.found);
+      const uint32_t bin_count = tk_find_digit<NT>(sm.total, remaining, sm.red, sm.found);
       const uint32_t digit = sm.found[0];
       const uint32_t rem = sm.found[1];
       __syncthreads();
@@ -789,7 +794,7 @@ __global__ void __launch_bounds__(kTkThreads, 1) topk_cluster_kernel(
     n_eq += u == T;
   }
   uint32_t tot_packed;
-  const uint32_t pre = tk_block_excl_scan((n_gt << 16) | n_eq, sm.red, &tot_packed);
+  const uint32_t pre = tk_block_excl_scan<NT>((n_gt << 16) | n_eq, sm.red, &tot_packed);
   if (tid == 0) {
     sm.cta_vals[2] = tot_packed >> 16;
     sm.cta_vals[3] = tot_packed & 0xffffu;
@@ -819,14 +824,14 @@ __global__ void __launch_bounds__(kTkThreads, 1) topk_cluster_kernel(
   // optional row ids: a separate pass over the finished output (written by
   // the whole cluster before the barrier), one block-table load per page run
   if (rm.rows != nullptr)
-    for (int i = crank * kTkThreads + tid; i < rm.kpad; i += CS * kTkThreads) rm.put(row, b, i, i < k ? out[i] : -1, pc);
+    for (int i = crank * NT + tid; i < rm.kpad; i += CS * NT) rm.put(row, b, i, i < k ? out[i] : -1, pc);
   if (threadIdx.x == 0) SD_PROBE_MARK(2, 4, 0);
 }
 
 // Cluster size for rows of up to max_seqlen scores with PER scores per thread
 // (0: does not fit in kTkMaxCluster CTAs).
-inline int topk_cluster_size(int max_seqlen, int per) {
-  const long long slice = (long long)kTkThreads * per;
+inline int topk_cluster_size(int max_seqlen, int per, int nt) {
+  const long long slice = (long long)nt * per;
   int cs = 1;
   while (cs < kTkMaxCluster && cs * slice < max_seqlen) cs <<= 1;
   return cs * slice >= max_seqlen ? cs : 0;
